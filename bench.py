@@ -1,0 +1,490 @@
+"""Benchmark of the Beam 1.0 attention core on B200.
+
+One step = the prefill of one local and one global attention layer of the
+batched-prefill workload (4 sequences x 8192 tokens, 48 query / 8 KV heads,
+head_dim 128), including the fused KV-cache append, through the C ABI.  The
+headline value is algorithmic TFLOP/s (visible (query, key) pairs x 4 x 128 x 48).
+Two decode measurements ride along on the same line: the 1M-context decode step
+across the 52-layer schedule (KV-read GB/s, tokens/s) and the batched decode step
+(64 sequences, contexts in [1024, 32768]).
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl beam|reference]
+N > 1 runs under torch.distributed.run, one process per GPU; every rank processes
+its own batch (weak scaling, no collective on the data path); the time is the
+max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+METRIC = "prefill TFLOP/s (% bf16 peak); decode KV-read GB/s and tokens/s at 1M ctx"
+HEAD_FLOPS_PER_PAIR = 4 * wl.HEAD_DIM * wl.N_Q_HEADS   # QK^T and PV, all query heads
+
+
+def prefill_flops(B: int, T: int, kind: int, window: int = wl.WINDOW) -> int:
+    pairs = wl.visible_pairs(T, window if kind == wl.LOCAL else None)
+    return B * pairs * HEAD_FLOPS_PER_PAIR
+
+
+def decode_kv_bytes(ctx, kind: int, window: int = wl.WINDOW) -> int:
+    """Algorithmic bytes of one decode layer: the visible K and V rows (4 KiB per
+    token per layer) plus the new token's q, k, v, gate and output."""
+    vis = sum(min(c, window) if kind == wl.LOCAL else c for c in ctx)
+    per_token = 2 * wl.N_KV_HEADS * wl.HEAD_DIM * 2
+    io = len(ctx) * 2 * (3 * wl.N_Q_HEADS * wl.HEAD_DIM + 2 * wl.N_KV_HEADS * wl.HEAD_DIM)
+    return vis * per_token + io
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+# ------------------------------------------------------------------ distributed helpers
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), \
+        int(os.environ.get("LOCAL_RANK", 0))
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(per_rank_units: float, world: int, seconds_max: float) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time."""
+    return per_rank_units * world / seconds_max
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.rows = []
+        self._stop = threading.Event()
+        self._th = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                out = subprocess.run(
+                    ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                     "--format=csv,noheader,nounits"], capture_output=True, text=True, timeout=5)
+                if out.returncode == 0 and out.stdout.strip():
+                    self.rows.append([x.strip() for x in out.stdout.strip().split(",")])
+            except Exception:
+                pass
+            self._stop.wait(0.2)
+
+    def __enter__(self):
+        self._th = threading.Thread(target=self._run, daemon=True)
+        self._th.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        self._th.join(timeout=10)
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[0]) for r in self.rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in self.rows for n, v in zip(names, r[4:8]) if v == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(self.rows)}
+
+
+# ------------------------------------------------------------------ GPU arm
+class PrefillLayer:
+    """Device buffers of one prefill layer call (inputs drawn on the device)."""
+
+    def __init__(self, torch, beam, kind, B, T, seed, tag):
+        self.torch, self.beam, self.kind, self.B, self.T = torch, beam, kind, B, T
+        self.params = beam.default_params()
+        dev = "cuda"
+        self.x = {}
+        for name, width in (("q", 6144), ("k", 1024), ("v", 1024), ("gate", 6144)):
+            t = torch.empty((B, T, width), dtype=torch.bfloat16, device=dev)
+            wl.device_normal_bf16_(t, seed, f"{tag}/{name}")
+            self.x[name] = t
+        inp = wl.prefill_inputs(1, 1, seed, layer=tag)
+        self.qw = torch.from_numpy(inp.q_norm_w).to(dev)
+        self.kw = torch.from_numpy(inp.k_norm_w).to(dev)
+        self.bias = torch.from_numpy(inp.gate_bias).to(dev)
+        self.out = torch.empty_like(self.x["q"])
+        self.layout = beam.beam_kv_layout(kind, self.params, B, T)
+        self.kc = torch.empty(self.layout.bytes_k // 2, dtype=torch.bfloat16, device=dev)
+        self.vc = torch.empty_like(self.kc)
+        self.ws = torch.empty(beam.beam_prefill_workspace_bytes(self.params, B, T),
+                              dtype=torch.uint8, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def run(self, x=None, out=None):
+        x = x or self.x
+        self.beam.beam_attn_prefill(self.kind, self.params, x["q"], x["k"], x["v"], x["gate"],
+                                    self.qw, self.kw, self.bias, out if out is not None else self.out,
+                                    self.kc, self.vc, self.layout, workspace=self.ws,
+                                    dev_status=self.status)
+
+    launches_per_call = 2  # prologue + attention
+
+
+class DecodeLayer:
+    def __init__(self, torch, beam, kind, ctx, slots, seed, tag, cache=None):
+        self.torch, self.beam, self.kind = torch, beam, kind
+        self.params = beam.default_params()
+        dev = "cuda"
+        ctx = np.asarray(ctx, np.int64)
+        self.B = len(ctx)
+        di = wl.decode_inputs(kind, ctx, slots, seed, layer=tag, with_cache=False)
+
+        def d(bits):
+            return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+        self.q, self.k, self.v, self.gate = d(di.q), d(di.k), d(di.v), d(di.gate)
+        self.qw = torch.from_numpy(di.q_norm_w).to(dev)
+        self.kw = torch.from_numpy(di.k_norm_w).to(dev)
+        self.bias = torch.from_numpy(di.gate_bias).to(dev)
+        self.pos = torch.from_numpy(di.pos).to(dev)
+        self.layout = beam.beam_kv_layout(kind, self.params, self.B, slots)
+        if cache is None:
+            self.kc = torch.empty(self.layout.bytes_k // 2, dtype=torch.bfloat16, device=dev)
+            self.vc = torch.empty_like(self.kc)
+            wl.device_normal_bf16_(self.kc, seed, f"{tag}/kc")
+            wl.device_normal_bf16_(self.vc, seed, f"{tag}/vc")
+        else:
+            self.kc, self.vc = cache
+        self.out = torch.empty((self.B, 6144), dtype=torch.bfloat16, device=dev)
+        self.ws = torch.empty(max(16, beam.beam_decode_workspace_bytes(kind, self.params, self.B,
+                                                                      self.layout)),
+                              dtype=torch.uint8, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.bytes = decode_kv_bytes(ctx, kind)
+
+    def run(self):
+        self.beam.beam_attn_decode(self.kind, self.params, self.q, self.k, self.v, self.gate,
+                                   self.qw, self.kw, self.bias, self.pos, self.kc, self.vc,
+                                   self.layout, self.out, workspace=self.ws, dev_status=self.status)
+
+    launches_per_call = 3  # prologue + split-K + combine
+
+
+def time_loop(torch, fn, steps, warmup):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ev[0].record()
+    for _ in range(steps):
+        fn()
+    ev[1].record()
+    torch.cuda.synchronize()
+    return ev[0].elapsed_time(ev[1]) / 1e3 / steps
+
+
+def bench_decode_1m(torch, beam, steps, warmup, seed):
+    """52-layer decode step at context 1,048,576: 9 global layers with 4 GiB caches,
+    43 local rings; the whole step is one CUDA graph replay."""
+    layers = []
+    ring_cache = None
+    for i in range(1, wl.N_LAYERS + 1):
+        kind = wl.layer_kind(i)
+        if kind == wl.GLOBAL:
+            layers.append(DecodeLayer(torch, beam, kind, [wl.MAX_CONTEXT], wl.MAX_CONTEXT, seed,
+                                      f"d1m/L{i}"))
+        else:
+            layers.append(DecodeLayer(torch, beam, kind, [wl.MAX_CONTEXT], wl.WINDOW, seed,
+                                      f"d1m/L{i}"))
+    del ring_cache
+    total_bytes = sum(L.bytes for L in layers)
+    glob_bytes = sum(L.bytes for L in layers if L.kind == wl.GLOBAL)
+
+    def step():
+        for L in layers:
+            L.run()
+
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        step()  # warm the launch path outside capture
+    torch.cuda.current_stream().wait_stream(stream)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    sec = time_loop(torch, graph.replay, steps, warmup)
+    # the dominant kernel: one global layer's decode call timed alone
+    g0 = next(L for L in layers if L.kind == wl.GLOBAL)
+    sec_g = time_loop(torch, g0.run, steps * 4, warmup)
+    status = [int(L.status.item()) for L in layers]
+    assert all(s == 0 for s in status), status
+    res = {
+        "workload": "decode_1m: B=1, context 1048576, 52 layers (9 global 4 GiB caches, 43 x 512-slot rings)",
+        "ms_per_token": sec * 1e3,
+        "tokens_per_s": 1.0 / sec,
+        "kv_read_GBps": total_bytes / sec / 1e9,
+        "bytes_per_step": total_bytes,
+        "global_layer_GBps": g0.bytes / sec_g / 1e9,
+        "global_layer_ms": sec_g * 1e3,
+        "gpu_launches_per_step": sum(L.launches_per_call for L in layers),
+    }
+    del graph, layers
+    torch.cuda.empty_cache()
+    return res, glob_bytes
+
+
+def bench_decode_batched(torch, beam, steps, warmup, seed):
+    w = wl.workload("batched_decode", seed)
+    g = DecodeLayer(torch, beam, wl.GLOBAL, w.ctx, w.extra["global_slots"], seed, "bdec/g")
+    l = DecodeLayer(torch, beam, wl.LOCAL, w.ctx, wl.WINDOW, seed, "bdec/l")
+
+    def step():
+        g.run()
+        l.run()
+    sec = time_loop(torch, step, steps * 4, warmup)
+    res = {
+        "workload": "batched_decode: 64 sequences, contexts U[1024,32768], one global + one local layer",
+        "ms_per_step": sec * 1e3,
+        "tokens_per_s": w.B / sec,
+        "kv_read_GBps": (g.bytes + l.bytes) / sec / 1e9,
+    }
+    del g, l
+    torch.cuda.empty_cache()
+    return res
+
+
+_CPU_INPUTS = {}
+
+
+def cpu_baseline_prefill(seconds_target=10.0, seconds_cap=30.0, seed=1234):
+    """The fp64 oracle, as it stands, on a bounded row sample of the batched-prefill
+    workload (global layer: rows drawn uniformly from 0..8191 of 4 sequences, all 48
+    heads).  Returns TFLOP/s of algorithmic work and the sample description."""
+    import oracle
+    P = oracle.params()
+    B, T = 4, 8192
+    key = (B, T, seed)
+    if key not in _CPU_INPUTS:
+        _CPU_INPUTS.clear()
+        _CPU_INPUTS[key] = wl.prefill_inputs(B, T, seed, layer="cpu")
+    inp = _CPU_INPUTS[key]
+    rng = np.random.default_rng(seed)
+    threads = oracle.n_threads_default()
+    done_flops, done_rows, t0 = 0, 0, time.perf_counter()
+    batch = max(8, threads)
+    while True:
+        rb = rng.integers(0, B, size=batch)
+        rt = rng.integers(0, T, size=batch)
+        oracle.prefill_rows(oracle.GLOBAL, P, inp.q, inp.k, inp.v, inp.gate, inp.q_norm_w,
+                            inp.k_norm_w, inp.gate_bias, rb, rt, n_threads=threads)
+        done_flops += int((rt + 1).sum()) * HEAD_FLOPS_PER_PAIR
+        done_rows += batch
+        el = time.perf_counter() - t0
+        if el >= seconds_target or el >= seconds_cap:
+            break
+    return {"value": done_flops / el / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"{done_rows} query rows x 48 heads of the global layer of batched_prefill "
+                      f"(B=4, T=8192), uniform row positions; {el:.1f} s"}
+
+
+def e2e_prefill(torch, beam, layers, steps, warmup):
+    """Same metric through the public call with pinned host buffers: each step copies
+    the step's inputs host->device and reads the outputs back."""
+    host_in = []
+    for L in layers:
+        host_in.append({k: v.cpu().pin_memory() for k, v in L.x.items()})
+    host_out = [torch.empty(L.out.shape, dtype=L.out.dtype, pin_memory=True) for L in layers]
+    dev_in = [{k: torch.empty_like(v) for k, v in L.x.items()} for L in layers]
+    h2d = sum(v.numel() * v.element_size() for d in host_in for v in d.values())
+    d2h = sum(o.numel() * o.element_size() for o in host_out)
+
+    def step():
+        for L, hi, di, ho in zip(layers, host_in, dev_in, host_out):
+            for k in hi:
+                di[k].copy_(hi[k], non_blocking=True)
+            L.run(di)
+            ho.copy_(L.out, non_blocking=True)
+    sec = time_loop(torch, step, max(1, steps // 2), max(1, warmup // 2))
+    return sec, h2d, d2h
+
+
+def run_gpu(args):
+    import torch
+    rank, world, local_rank = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    import global_nope_gqa_b200 as beam
+    beam.lib()
+    pk = peaks()
+    w = wl.workload("batched_prefill", args.seed + rank)
+    layers = [PrefillLayer(torch, beam, kind, w.B, w.T, w.seed, f"bench/{kind}")
+              for kind in (wl.LOCAL, wl.GLOBAL)]
+    flops_step = sum(prefill_flops(w.B, w.T, L.kind) for L in layers)
+
+    def step():
+        for L in layers:
+            L.run()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    # per-call events on the launching stream for the dominant (global) layer
+    stream = torch.cuda.current_stream()
+    ev_step = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ev_g = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        ev_step[0].record(stream)
+        for i in range(args.steps):
+            layers[0].run()
+            ev_g[i][0].record(stream)
+            layers[1].run()
+            ev_g[i][1].record(stream)
+        ev_step[1].record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    sec = ev_step[0].elapsed_time(ev_step[1]) / 1e3 / args.steps
+    sec_g = sum(a.elapsed_time(b) for a, b in ev_g) / 1e3 / args.steps
+    sec_max = max_over_ranks(sec, "cuda")
+    value = aggregate(flops_step, world, sec_max) / 1e12
+    for L in layers:
+        assert int(L.status.item()) == 0, "device status set during the bench"
+
+    g_flops = prefill_flops(w.B, w.T, wl.GLOBAL)
+    achieved = g_flops / sec_g / 1e12
+    e2e_sec, h2d, d2h = e2e_prefill(torch, beam, layers, args.steps, args.warmup)
+    e2e_sec = max_over_ranks(e2e_sec, "cuda")
+    result = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(sec_max * 1e3, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic: N(0,1) bf16 activations drawn on the device (seeded torch Philox)",
+        "config": {"workload": "batched_prefill: B=4, T=8192 per GPU, one local (window 512, RoPE) "
+                               "+ one global (NoPE, SSMax) layer, 48 q / 8 kv heads, d=128, "
+                               "fused KV append",
+                   "global_batch": w.B * world, "seq_len": w.T, "parallelism": f"dp{world}",
+                   "l2": "inputs larger than L2 (Q alone is 403 MB per layer)"},
+        "pct_of_bf16_peak": round(100 * value / world / pk["bf16_tflops"], 2),
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": pk["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": round(achieved / pk["bf16_tflops"], 4),
+                     "traffic": None, "kernel": "global-layer prefill call (prologue + attention)",
+                     "peak_source": pk["source"] + " burst bf16"},
+        "e2e": {"value": round(aggregate(flops_step, world, e2e_sec) / 1e12, 3), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps * sum(L.launches_per_call for L in layers),
+        "clocks": clocks.summary(),
+    }
+    del layers
+    torch.cuda.empty_cache()
+    if rank == 0 and not args.no_decode:
+        d1m, _ = bench_decode_1m(torch, beam, args.steps, args.warmup, args.seed)
+        d1m["pct_of_hbm"] = round(100 * d1m["kv_read_GBps"] / pk["hbm_gbs"], 2)
+        result["decode_1m"] = d1m
+        db = bench_decode_batched(torch, beam, args.steps, args.warmup, args.seed)
+        db["pct_of_hbm"] = round(100 * db["kv_read_GBps"] / pk["hbm_gbs"], 2)
+        result["decode_batched"] = db
+    if rank == 0 and world == 1 and not args.no_cpu:
+        result["cpu_baseline"] = cpu_baseline_prefill(seed=args.seed)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    per_step = []
+    base = None
+    for i in range(args.warmup + args.steps):
+        b = cpu_baseline_prefill(seconds_target=3.0, seconds_cap=20.0, seed=args.seed)
+        if i >= args.warmup:
+            per_step.append(b)
+        base = b
+    value = statistics.mean(x["value"] for x in per_step)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic: N(0,1) bf16 activations (seeded numpy Philox)",
+        "config": {"workload": "batched_prefill: B=4, T=8192, global layer row sample",
+                   "global_batch": 4, "seq_len": 8192, "parallelism": "none (host cores)"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": base["cores"],
+                         "kind": "oracle", "sample": base["sample"]},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="beam", choices=["beam", "reference"])
+    ap.add_argument("--seed", type=int, default=1234)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

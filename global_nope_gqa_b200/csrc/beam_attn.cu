@@ -1,0 +1,388 @@
+// beam_attn.cu -- the C ABI of the attention core (declared in beam_attn.h):
+// host-side validation, workspace carving and kernel launches.
+//
+// Every call validates its arguments on the host and returns before any launch
+// when they are wrong; kernels are launched on the caller's stream and the call
+// returns without synchronising.  Nothing here allocates device memory.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "beam_attn.h"
+#include "common.cuh"
+#include "decode.cuh"
+#include "prefill_mma.cuh"
+#include "prologue.cuh"
+
+using namespace beam;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  int sm_count = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+
+// Per-device attributes: SM count and the dynamic shared-memory opt-ins.
+int device_info(DeviceInfo **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BEAM_ERR_CUDA;
+  DeviceInfo &d = g_dev[dev];
+  if (!d.ready) {
+    if (cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return BEAM_ERR_CUDA;
+    if (cudaFuncSetAttribute(decode_splitk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kDecSmem) != cudaSuccess)
+      return BEAM_ERR_CUDA;
+    if (cudaFuncSetAttribute(prefill_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kPfSmem) != cudaSuccess)
+      return BEAM_ERR_CUDA;
+    d.ready = true;
+  }
+  *out = &d;
+  return BEAM_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int check_params(int kind, const beam_attn_params *p) {
+  if (!p) return BEAM_ERR_INVALID_ARG;
+  if (kind != BEAM_LOCAL && kind != BEAM_GLOBAL) return BEAM_ERR_INVALID_ARG;
+  if (p->n_q_heads != kHq || p->n_kv_heads != kHkv || p->head_dim != kD)
+    return BEAM_ERR_UNSUPPORTED;
+  if (p->window < 1) return BEAM_ERR_INVALID_ARG;
+  if (!(p->rms_eps >= 0.f) || !(p->ssmax_base > 0.f) || !(p->rope_theta > 0.f) ||
+      !std::isfinite(p->softmax_scale) || !std::isfinite(p->ssmax_exp))
+    return BEAM_ERR_INVALID_ARG;
+  return BEAM_OK;
+}
+
+int check_layout(int kind, const beam_attn_params *p, const beam_kv_layout_t *L) {
+  if (!L) return BEAM_ERR_INVALID_ARG;
+  if (L->slots_per_seq < 1 || L->stride_slot != kD) return BEAM_ERR_INVALID_ARG;
+  if (L->stride_head < L->slots_per_seq * kD || L->stride_seq < kHkv * L->stride_head)
+    return BEAM_ERR_INVALID_ARG;
+  if ((L->stride_head % 8) || (L->stride_seq % 8)) return BEAM_ERR_ALIGNMENT;
+  if (kind == BEAM_LOCAL && L->slots_per_seq != p->window) return BEAM_ERR_INVALID_ARG;
+  return BEAM_OK;
+}
+
+void fill_inv_freq(double (&f)[64], double theta) {
+  for (int i = 0; i < 64; ++i) f[i] = std::pow(theta, -2.0 * i / (double)kD);
+}
+
+int launch_status() { return cudaGetLastError() == cudaSuccess ? BEAM_OK : BEAM_ERR_CUDA; }
+
+// Decode split size: cache slots per CTA.  A local ring is one split; a global
+// cache is cut so that the grid holds several waves of the SMs at its largest
+// context, in runs of at least 512 slots (the partial results are then well
+// under 1% of the bytes streamed).
+int decode_split(int kind, const beam_attn_params *p, int32_t B, int64_t slots, int sm_count) {
+  if (kind == BEAM_LOCAL) return (int)round_up((size_t)p->window, kDecTile);
+  const int64_t target_ctas = (int64_t)sm_count * 2 * 8;  // ~8 waves at 2 CTAs per SM
+  int64_t split = 512;
+  while (split < 16384 && (int64_t)B * kHkv * ((slots + split - 1) / split) > target_ctas)
+    split *= 2;
+  return (int)split;
+}
+
+struct DecodeWorkspace {
+  uint16_t *qn;
+  float *part_o;
+  float *part_ml;
+  size_t bytes;
+};
+
+DecodeWorkspace decode_workspace(void *base, int32_t B, int n_split_max) {
+  DecodeWorkspace w;
+  uint8_t *p = static_cast<uint8_t *>(base);
+  size_t off = 0;
+  w.qn = reinterpret_cast<uint16_t *>(p + off);
+  off += round_up((size_t)B * kHq * kD * 2, 256);
+  w.part_o = reinterpret_cast<float *>(p + off);
+  off += round_up((size_t)B * kHkv * n_split_max * kGroup * kD * 4, 256);
+  w.part_ml = reinterpret_cast<float *>(p + off);
+  off += round_up((size_t)B * kHkv * n_split_max * kGroup * 2 * 4, 256);
+  w.bytes = off;
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+void beam_default_params(beam_attn_params *p) {
+  if (!p) return;
+  p->n_q_heads = kHq;
+  p->n_kv_heads = kHkv;
+  p->head_dim = kD;
+  p->window = 512;
+  p->rope_theta = 10000.f;
+  p->rms_eps = 1e-6f;
+  p->ssmax_base = 2048.f;
+  p->ssmax_exp = 0.1f;
+  p->softmax_scale = (float)(1.0 / std::sqrt(128.0));
+}
+
+int beam_kv_layout(int kind, const beam_attn_params *p, int32_t batch, int64_t capacity_tokens,
+                   beam_kv_layout_t *out) {
+  int st = check_params(kind, p);
+  if (st) return st;
+  if (!out || batch < 0) return BEAM_ERR_INVALID_ARG;
+  const int64_t slots = kind == BEAM_LOCAL ? (int64_t)p->window : capacity_tokens;
+  if (slots < 1) return BEAM_ERR_INVALID_ARG;
+  out->slots_per_seq = slots;
+  out->stride_slot = kD;
+  out->stride_head = slots * kD;
+  out->stride_seq = (int64_t)kHkv * slots * kD;
+  out->bytes_k = (int64_t)batch * out->stride_seq * 2;
+  out->bytes_v = out->bytes_k;
+  return BEAM_OK;
+}
+
+size_t beam_prefill_workspace_bytes(const beam_attn_params *p, int32_t B, int32_t T) {
+  (void)p;
+  if (B <= 0 || T <= 0) return 0;
+  const size_t tok = (size_t)B * T;
+  return round_up(tok * kHq * kD * 2, 256) + round_up(tok * kHkv * kD * 2, 256);
+}
+
+int beam_attn_prefill(int kind, const beam_attn_params *p, int32_t B, int32_t T, const void *q,
+                      const void *k, const void *v, const void *gate, const float *q_norm_w,
+                      const float *k_norm_w, const float *gate_bias, void *out, void *k_cache,
+                      void *v_cache, const beam_kv_layout_t *layout, void *workspace,
+                      size_t workspace_bytes, int32_t *dev_status, beam_stream_t stream) {
+  int st = check_params(kind, p);
+  if (st) return st;
+  if (B < 0 || T < 0) return BEAM_ERR_INVALID_ARG;
+  if (B == 0 || T == 0) return BEAM_OK;
+  if (!q || !k || !v || !gate || !q_norm_w || !k_norm_w || !gate_bias || !out)
+    return BEAM_ERR_INVALID_ARG;
+  if ((k_cache == nullptr) != (v_cache == nullptr)) return BEAM_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(gate) || !aligned16(out) ||
+      !aligned16(q_norm_w) || !aligned16(k_norm_w) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      !aligned16(workspace))
+    return BEAM_ERR_ALIGNMENT;
+  if (k_cache) {
+    st = check_layout(kind, p, layout);
+    if (st) return st;
+    if (kind == BEAM_GLOBAL && layout->slots_per_seq < T) return BEAM_ERR_CAPACITY;
+  }
+  const size_t need = beam_prefill_workspace_bytes(p, B, T);
+  if (!workspace || workspace_bytes < need) return BEAM_ERR_WORKSPACE;
+  if ((int64_t)B * T > INT32_MAX) return BEAM_ERR_UNSUPPORTED;
+  DeviceInfo *dev = nullptr;
+  if ((st = device_info(&dev))) return st;
+
+  const size_t tok = (size_t)B * T;
+  uint16_t *qn = static_cast<uint16_t *>(workspace);
+  uint16_t *kn = reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(workspace) +
+                                              round_up(tok * kHq * kD * 2, 256));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+  PrologueArgs pa;
+  memset(&pa, 0, sizeof pa);
+  pa.q = static_cast<const uint16_t *>(q);
+  pa.k = static_cast<const uint16_t *>(k);
+  pa.v = static_cast<const uint16_t *>(v);
+  pa.qw = q_norm_w;
+  pa.kw = k_norm_w;
+  pa.q_out = qn;
+  pa.k_out = kn;
+  pa.k_cache = static_cast<uint16_t *>(k_cache);
+  pa.v_cache = static_cast<uint16_t *>(v_cache);
+  if (k_cache) {
+    pa.stride_seq = layout->stride_seq;
+    pa.stride_head = layout->stride_head;
+    pa.slots = layout->slots_per_seq;
+  }
+  pa.pos0 = nullptr;
+  pa.status = dev_status;
+  pa.T = T;
+  pa.kind = kind;
+  pa.window = p->window;
+  pa.eps = p->rms_eps;
+  fill_inv_freq(pa.inv_freq, p->rope_theta);
+  prologue_kernel<<<(unsigned)tok, 128, 0, s>>>(pa);
+  if ((st = launch_status())) return st;
+
+  PrefillArgs fa;
+  fa.qn = qn;
+  fa.kn = kn;
+  fa.v = static_cast<const uint16_t *>(v);
+  fa.gate = static_cast<const uint16_t *>(gate);
+  fa.gate_bias = gate_bias;
+  fa.out = static_cast<uint16_t *>(out);
+  fa.T = T;
+  fa.kind = kind;
+  fa.window = p->window;
+  fa.n_qblocks = (T + kPfBM - 1) / kPfBM;
+  fa.scale_log2 = p->softmax_scale * kLog2e;
+  fa.ssmax_base = p->ssmax_base;
+  fa.ssmax_exp = p->ssmax_exp;
+  dim3 grid(fa.n_qblocks, kHq, B);
+  prefill_mma_kernel<<<grid, kPfThreads, kPfSmem, s>>>(fa);
+  return launch_status();
+}
+
+int beam_kv_append(int kind, const beam_attn_params *p, int32_t B, int32_t T, const void *k,
+                   const void *v, const float *k_norm_w, const int64_t *pos0, void *k_cache,
+                   void *v_cache, const beam_kv_layout_t *layout, int32_t *dev_status,
+                   beam_stream_t stream) {
+  int st = check_params(kind, p);
+  if (st) return st;
+  if (B < 0 || T < 0) return BEAM_ERR_INVALID_ARG;
+  if (B == 0 || T == 0) return BEAM_OK;
+  if (!k || !v || !k_norm_w || !pos0 || !k_cache || !v_cache) return BEAM_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_norm_w) || !aligned16(k_cache) ||
+      !aligned16(v_cache) || (reinterpret_cast<uintptr_t>(pos0) & 7u))
+    return BEAM_ERR_ALIGNMENT;
+  if ((st = check_layout(kind, p, layout))) return st;
+  if ((int64_t)B * T > INT32_MAX) return BEAM_ERR_UNSUPPORTED;
+  DeviceInfo *dev = nullptr;
+  if ((st = device_info(&dev))) return st;
+  PrologueArgs pa;
+  memset(&pa, 0, sizeof pa);
+  pa.k = static_cast<const uint16_t *>(k);
+  pa.v = static_cast<const uint16_t *>(v);
+  pa.qw = k_norm_w;  // unused: no query rows
+  pa.kw = k_norm_w;
+  pa.k_cache = static_cast<uint16_t *>(k_cache);
+  pa.v_cache = static_cast<uint16_t *>(v_cache);
+  pa.stride_seq = layout->stride_seq;
+  pa.stride_head = layout->stride_head;
+  pa.slots = layout->slots_per_seq;
+  pa.pos0 = pos0;
+  pa.status = dev_status;
+  pa.T = T;
+  pa.kind = kind;
+  pa.window = p->window;
+  pa.eps = p->rms_eps;
+  fill_inv_freq(pa.inv_freq, p->rope_theta);
+  prologue_kernel<<<(unsigned)((size_t)B * T), 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(pa);
+  return launch_status();
+}
+
+size_t beam_decode_workspace_bytes(int kind, const beam_attn_params *p, int32_t B,
+                                   const beam_kv_layout_t *layout) {
+  if (check_params(kind, p) || !layout || B <= 0 || layout->slots_per_seq < 1) return 0;
+  DeviceInfo *dev = nullptr;
+  int sm = 148;
+  if (device_info(&dev) == BEAM_OK) sm = dev->sm_count;
+  const int split = decode_split(kind, p, B, layout->slots_per_seq, sm);
+  const int64_t vis_max = kind == BEAM_LOCAL ? p->window : layout->slots_per_seq;
+  const int n_split_max = (int)((vis_max + split - 1) / split);
+  return decode_workspace(nullptr, B, n_split_max).bytes;
+}
+
+int beam_attn_decode(int kind, const beam_attn_params *p, int32_t B, const void *q, const void *k,
+                     const void *v, const void *gate, const float *q_norm_w,
+                     const float *k_norm_w, const float *gate_bias, const int64_t *pos,
+                     void *k_cache, void *v_cache, const beam_kv_layout_t *layout, void *out,
+                     void *workspace, size_t workspace_bytes, int32_t *dev_status,
+                     beam_stream_t stream) {
+  int st = check_params(kind, p);
+  if (st) return st;
+  if (B < 0) return BEAM_ERR_INVALID_ARG;
+  if (B == 0) return BEAM_OK;
+  if (!q || !k || !v || !gate || !q_norm_w || !k_norm_w || !gate_bias || !pos || !k_cache ||
+      !v_cache || !out)
+    return BEAM_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(gate) || !aligned16(out) ||
+      !aligned16(q_norm_w) || !aligned16(k_norm_w) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      !aligned16(workspace) || (reinterpret_cast<uintptr_t>(pos) & 7u))
+    return BEAM_ERR_ALIGNMENT;
+  if ((st = check_layout(kind, p, layout))) return st;
+  DeviceInfo *dev = nullptr;
+  if ((st = device_info(&dev))) return st;
+  const int split = decode_split(kind, p, B, layout->slots_per_seq, dev->sm_count);
+  const int64_t vis_max = kind == BEAM_LOCAL ? p->window : layout->slots_per_seq;
+  const int n_split_max = (int)((vis_max + split - 1) / split);
+  DecodeWorkspace w = decode_workspace(workspace, B, n_split_max);
+  if (!workspace || workspace_bytes < w.bytes) return BEAM_ERR_WORKSPACE;
+  if (n_split_max > 65535) return BEAM_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+  PrologueArgs pa;
+  memset(&pa, 0, sizeof pa);
+  pa.q = static_cast<const uint16_t *>(q);
+  pa.k = static_cast<const uint16_t *>(k);
+  pa.v = static_cast<const uint16_t *>(v);
+  pa.qw = q_norm_w;
+  pa.kw = k_norm_w;
+  pa.q_out = w.qn;
+  pa.k_out = nullptr;
+  pa.k_cache = static_cast<uint16_t *>(k_cache);
+  pa.v_cache = static_cast<uint16_t *>(v_cache);
+  pa.stride_seq = layout->stride_seq;
+  pa.stride_head = layout->stride_head;
+  pa.slots = layout->slots_per_seq;
+  pa.pos0 = pos;
+  pa.status = dev_status;
+  pa.T = 1;
+  pa.kind = kind;
+  pa.window = p->window;
+  pa.eps = p->rms_eps;
+  fill_inv_freq(pa.inv_freq, p->rope_theta);
+  prologue_kernel<<<(unsigned)B, 128, 0, s>>>(pa);
+  if ((st = launch_status())) return st;
+
+  DecodeArgs da;
+  da.qn = w.qn;
+  da.k_cache = static_cast<const uint16_t *>(k_cache);
+  da.v_cache = static_cast<const uint16_t *>(v_cache);
+  da.stride_seq = layout->stride_seq;
+  da.stride_head = layout->stride_head;
+  da.slots = layout->slots_per_seq;
+  da.pos = pos;
+  da.kind = kind;
+  da.window = p->window;
+  da.split = split;
+  da.n_split_max = n_split_max;
+  da.scale_log2 = p->softmax_scale * kLog2e;
+  da.ssmax_base = p->ssmax_base;
+  da.ssmax_exp = p->ssmax_exp;
+  da.part_o = w.part_o;
+  da.part_ml = w.part_ml;
+  dim3 grid(n_split_max, kHkv, B);
+  decode_splitk_kernel<<<grid, kDecThreads, kDecSmem, s>>>(da);
+  if ((st = launch_status())) return st;
+
+  CombineArgs ca;
+  ca.part_o = w.part_o;
+  ca.part_ml = w.part_ml;
+  ca.pos = pos;
+  ca.gate = static_cast<const uint16_t *>(gate);
+  ca.gate_bias = gate_bias;
+  ca.out = static_cast<uint16_t *>(out);
+  ca.kind = kind;
+  ca.window = p->window;
+  ca.split = split;
+  ca.n_split_max = n_split_max;
+  ca.slots = layout->slots_per_seq;
+  decode_combine_kernel<<<dim3(kHq, B), 256, 0, s>>>(ca);
+  return launch_status();
+}
+
+const char *beam_status_string(int status) {
+  switch (status) {
+    case BEAM_OK: return "ok";
+    case BEAM_ERR_INVALID_ARG: return "invalid argument";
+    case BEAM_ERR_UNSUPPORTED: return "unsupported head layout or size";
+    case BEAM_ERR_CUDA: return "CUDA launch or query failed";
+    case BEAM_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait ran out";
+    case BEAM_ERR_CAPACITY: return "position does not fit the cache";
+    case BEAM_ERR_WORKSPACE: return "workspace missing or too small";
+    case BEAM_ERR_ALIGNMENT: return "tensor pointer or stride not 16-byte aligned";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

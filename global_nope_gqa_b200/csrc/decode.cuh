@@ -1,0 +1,307 @@
+// decode.cuh -- split-K decode attention over the bf16 KV cache, then the gate.
+//
+// "Beam 1.0: Local RoPE, Global NoPE and Scalable Softmax": one new query per
+// sequence attends over the cached keys it can see (section "Two attention
+// paths": keys t-511 .. t in a local layer, 0 .. t in a global one); the six
+// query heads of a GQA group share one KV head (section "Follow the tensors"),
+// and the time goes into streaming the global caches, 4 KiB per token per
+// layer (section "KV memory").
+//
+// decode_splitk_kernel: grid (split, KV head, sequence), 128 threads.  A CTA
+// streams a contiguous run of `split` cache slots of one (sequence, KV head) --
+// keys and values are contiguous in the head-major cache -- through a 3-stage
+// cp.async ring of 64-slot tiles (16-byte coalesced loads, XOR-swizzled rows).
+// The six heads of the group are the M rows of m16n8k16 tensor-core MMAs
+// (rows 6..15 are zero): S = Q K^T and O += P V.  The MMAs exist to take the
+// 6 x 128 x 2 multiply-adds per cached row off the FP32 pipe, which would
+// otherwise bound the kernel below HBM speed.  Each warp keeps its own online
+// softmax over a quarter of every tile; the four warps merge in shared memory and
+// the CTA writes one partial (m, l, o[128]) per head.
+//
+// decode_combine_kernel: one CTA per (sequence, query head) merges the partials
+// with the log-sum-exp rule and applies Y = O/l * sigmoid(G + b_h).
+#pragma once
+
+#include "common.cuh"
+
+namespace beam {
+
+constexpr int kDecThreads = 128;
+constexpr int kDecTile = 64;    // cache slots per shared-memory tile
+constexpr int kDecStages = 3;   // 96 KiB: two CTAs per SM
+constexpr int kDecTileBytes = kDecTile * kD * 2;                   // 16 KiB
+constexpr int kDecSmem = kDecStages * 2 * kDecTileBytes;
+
+struct DecodeArgs {
+  const uint16_t *qn;       // [B][48][128] prepared queries
+  const uint16_t *k_cache;
+  const uint16_t *v_cache;
+  int64_t stride_seq, stride_head, slots;
+  const int64_t *pos;       // [B] 0-based position of the new token
+  int kind, window;
+  int split;                // cache slots per CTA (multiple of kDecTile)
+  int n_split_max;          // partial slots reserved per (sequence, KV head)
+  float scale_log2;         // softmax_scale * log2(e)
+  float ssmax_base, ssmax_exp;
+  float *part_o;            // [B][8][n_split_max][6][128]
+  float *part_ml;           // [B][8][n_split_max][6][2]  (running max in log2 units, sum)
+};
+
+// Number of visible slots of sequence b (0 when the position is invalid).
+__device__ __forceinline__ int64_t decode_visible(const DecodeArgs &a, int64_t t) {
+  if (t < 0) return 0;
+  if (a.kind == BEAM_LOCAL) return t + 1 < a.window ? t + 1 : a.window;
+  return t < a.slots ? t + 1 : 0;
+}
+
+__global__ void __launch_bounds__(kDecThreads) decode_splitk_kernel(const DecodeArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int s_idx = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int64_t t = a.pos[b];
+  const int64_t n_vis = decode_visible(a, t);
+  const int64_t key_lo = (int64_t)s_idx * a.split;
+  if (key_lo >= n_vis) return;
+  const int64_t key_hi = min(n_vis, key_lo + a.split);
+  const int n_keys = (int)(key_hi - key_lo);
+  const int n_tiles = (n_keys + kDecTile - 1) / kDecTile;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const size_t head_off = (size_t)b * a.stride_seq + (size_t)g * a.stride_head;
+  const uint16_t *kbase = a.k_cache + head_off;
+  const uint16_t *vbase = a.v_cache + head_off;
+
+  float factor = a.scale_log2;
+  if (a.kind == BEAM_GLOBAL) factor *= ssmax_factor(t + 1, a.ssmax_base, a.ssmax_exp);
+
+  // Query fragments: A rows = heads (lane/4 < 6 valid), 8 k-steps over d.
+  uint32_t qa[8][2];
+  {
+    const int h = lane >> 2;
+    const uint16_t *qrow = a.qn + ((size_t)b * kHq + g * kGroup + (h < kGroup ? h : 0)) * kD;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const int d0 = ks * 16 + (lane & 3) * 2;
+      uint32_t lo = *reinterpret_cast<const uint32_t *>(qrow + d0);
+      uint32_t hi = *reinterpret_cast<const uint32_t *>(qrow + d0 + 8);
+      qa[ks][0] = h < kGroup ? lo : 0u;
+      qa[ks][1] = h < kGroup ? hi : 0u;
+    }
+  }
+
+  auto load_tile = [&](int tile, int stage) {
+    uint8_t *ks = smem + stage * 2 * kDecTileBytes;
+    uint8_t *vs = ks + kDecTileBytes;
+    const int64_t row0 = key_lo + (int64_t)tile * kDecTile;
+#pragma unroll
+    for (int it = 0; it < (kDecTile * 16) / kDecThreads; ++it) {
+      const int id = tid + it * kDecThreads;
+      const int r = id >> 4, c = id & 15;
+      const bool valid = row0 + r < key_hi;
+      const int64_t row = valid ? row0 + r : key_lo;
+      const uint32_t off = swz256(r, c);
+      cp_async16(smem_u32(ks + off), kbase + row * kD + c * 8, valid);
+      cp_async16(smem_u32(vs + off), vbase + row * kD + c * 8, valid);
+    }
+  };
+
+#pragma unroll
+  for (int st = 0; st < kDecStages - 1; ++st) {
+    if (st < n_tiles) load_tile(st, st);
+    cp_async_commit();
+  }
+
+  float m_run = -INFINITY;   // running max (log2 units) of head lane/4
+  float l_run = 0.f;         // this thread's share of the running sum
+  float o[16][4];
+#pragma unroll
+  for (int nb = 0; nb < 16; ++nb) o[nb][0] = o[nb][1] = o[nb][2] = o[nb][3] = 0.f;
+
+  for (int tile = 0; tile < n_tiles; ++tile) {
+    cp_async_wait<kDecStages - 2>();
+    __syncthreads();
+    {  // refill the stage that the previous iteration finished with
+      const int nt = tile + kDecStages - 1;
+      if (nt < n_tiles) load_tile(nt, nt % kDecStages);
+      cp_async_commit();
+    }
+    const uint8_t *ks = smem + (tile % kDecStages) * 2 * kDecTileBytes;
+    const uint8_t *vs = ks + kDecTileBytes;
+    const int wrow = warp * 16;  // this warp's 16 slots of the tile
+
+    // S[head][key] for the warp's 16 keys: two n-blocks of 8 keys.
+    float s[2][4];
+#pragma unroll
+    for (int nb = 0; nb < 2; ++nb) s[nb][0] = s[nb][1] = s[nb][2] = s[nb][3] = 0.f;
+#pragma unroll
+    for (int kstep = 0; kstep < 8; ++kstep) {
+      // matrices: (keys 0-7, d lo), (keys 0-7, d hi), (keys 8-15, d lo), (keys 8-15, d hi)
+      const int r = wrow + (lane & 7) + ((lane >> 4) << 3);
+      const int c = kstep * 2 + ((lane >> 3) & 1);
+      uint32_t kb[4];
+      ldmatrix_x4(kb, smem_u32(ks + swz256(r, c)));
+      const uint32_t afr[4] = {qa[kstep][0], 0u, qa[kstep][1], 0u};
+      mma_bf16_16816(s[0], afr, kb[0], kb[1]);
+      mma_bf16_16816(s[1], afr, kb[2], kb[3]);
+    }
+    // scale, mask the ragged end, online softmax for head lane/4
+    const int key0 = tile * kDecTile + wrow + (lane & 3) * 2;  // key of s[0][0] within the run
+    float mx = -INFINITY;
+#pragma unroll
+    for (int nb = 0; nb < 2; ++nb)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int kk = key0 + nb * 8 + e;
+        float v = s[nb][e] * factor;
+        v = kk < n_keys ? v : -INFINITY;
+        s[nb][e] = v;
+        mx = fmaxf(mx, v);
+      }
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const float m_new = fmaxf(m_run, mx);
+    const float m_use = m_new == -INFINITY ? 0.f : m_new;
+    const float corr = exp2f(m_run - m_use);
+    m_run = m_new;
+    float p[2][2];
+    float psum = 0.f;
+#pragma unroll
+    for (int nb = 0; nb < 2; ++nb)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        p[nb][e] = exp2f(s[nb][e] - m_use);
+        psum += p[nb][e];
+      }
+    l_run = l_run * corr + psum;
+#pragma unroll
+    for (int nb = 0; nb < 16; ++nb) { o[nb][0] *= corr; o[nb][1] *= corr; }
+
+    // O[head][d] += P[head][key16] V[key16][d]
+    const uint32_t pa[4] = {pack_bf16(p[0][0], p[0][1]), 0u, pack_bf16(p[1][0], p[1][1]), 0u};
+#pragma unroll
+    for (int nb = 0; nb < 16; nb += 2) {
+      // matrices: (keys 0-7, d block nb), (keys 8-15, nb), (keys 0-7, nb+1), (keys 8-15, nb+1)
+      const int r = wrow + (lane & 7) + (((lane >> 3) & 1) << 3);
+      const int c = nb + (lane >> 4);
+      uint32_t vb[4];
+      ldmatrix_x4_trans(vb, smem_u32(vs + swz256(r, c)));
+      mma_bf16_16816(o[nb], pa, vb[0], vb[1]);
+      mma_bf16_16816(o[nb + 1], pa, vb[2], vb[3]);
+    }
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+
+  // Merge the four warps.  Shared memory is free again: reuse it.
+  float *sm_o = reinterpret_cast<float *>(smem);                 // [4 warps][6][128]
+  float *sm_m = sm_o + 4 * kGroup * kD;                          // [4][6]
+  float *sm_l = sm_m + 4 * kGroup;                               // [4][6]
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+  const int h = lane >> 2;
+  if (h < kGroup) {
+#pragma unroll
+    for (int nb = 0; nb < 16; ++nb) {
+      const int d0 = nb * 8 + (lane & 3) * 2;
+      sm_o[(warp * kGroup + h) * kD + d0] = o[nb][0];
+      sm_o[(warp * kGroup + h) * kD + d0 + 1] = o[nb][1];
+    }
+    if ((lane & 3) == 0) {
+      sm_m[warp * kGroup + h] = m_run;
+      sm_l[warp * kGroup + h] = l_run;
+    }
+  }
+  __syncthreads();
+  const size_t part = ((size_t)b * kHkv + g) * a.n_split_max + s_idx;
+  for (int idx = tid; idx < kGroup * kD; idx += kDecThreads) {
+    const int hh = idx / kD, d = idx - hh * kD;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) M = fmaxf(M, sm_m[w * kGroup + hh]);
+    const float Mu = M == -INFINITY ? 0.f : M;
+    float acc = 0.f, L = 0.f;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const float sc = exp2f(sm_m[w * kGroup + hh] - Mu);
+      acc += sc * sm_o[(w * kGroup + hh) * kD + d];
+      L += sc * sm_l[w * kGroup + hh];
+    }
+    a.part_o[part * (kGroup * kD) + idx] = acc;
+    if (d == 0) {
+      a.part_ml[(part * kGroup + hh) * 2 + 0] = M;
+      a.part_ml[(part * kGroup + hh) * 2 + 1] = L;
+    }
+  }
+}
+
+struct CombineArgs {
+  const float *part_o;
+  const float *part_ml;
+  const int64_t *pos;
+  const uint16_t *gate;     // [B][48*128]
+  const float *gate_bias;   // [48]
+  uint16_t *out;            // [B][48*128]
+  int kind, window, split, n_split_max;
+  int64_t slots;
+};
+
+// 256 threads: warp w merges splits w, w+8, ...; lane l owns d = 4l .. 4l+3.
+__global__ void __launch_bounds__(256) decode_combine_kernel(const CombineArgs a) {
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int g = h / kGroup, hh = h - g * kGroup;
+  const int64_t t = a.pos[b];
+  int64_t n_vis;
+  if (t < 0) n_vis = 0;
+  else if (a.kind == BEAM_LOCAL) n_vis = t + 1 < a.window ? t + 1 : a.window;
+  else n_vis = t < a.slots ? t + 1 : 0;
+  if (n_vis == 0) return;  // invalid position: output untouched, status set upstream
+  const int n_split = (int)((n_vis + a.split - 1) / a.split);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  __shared__ float sm_o[8][kD];
+  __shared__ float sm_m[8], sm_l[8];
+  float M = -INFINITY, L = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  const size_t base = ((size_t)b * kHkv + g) * a.n_split_max;
+  for (int s = warp; s < n_split; s += 8) {
+    const size_t part = base + s;
+    const float m = a.part_ml[(part * kGroup + hh) * 2 + 0];
+    const float l = a.part_ml[(part * kGroup + hh) * 2 + 1];
+    const float4 v = reinterpret_cast<const float4 *>(a.part_o + (part * kGroup + hh) * kD)[lane];
+    const float Mn = fmaxf(M, m);
+    const float Mu = Mn == -INFINITY ? 0.f : Mn;
+    const float c0 = exp2f(M - Mu), c1 = exp2f(m - Mu);
+    acc.x = acc.x * c0 + v.x * c1; acc.y = acc.y * c0 + v.y * c1;
+    acc.z = acc.z * c0 + v.z * c1; acc.w = acc.w * c0 + v.w * c1;
+    L = L * c0 + l * c1;
+    M = Mn;
+  }
+  reinterpret_cast<float4 *>(sm_o[warp])[lane] = acc;
+  if (lane == 0) { sm_m[warp] = M; sm_l[warp] = L; }
+  __syncthreads();
+  if (warp == 0) {
+    float Mt = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) Mt = fmaxf(Mt, sm_m[w]);
+    const float Mu = Mt == -INFINITY ? 0.f : Mt;
+    float Lt = 0.f, r[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      const float c = exp2f(sm_m[w] - Mu);
+      Lt += c * sm_l[w];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) r[e] += c * sm_o[w][lane * 4 + e];
+    }
+    const float inv = 1.0f / Lt;
+    const float bias = a.gate_bias[h];
+    const uint2 graw = reinterpret_cast<const uint2 *>(a.gate + ((size_t)b * kHq + h) * kD)[lane];
+    const float gl[4] = {bf16_lo(graw.x), bf16_hi(graw.x), bf16_lo(graw.y), bf16_hi(graw.y)};
+    float y[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) y[e] = r[e] * inv * (1.0f / (1.0f + expf(-(gl[e] + bias))));
+    uint2 packed;
+    packed.x = pack_bf16(y[0], y[1]);
+    packed.y = pack_bf16(y[2], y[3]);
+    reinterpret_cast<uint2 *>(a.out + ((size_t)b * kHq + h) * kD)[lane] = packed;
+  }
+}
+
+}  // namespace beam

@@ -1,0 +1,153 @@
+// prologue.cuh -- QK-RMSNorm + RoPE (local) and the KV-cache append.
+//
+// "Beam 1.0: Local RoPE, Global NoPE and Scalable Softmax", section "Follow the
+// tensors, not the parameter label": Q and K are RMS-normalised along the
+// 128-wide head axis (eps 1e-6, learned weight), V is not; local layers then
+// rotate Q and K with RoPE; global layers leave K alone and scale only Q by a(p).
+// Here a(p) is not applied: the attention kernels fold it into the fp32 score
+// scale, so the prepared Q of a global layer is the normalised Q.
+//
+// One CTA of 128 threads per token.  Each half-warp owns one 128-wide row:
+// lane l (0..15) holds coordinates 8l .. 8l+7 as one 16-byte load, so the
+// rotate-half partner of lane l is lane l ^ 8.  The 64 RoPE angles of a token
+// are formed once per lane in fp64 (t * frequency, then reduced to [-pi, pi]),
+// because in fp32 t * frequency is off by up to ~0.06 rad at t ~ 1e6; the
+// reduced angle then goes through fp32 sincosf.  Rows: 48 query heads, 8 key
+// heads, and 8 value heads when a cache is written (copied unchanged).
+#pragma once
+
+#include "common.cuh"
+
+namespace beam {
+
+struct PrologueArgs {
+  const uint16_t *q;     // [tokens][48*128] or null (append only)
+  const uint16_t *k;     // [tokens][8*128]
+  const uint16_t *v;     // [tokens][8*128] (read only when a cache is written)
+  const float *qw;       // [128]
+  const float *kw;       // [128]
+  uint16_t *q_out;       // [tokens][48*128] prepared queries, or null
+  uint16_t *k_out;       // [tokens][8*128] prepared keys, or null
+  uint16_t *k_cache;     // layer caches, or null
+  uint16_t *v_cache;
+  int64_t stride_seq, stride_head, slots;
+  const int64_t *pos0;   // device [B]: position of token 0 of each sequence, or null (= 0)
+  int32_t *status;
+  int T;                 // tokens per sequence in this call
+  int kind;
+  int window;
+  float eps;
+  double inv_freq[64];   // theta^(-2i/128), formed on the host in double
+};
+
+__device__ __forceinline__ void rope_angles(const PrologueArgs &a, int64_t t, int sub,
+                                            float (&cs)[8], float (&sn)[8]) {
+  const double two_pi = 6.283185307179586;
+  const double inv_two_pi = 0.15915494309189535;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    double phi = (double)t * a.inv_freq[sub * 8 + e];
+    double n = rint(phi * inv_two_pi);
+    double r = fma(-n, two_pi, phi);  // |r| <= pi (+ rounding)
+    sincosf((float)r, &sn[e], &cs[e]);
+  }
+}
+
+__global__ void __launch_bounds__(128) prologue_kernel(const PrologueArgs a) {
+  const int tok = blockIdx.x;
+  const int b = tok / a.T;
+  const int i = tok - b * a.T;
+  const int64_t t = (a.pos0 ? a.pos0[b] : 0) + i;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int half = lane >> 4, l16 = lane & 15;
+  const bool local = a.kind == BEAM_LOCAL;
+
+  // Cache target of this token.
+  bool write_cache = a.k_cache != nullptr;
+  int64_t slot = 0;
+  if (write_cache) {
+    if (t < 0) {
+      set_status(a.status, BEAM_ERR_CAPACITY);
+      write_cache = false;
+    } else if (local) {
+      write_cache = i >= a.T - a.window;  // earlier tokens of the call leave the window
+      slot = t % a.window;
+    } else {
+      slot = t;
+      if (t >= a.slots) {
+        if (threadIdx.x == 0) set_status(a.status, BEAM_ERR_CAPACITY);
+        write_cache = false;
+      }
+    }
+  }
+
+  float cs[8], sn[8];
+  if (local) rope_angles(a, t < 0 ? 0 : t, l16 & 7, cs, sn);
+
+  float wq[8], wk[8];
+  {
+    const float4 *q4 = reinterpret_cast<const float4 *>(a.qw) + l16 * 2;
+    const float4 *k4 = reinterpret_cast<const float4 *>(a.kw) + l16 * 2;
+    float4 x0 = q4[0], x1 = q4[1], y0 = k4[0], y1 = k4[1];
+    wq[0] = x0.x; wq[1] = x0.y; wq[2] = x0.z; wq[3] = x0.w;
+    wq[4] = x1.x; wq[5] = x1.y; wq[6] = x1.z; wq[7] = x1.w;
+    wk[0] = y0.x; wk[1] = y0.y; wk[2] = y0.z; wk[3] = y0.w;
+    wk[4] = y1.x; wk[5] = y1.y; wk[6] = y1.z; wk[7] = y1.w;
+  }
+
+  const unsigned half_mask = 0xFFFFu << (half * 16);  // shuffles stay inside the half-warp
+  const int n_rows = kHq + kHkv + kHkv;  // q heads, k heads, v heads
+  for (int row = warp * 2 + half; row < n_rows; row += 8) {
+    const bool is_q = row < kHq;
+    const bool is_k = !is_q && row < kHq + kHkv;
+    const bool is_v = row >= kHq + kHkv;
+    if (is_q && (a.q == nullptr || a.q_out == nullptr)) continue;
+    if (is_k && a.k_out == nullptr && !write_cache) continue;
+    if (is_v && !write_cache) continue;
+    const int head = is_q ? row : (is_k ? row - kHq : row - kHq - kHkv);
+    const uint16_t *src = is_q ? a.q + (size_t)tok * (kHq * kD) + head * kD
+                               : (is_k ? a.k : a.v) + (size_t)tok * (kHkv * kD) + head * kD;
+    uint4 raw = *reinterpret_cast<const uint4 *>(src + l16 * 8);
+    uint4 res = raw;
+    if (!is_v) {
+      float x[8];
+      x[0] = bf16_lo(raw.x); x[1] = bf16_hi(raw.x); x[2] = bf16_lo(raw.y); x[3] = bf16_hi(raw.y);
+      x[4] = bf16_lo(raw.z); x[5] = bf16_hi(raw.z); x[6] = bf16_lo(raw.w); x[7] = bf16_hi(raw.w);
+      float ss = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
+#pragma unroll
+      for (int off = 1; off < 16; off <<= 1) ss += __shfl_xor_sync(half_mask, ss, off);
+      const float inv_rms = rsqrtf(ss * (1.0f / kD) + a.eps);
+      const float *w = is_q ? wq : wk;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) x[e] = x[e] * inv_rms * w[e];
+      if (local) {
+        // rotate-half: coordinate c < 64 pairs with c + 64, held by lane l16 ^ 8
+        float y[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          float partner = __shfl_xor_sync(half_mask, x[e], 8);
+          y[e] = (l16 < 8) ? (x[e] * cs[e] - partner * sn[e]) : (x[e] * cs[e] + partner * sn[e]);
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = y[e];
+      }
+      res.x = pack_bf16(x[0], x[1]); res.y = pack_bf16(x[2], x[3]);
+      res.z = pack_bf16(x[4], x[5]); res.w = pack_bf16(x[6], x[7]);
+    }
+    if (is_q) {
+      *reinterpret_cast<uint4 *>(a.q_out + (size_t)tok * (kHq * kD) + head * kD + l16 * 8) = res;
+    } else {
+      if (is_k && a.k_out)
+        *reinterpret_cast<uint4 *>(a.k_out + (size_t)tok * (kHkv * kD) + head * kD + l16 * 8) = res;
+      if (write_cache) {
+        uint16_t *cache = is_k ? a.k_cache : a.v_cache;
+        size_t off = (size_t)b * a.stride_seq + (size_t)head * a.stride_head + (size_t)slot * kD;
+        *reinterpret_cast<uint4 *>(cache + off + l16 * 8) = res;
+      }
+    }
+  }
+}
+
+}  // namespace beam
