@@ -19,7 +19,6 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -48,6 +47,14 @@ def decode_kv_bytes(ctx, kind: int, window: int = wl.WINDOW) -> int:
     per_token = 2 * wl.N_KV_HEADS * wl.HEAD_DIM * 2
     io = len(ctx) * 2 * (3 * wl.N_Q_HEADS * wl.HEAD_DIM + 2 * wl.N_KV_HEADS * wl.HEAD_DIM)
     return vis * per_token + io
+
+
+def _jsonable(o):
+    if isinstance(o, (np.integer,)):
+        return int(o)
+    if isinstance(o, (np.floating,)):
+        return float(o)
+    raise TypeError(type(o))
 
 
 def peaks():
@@ -86,47 +93,72 @@ def aggregate(per_rank_units: float, world: int, seconds_max: float) -> float:
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Samples SM clocks and clock-event reasons through NVML (read-only queries)
+    every 50 ms while the timed region runs."""
+    BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+            "hw_thermal_slowdown": 0x40}
 
-    def __init__(self, index: int):
-        self.index = index
+    def __init__(self, cuda_index: int):
         self.rows = []
         self._stop = threading.Event()
         self._th = None
+        self._handle = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(cuda_index).uuid)
+            h = None
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                cand = pynvml.nvmlDeviceGetHandleByIndex(i)
+                u = pynvml.nvmlDeviceGetUUID(cand)
+                u = u.decode() if isinstance(u, bytes) else u
+                if u.replace("GPU-", "") == uuid.replace("GPU-", ""):
+                    h = cand
+            if h is None and pynvml.nvmlDeviceGetCount() == 1:
+                h = pynvml.nvmlDeviceGetHandleByIndex(0)
+            self._nvml, self._handle = pynvml, h
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM) if h else None
+        except Exception:
+            self._handle = None
+            self.max_mhz = None
+
+    def _sample(self):
+        n = self._nvml
+        sm = n.nvmlDeviceGetClockInfo(self._handle, n.NVML_CLOCK_SM)
+        try:
+            reasons = n.nvmlDeviceGetCurrentClocksEventReasons(self._handle)
+        except AttributeError:
+            reasons = n.nvmlDeviceGetCurrentClocksThrottleReasons(self._handle)
+        self.rows.append((sm, reasons))
 
     def _run(self):
         while not self._stop.is_set():
             try:
-                out = subprocess.run(
-                    ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                     "--format=csv,noheader,nounits"], capture_output=True, text=True, timeout=5)
-                if out.returncode == 0 and out.stdout.strip():
-                    self.rows.append([x.strip() for x in out.stdout.strip().split(",")])
+                self._sample()
             except Exception:
                 pass
-            self._stop.wait(0.2)
+            self._stop.wait(0.05)
 
     def __enter__(self):
-        self._th = threading.Thread(target=self._run, daemon=True)
-        self._th.start()
+        if self._handle is not None:
+            self._sample()   # first query outside the timed region
+            self._th = threading.Thread(target=self._run, daemon=True)
+            self._th.start()
         return self
 
     def __exit__(self, *exc):
         self._stop.set()
-        self._th.join(timeout=10)
+        if self._th:
+            self._th.join(timeout=10)
 
     def summary(self):
-        if not self.rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        sm = [float(r[0]) for r in self.rows if r[0].replace(".", "").isdigit()]
-        mx = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in self.rows for n, v in zip(names, r[4:8]) if v == "Active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
-                "samples": len(self.rows)}
+        rows = self.rows[1:] or self.rows
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"]}
+        reasons = sorted({name for _, r in rows for name, bit in self.BITS.items() if r & bit})
+        return {"sm_mhz": statistics.median(sm for sm, _ in rows), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(rows)}
 
 
 # ------------------------------------------------------------------ GPU arm
@@ -437,7 +469,7 @@ def run_gpu(args):
     if rank == 0 and world == 1 and not args.no_cpu:
         result["cpu_baseline"] = cpu_baseline_prefill(seed=args.seed)
     if rank == 0:
-        print(json.dumps(result), flush=True)
+        print(json.dumps(result, default=_jsonable), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
 
@@ -465,13 +497,13 @@ def run_reference(args):
                          "kind": "oracle", "sample": base["sample"]},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
-    print(json.dumps(line), flush=True)
+    print(json.dumps(line, default=_jsonable), flush=True)
 
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="beam", choices=["beam", "reference"])
     ap.add_argument("--seed", type=int, default=1234)

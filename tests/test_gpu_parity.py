@@ -15,6 +15,10 @@ pytestmark = pytest.mark.gpu
 
 ATOL = 1e-2
 RTOL = 1e-2
+# Prepared keys are formed in fp32 on the device and in double by the oracle, then
+# both are rounded to bf16: the two may sit one bf16 step apart, and where RoPE
+# cancels (a small coordinate from O(1) terms) the fp32 rounding adds ~1e-6.
+K_ABS = 1e-5
 
 
 @pytest.fixture(scope="module")
@@ -219,9 +223,10 @@ def test_prefill_fused_append_bit_exact(env, kind, B, T):
             kr, vr = orc.kv_row(kind, P, inp.k[b, t], inp.v[b, t], inp.k_norm_w, t)
             np.testing.assert_array_equal(vh[b, :, s], vr)
             d = np.abs(as_f64(kh[b, :, s]) - as_f64(kr))
-            assert np.all(d <= np.abs(as_f64(kr)) * 2.0 ** -7 + 1e-30), (b, t)
+            assert np.all(d <= np.abs(as_f64(kr)) * 2.0 ** -7 + K_ABS), (b, t)
             written[b, s] = True
-    assert np.all(kh[~written] == sentinel) and np.all(vh[~written] == sentinel)
+    assert np.all(kh.transpose(0, 2, 1, 3)[~written] == sentinel)
+    assert np.all(vh.transpose(0, 2, 1, 3)[~written] == sentinel)
 
 
 @pytest.mark.parametrize("kind", [wl.GLOBAL, wl.LOCAL])
@@ -255,10 +260,11 @@ def test_kv_append_positions_bit_exact(env, kind):
             kr, vr = orc.kv_row(kind, P, k[b, i], v[b, i], kw, t)
             np.testing.assert_array_equal(vh[b, :, s], vr)
             d = np.abs(as_f64(kh[b, :, s]) - as_f64(kr))
-            assert np.all(d <= np.abs(as_f64(kr)) * 2.0 ** -7 + 1e-30), (b, i)
+            assert np.all(d <= np.abs(as_f64(kr)) * 2.0 ** -7 + K_ABS), (b, i)
             written[b, s] = True
     sentinel = wl.f32_to_bf16_bits(np.float32([-7.0]))[0]
-    assert np.all(vh[~written] == sentinel)
+    assert np.all(vh.transpose(0, 2, 1, 3)[~written] == sentinel)
+    assert np.all(kh.transpose(0, 2, 1, 3)[~written] == sentinel)
 
 
 def test_kv_append_capacity_sets_status(env):
