@@ -21,12 +21,13 @@ LOCAL, GLOBAL = 0, 1
 STATUS = {
     0: "BEAM_OK", -1: "BEAM_ERR_INVALID_ARG", -2: "BEAM_ERR_UNSUPPORTED", -3: "BEAM_ERR_CUDA",
     -4: "BEAM_ERR_DEVICE_TIMEOUT", -5: "BEAM_ERR_CAPACITY", -6: "BEAM_ERR_WORKSPACE",
-    -7: "BEAM_ERR_ALIGNMENT",
+    -7: "BEAM_ERR_ALIGNMENT", -8: "BEAM_ERR_SCRATCH_LIMIT",
 }
 
 EXPORTS = (
     "beam_default_params", "beam_kv_layout", "beam_prefill_workspace_bytes", "beam_attn_prefill",
     "beam_kv_append", "beam_decode_workspace_bytes", "beam_attn_decode", "beam_status_string",
+    "beam_attn_decode_noalloc",
 )
 
 
@@ -83,6 +84,9 @@ def lib() -> ctypes.CDLL:
         L.beam_attn_decode.restype = ctypes.c_int
         L.beam_attn_decode.argtypes = [ctypes.c_int, pp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                        vp, lp, vp, vp, sz, vp, vp]
+        L.beam_attn_decode_noalloc.restype = ctypes.c_int
+        L.beam_attn_decode_noalloc.argtypes = [ctypes.c_int, pp, i32, vp, vp, vp, vp, vp, vp, vp,
+                                               vp, vp, vp, lp, vp, vp, vp]
         L.beam_status_string.restype = ctypes.c_char_p
         L.beam_status_string.argtypes = [ctypes.c_int]
         _lib = L
@@ -184,6 +188,19 @@ def beam_attn_decode(kind, params, q, k, v, gate, q_norm_w, k_norm_w, gate_bias,
         ctypes.byref(layout), _ptr(out), _ptr(workspace), ws_bytes, _ptr(dev_status),
         _stream(stream))
     _check("beam_attn_decode", rc)
+    return out
+
+
+def beam_attn_decode_noalloc(kind, params, q, k, v, gate, q_norm_w, k_norm_w, gate_bias, pos,
+                             k_cache, v_cache, layout: KVLayout, out, dev_status=None, stream=None):
+    """Same as beam_attn_decode, for callers that cannot allocate: the scratch is the
+    library's fixed 8 MiB device array (shared by all calls; overlapping calls race)."""
+    B = q.shape[0]
+    rc = lib().beam_attn_decode_noalloc(
+        kind, ctypes.byref(params), B, _ptr(q), _ptr(k), _ptr(v), _ptr(gate), _ptr(q_norm_w),
+        _ptr(k_norm_w), _ptr(gate_bias), _ptr(pos), _ptr(k_cache), _ptr(v_cache),
+        ctypes.byref(layout), _ptr(out), _ptr(dev_status), _stream(stream))
+    _check("beam_attn_decode_noalloc", rc)
     return out
 
 

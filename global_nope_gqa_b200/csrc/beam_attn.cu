@@ -371,6 +371,57 @@ int beam_attn_decode(int kind, const beam_attn_params *p, int32_t B, const void 
   return launch_status();
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Fixed device scratch of beam_attn_decode_noalloc.  In host code the name
+// g_decode_scratch is only a host-side stand-in for the array, not its device
+// address: passing it to a kernel would fault or, where the GPU can reach host
+// memory, silently touch the wrong memory.  The device address is looked up
+// once per device with cudaGetSymbolAddress while that device is current.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB
+static __device__ __align__(256) uint8_t g_decode_scratch[kNoAllocScratchBytes];
+
+void *g_scratch_addr[kMaxDevices];
+
+int noalloc_scratch(void **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BEAM_ERR_CUDA;
+  if (!g_scratch_addr[dev]) {
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_decode_scratch) != cudaSuccess || !ptr) return BEAM_ERR_CUDA;
+    g_scratch_addr[dev] = ptr;
+  }
+  *out = g_scratch_addr[dev];
+  return BEAM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int beam_attn_decode_noalloc(int kind, const beam_attn_params *p, int32_t B, const void *q,
+                             const void *k, const void *v, const void *gate,
+                             const float *q_norm_w, const float *k_norm_w,
+                             const float *gate_bias, const int64_t *pos, void *k_cache,
+                             void *v_cache, const beam_kv_layout_t *layout, void *out,
+                             int32_t *dev_status, beam_stream_t stream) {
+  int st = check_params(kind, p);
+  if (st) return st;
+  if (B < 0) return BEAM_ERR_INVALID_ARG;
+  if (B == 0) return BEAM_OK;
+  if ((st = check_layout(kind, p, layout))) return st;
+  const size_t need = beam_decode_workspace_bytes(kind, p, B, layout);
+  if (need == 0) return BEAM_ERR_CUDA;
+  if (need > kNoAllocScratchBytes) return BEAM_ERR_SCRATCH_LIMIT;
+  void *scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch))) return st;
+  return beam_attn_decode(kind, p, B, q, k, v, gate, q_norm_w, k_norm_w, gate_bias, pos, k_cache,
+                          v_cache, layout, out, scratch, kNoAllocScratchBytes, dev_status, stream);
+}
+
 const char *beam_status_string(int status) {
   switch (status) {
     case BEAM_OK: return "ok";
@@ -381,6 +432,7 @@ const char *beam_status_string(int status) {
     case BEAM_ERR_CAPACITY: return "position does not fit the cache";
     case BEAM_ERR_WORKSPACE: return "workspace missing or too small";
     case BEAM_ERR_ALIGNMENT: return "tensor pointer or stride not 16-byte aligned";
+    case BEAM_ERR_SCRATCH_LIMIT: return "call needs more than the fixed 8 MiB decode scratch";
     default: return "unknown status";
   }
 }

@@ -67,7 +67,9 @@ typedef enum {
   BEAM_ERR_DEVICE_TIMEOUT = -4, /* device side: a bounded wait ran out */
   BEAM_ERR_CAPACITY = -5,       /* a position does not fit the cache (host or device) */
   BEAM_ERR_WORKSPACE = -6,      /* workspace null or smaller than the query function says */
-  BEAM_ERR_ALIGNMENT = -7       /* a tensor pointer is not 16-byte aligned */
+  BEAM_ERR_ALIGNMENT = -7,      /* a tensor pointer is not 16-byte aligned */
+  BEAM_ERR_SCRATCH_LIMIT = -8   /* beam_attn_decode_noalloc: the call needs more scratch than
+                                   the library's fixed device array holds */
 } beam_status;
 
 /* Sublayer hyper-parameters.  The kernels are built for 48 query heads, 8 KV
@@ -164,6 +166,40 @@ BEAM_API int beam_attn_decode(int kind, const beam_attn_params *p, int32_t B, co
                      void *k_cache, void *v_cache, const beam_kv_layout_t *layout, void *out,
                      void *workspace, size_t workspace_bytes, int32_t *dev_status,
                      beam_stream_t stream);
+
+/* Decode without any allocation, for callers that cannot call cudaMalloc.
+ *
+ * There is no counterpart in the paper: this is a deployment convenience.  Some
+ * hosts hand a library only the buffers of its inputs and outputs and forbid
+ * it any device allocation of its own -- for example a serving runtime that
+ * pre-partitions all device memory into its own pools, or a latency-critical
+ * loop in which an allocation (and the device synchronisation that cudaMalloc
+ * and cudaFree can imply) is not acceptable -- yet beam_attn_decode needs a
+ * workspace for the prepared queries and the split-K partial results.
+ *
+ * This entry point computes exactly what beam_attn_decode computes, with the
+ * same arguments minus the workspace.  Its scratch is a fixed array of
+ * 8 MiB (8,388,608 bytes) of device memory inside the library, which every GPU
+ * that loads the library holds until the process exits.  A call whose
+ * beam_decode_workspace_bytes() would exceed 8 MiB returns
+ * BEAM_ERR_SCRATCH_LIMIT before any launch (roughly: B * 8 * splits * 3.1 KB +
+ * B * 12 KB; B = 64 at a 32K-slot cache or B = 1 at a 1M-slot cache fit).
+ *
+ * The first call on each device looks up the array's device address (with that
+ * device current) and caches it; make that first call before any stream
+ * capture.  All calls share the one array and it keeps whatever the last call
+ * left in it; nothing in it needs to start at zero, because every value read
+ * is written earlier in the same call.  Calls whose kernels overlap on the GPU
+ * (on different streams, or from several threads) race on the array: issue
+ * them on one stream, one after the other.  The call allocates nothing and
+ * calls no allocating routine. */
+BEAM_API int beam_attn_decode_noalloc(int kind, const beam_attn_params *p, int32_t B,
+                                      const void *q, const void *k, const void *v,
+                                      const void *gate, const float *q_norm_w,
+                                      const float *k_norm_w, const float *gate_bias,
+                                      const int64_t *pos, void *k_cache, void *v_cache,
+                                      const beam_kv_layout_t *layout, void *out,
+                                      int32_t *dev_status, beam_stream_t stream);
 
 /* Static description of a status code. */
 BEAM_API const char *beam_status_string(int status);

@@ -164,5 +164,5 @@ def test_host_validation_rejects_before_launch(beam):
 
     assert L.beam_kv_append(1, P, 1, 4, A, A, A, None, A, A, ctypes.byref(glob), None, None) == -1
     assert L.beam_kv_append(1, P, 1, 0, A, A, A, A, A, A, ctypes.byref(glob), None, None) == 0
-    for s in (0, -1, -2, -3, -4, -5, -6, -7, 99):
+    for s in (0, -1, -2, -3, -4, -5, -6, -7, -8, 99):
         assert isinstance(beam.beam_status_string(s), str)
