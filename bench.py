@@ -388,8 +388,10 @@ def run_gpu(args):
     beam.lib()
     pk = peaks()
     w = wl.workload("batched_prefill", args.seed + rank)
-    layers = [PrefillLayer(torch, beam, kind, w.B, w.T, w.seed, f"bench/{kind}")
-              for kind in (wl.LOCAL, wl.GLOBAL)]
+    if args.batch:
+        w.B = args.batch
+    kinds = {"both": (wl.LOCAL, wl.GLOBAL), "global": (wl.GLOBAL,), "local": (wl.LOCAL,)}[args.layers]
+    layers = [PrefillLayer(torch, beam, kind, w.B, w.T, w.seed, f"bench/{kind}") for kind in kinds]
     flops_step = sum(prefill_flops(w.B, w.T, L.kind) for L in layers)
 
     def step():
@@ -410,25 +412,31 @@ def run_gpu(args):
     with ClockSampler(torch.cuda.current_device()) as clocks:
         ev_step[0].record(stream)
         for i in range(args.steps):
-            layers[0].run()
-            ev_g[i][0].record(stream)
-            layers[1].run()
-            ev_g[i][1].record(stream)
+            for L in layers:
+                if L.kind == wl.GLOBAL:
+                    ev_g[i][0].record(stream)
+                L.run()
+                if L.kind == wl.GLOBAL:
+                    ev_g[i][1].record(stream)
         ev_step[1].record(stream)
         torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     sec = ev_step[0].elapsed_time(ev_step[1]) / 1e3 / args.steps
-    sec_g = sum(a.elapsed_time(b) for a, b in ev_g) / 1e3 / args.steps
+    has_global = any(L.kind == wl.GLOBAL for L in layers)
+    sec_g = (sum(a.elapsed_time(b) for a, b in ev_g) / 1e3 / args.steps) if has_global else sec
     sec_max = max_over_ranks(sec, "cuda")
     value = aggregate(flops_step, world, sec_max) / 1e12
     for L in layers:
         assert int(L.status.item()) == 0, "device status set during the bench"
 
-    g_flops = prefill_flops(w.B, w.T, wl.GLOBAL)
+    g_flops = prefill_flops(w.B, w.T, wl.GLOBAL) if has_global else flops_step
     achieved = g_flops / sec_g / 1e12
-    e2e_sec, h2d, d2h = e2e_prefill(torch, beam, layers, args.steps, args.warmup)
-    e2e_sec = max_over_ranks(e2e_sec, "cuda")
+    if args.no_e2e:
+        e2e_sec, h2d, d2h = float("nan"), 0, 0
+    else:
+        e2e_sec, h2d, d2h = e2e_prefill(torch, beam, layers, args.steps, args.warmup)
+        e2e_sec = max_over_ranks(e2e_sec, "cuda")
     result = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -442,9 +450,9 @@ def run_gpu(args):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic: N(0,1) bf16 activations drawn on the device (seeded torch Philox)",
-        "config": {"workload": "batched_prefill: B=4, T=8192 per GPU, one local (window 512, RoPE) "
-                               "+ one global (NoPE, SSMax) layer, 48 q / 8 kv heads, d=128, "
-                               "fused KV append",
+        "config": {"workload": f"batched_prefill: B={w.B}, T={w.T} per GPU, layers={args.layers} "
+                               "(local: window 512, RoPE; global: NoPE, SSMax), 48 q / 8 kv heads, "
+                               "d=128, fused KV append",
                    "global_batch": w.B * world, "seq_len": w.T, "parallelism": f"dp{world}",
                    "l2": "inputs larger than L2 (Q alone is 403 MB per layer)"},
         "pct_of_bf16_peak": round(100 * value / world / pk["bf16_tflops"], 2),
@@ -452,8 +460,9 @@ def run_gpu(args):
                      "unit": "TFLOP/s", "frac": round(achieved / pk["bf16_tflops"], 4),
                      "traffic": None, "kernel": "global-layer prefill call (prologue + attention)",
                      "peak_source": pk["source"] + " burst bf16"},
-        "e2e": {"value": round(aggregate(flops_step, world, e2e_sec) / 1e12, 3), "unit": "TFLOP/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "e2e": None if args.no_e2e else {
+            "value": round(aggregate(flops_step, world, e2e_sec) / 1e12, 3), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps * sum(L.launches_per_call for L in layers),
         "clocks": clocks.summary(),
     }
@@ -509,6 +518,10 @@ def main(argv=None):
     ap.add_argument("--seed", type=int, default=1234)
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--layers", default="both", choices=["both", "global", "local"],
+                    help="prefill layers per step (profiling cases; the headline step is both)")
+    ap.add_argument("--batch", type=int, default=0, help="override B (profiling cases)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3

@@ -4,16 +4,20 @@
 // Every call validates its arguments on the host and returns before any launch
 // when they are wrong; kernels are launched on the caller's stream and the call
 // returns without synchronising.  Nothing here allocates device memory.
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include <cmath>
 #include <cstdint>
+#include <cstdio>
+#include <cstdlib>
 #include <cstring>
 
 #include "beam_attn.h"
 #include "common.cuh"
 #include "decode.cuh"
-#include "prefill_mma.cuh"
+#include "prefill_tc.cuh"
 #include "prologue.cuh"
 
 using namespace beam;
@@ -28,20 +32,38 @@ struct DeviceInfo {
 };
 DeviceInfo g_dev[kMaxDevices];
 
+// With BEAM_VERBOSE set in the environment, CUDA failures are also printed to stderr.
+bool verbose() {
+  static const bool v = std::getenv("BEAM_VERBOSE") != nullptr;
+  return v;
+}
+
+int cuda_status(cudaError_t e, const char *what) {
+  if (e == cudaSuccess) return BEAM_OK;
+  if (verbose()) std::fprintf(stderr, "beam_attn: %s: %s\n", what, cudaGetErrorString(e));
+  return BEAM_ERR_CUDA;
+}
+
+
 // Per-device attributes: SM count and the dynamic shared-memory opt-ins.
 int device_info(DeviceInfo **out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BEAM_ERR_CUDA;
   DeviceInfo &d = g_dev[dev];
   if (!d.ready) {
-    if (cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      return BEAM_ERR_CUDA;
-    if (cudaFuncSetAttribute(decode_splitk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kDecSmem) != cudaSuccess)
-      return BEAM_ERR_CUDA;
-    if (cudaFuncSetAttribute(prefill_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kPfSmem) != cudaSuccess)
-      return BEAM_ERR_CUDA;
+    int st;
+    if ((st = cuda_status(cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev),
+                          "SM count")))
+      return st;
+    if ((st = cuda_status(cudaFuncSetAttribute(decode_splitk_kernel,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem),
+                          "decode shared-memory opt-in")))
+      return st;
+    if ((st = cuda_status(cudaFuncSetAttribute(prefill_tc_kernel,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               kTcSmemBytes),
+                          "prefill shared-memory opt-in")))
+      return st;
     d.ready = true;
   }
   *out = &d;
@@ -78,7 +100,37 @@ void fill_inv_freq(double (&f)[64], double theta) {
   for (int i = 0; i < 64; ++i) f[i] = std::pow(theta, -2.0 * i / (double)kD);
 }
 
-int launch_status() { return cudaGetLastError() == cudaSuccess ? BEAM_OK : BEAM_ERR_CUDA; }
+int launch_status() { return cuda_status(cudaGetLastError(), "kernel launch"); }
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link to libcuda).
+PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
+
+int encode_fn() {
+  if (g_encode_tiled) return BEAM_OK;
+  void *fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || !fn)
+    return BEAM_ERR_CUDA;
+  g_encode_tiled = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return BEAM_OK;
+}
+
+// 4-D bf16 map over a token-major activation [B][T][heads][128]: coordinates
+// (d, head, t, b), 128-byte swizzled boxes of 64 d x 1 head x 128 tokens.  Tokens past
+// T read as zeros.
+int make_head_map(CUtensorMap *map, const void *base, int heads, int T, int B) {
+  const cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)heads, (cuuint64_t)T, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)kD * 2, (cuuint64_t)heads * kD * 2,
+                                 (cuuint64_t)T * heads * kD * 2};
+  const cuuint32_t box[4] = {64, 1, (cuuint32_t)kTcBM, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = g_encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base),
+                              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? BEAM_OK : BEAM_ERR_CUDA;
+}
 
 // Decode split size: cache slots per CTA.  A local ring is one split; a global
 // cache is cut so that the grid holds several waves of the SMs at its largest
@@ -213,22 +265,26 @@ int beam_attn_prefill(int kind, const beam_attn_params *p, int32_t B, int32_t T,
   prologue_kernel<<<(unsigned)tok, 128, 0, s>>>(pa);
   if ((st = launch_status())) return st;
 
-  PrefillArgs fa;
-  fa.qn = qn;
-  fa.kn = kn;
-  fa.v = static_cast<const uint16_t *>(v);
+  if ((st = encode_fn())) return st;
+  CUtensorMap tm_q, tm_k, tm_v;
+  if ((st = make_head_map(&tm_q, qn, kHq, T, B))) return st;
+  if ((st = make_head_map(&tm_k, kn, kHkv, T, B))) return st;
+  if ((st = make_head_map(&tm_v, v, kHkv, T, B))) return st;
+  PrefillTcArgs fa;
   fa.gate = static_cast<const uint16_t *>(gate);
   fa.gate_bias = gate_bias;
   fa.out = static_cast<uint16_t *>(out);
+  fa.status = dev_status;
   fa.T = T;
   fa.kind = kind;
   fa.window = p->window;
-  fa.n_qblocks = (T + kPfBM - 1) / kPfBM;
+  fa.n_qblocks = (T + kTcBM - 1) / kTcBM;
   fa.scale_log2 = p->softmax_scale * kLog2e;
   fa.ssmax_base = p->ssmax_base;
   fa.ssmax_exp = p->ssmax_exp;
-  dim3 grid(fa.n_qblocks, kHq, B);
-  prefill_mma_kernel<<<grid, kPfThreads, kPfSmem, s>>>(fa);
+  if (fa.n_qblocks > 65535 || (int64_t)B * (kHq / 2) > INT32_MAX) return BEAM_ERR_UNSUPPORTED;
+  dim3 grid((unsigned)(B * (kHq / 2)), (unsigned)fa.n_qblocks);
+  prefill_tc_kernel<<<grid, kTcThreads, kTcSmemBytes, s>>>(tm_q, tm_k, tm_v, fa);
   return launch_status();
 }
 
