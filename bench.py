@@ -133,12 +133,11 @@ class ClockSampler:
         self.rows.append((sm, reasons))
 
     def _run(self):
-        while not self._stop.is_set():
+        while not self._stop.wait(0.05):
             try:
                 self._sample()
             except Exception:
                 pass
-            self._stop.wait(0.05)
 
     def __enter__(self):
         if self._handle is not None:
@@ -394,12 +393,26 @@ def run_gpu(args):
     layers = [PrefillLayer(torch, beam, kind, w.B, w.T, w.seed, f"bench/{kind}") for kind in kinds]
     flops_step = sum(prefill_flops(w.B, w.T, L.kind) for L in layers)
 
-    def step():
+    # Each layer call is captured once in a CUDA graph and replayed: the timed region is
+    # then a handful of host calls, so nothing on the host can starve the GPU between
+    # kernels (the replays run exactly the kernels a direct call launches).
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
         for L in layers:
             L.run()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graphs = []
+    for L in layers:
+        gph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gph):
+            L.run()
+        graphs.append(gph)
 
     for _ in range(args.warmup):
-        step()
+        for gph in graphs:
+            gph.replay()
     torch.cuda.synchronize()
     # per-call events on the launching stream for the dominant (global) layer
     stream = torch.cuda.current_stream()
@@ -412,10 +425,10 @@ def run_gpu(args):
     with ClockSampler(torch.cuda.current_device()) as clocks:
         ev_step[0].record(stream)
         for i in range(args.steps):
-            for L in layers:
+            for L, gph in zip(layers, graphs):
                 if L.kind == wl.GLOBAL:
                     ev_g[i][0].record(stream)
-                L.run()
+                gph.replay()
                 if L.kind == wl.GLOBAL:
                     ev_g[i][1].record(stream)
         ev_step[1].record(stream)
@@ -466,7 +479,7 @@ def run_gpu(args):
         "gpu_launches": args.steps * sum(L.launches_per_call for L in layers),
         "clocks": clocks.summary(),
     }
-    del layers
+    del graphs, layers
     torch.cuda.empty_cache()
     if rank == 0 and not args.no_decode:
         d1m, _ = bench_decode_1m(torch, beam, args.steps, args.warmup, args.seed)

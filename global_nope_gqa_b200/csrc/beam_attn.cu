@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstdio>
@@ -203,7 +204,8 @@ size_t beam_prefill_workspace_bytes(const beam_attn_params *p, int32_t B, int32_
   (void)p;
   if (B <= 0 || T <= 0) return 0;
   const size_t tok = (size_t)B * T;
-  return round_up(tok * kHq * kD * 2, 256) + round_up(tok * kHkv * kD * 2, 256);
+  // prepared keys [B][T][8][128] bf16, then the RoPE cos/sin table [T][128] fp32
+  return round_up(tok * kHkv * kD * 2, 256) + round_up((size_t)T * 128 * 4, 256);
 }
 
 int beam_attn_prefill(int kind, const beam_attn_params *p, int32_t B, int32_t T, const void *q,
@@ -234,9 +236,9 @@ int beam_attn_prefill(int kind, const beam_attn_params *p, int32_t B, int32_t T,
   if ((st = device_info(&dev))) return st;
 
   const size_t tok = (size_t)B * T;
-  uint16_t *qn = static_cast<uint16_t *>(workspace);
-  uint16_t *kn = reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(workspace) +
-                                              round_up(tok * kHq * kD * 2, 256));
+  uint16_t *kn = static_cast<uint16_t *>(workspace);
+  float *rope_tab = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
+                                              round_up(tok * kHkv * kD * 2, 256));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
 
   PrologueArgs pa;
@@ -246,8 +248,9 @@ int beam_attn_prefill(int kind, const beam_attn_params *p, int32_t B, int32_t T,
   pa.v = static_cast<const uint16_t *>(v);
   pa.qw = q_norm_w;
   pa.kw = k_norm_w;
-  pa.q_out = qn;
+  pa.q_out = nullptr;  // queries are normalised inside the attention kernel
   pa.k_out = kn;
+  pa.rope_tab = kind == BEAM_LOCAL ? rope_tab : nullptr;
   pa.k_cache = static_cast<uint16_t *>(k_cache);
   pa.v_cache = static_cast<uint16_t *>(v_cache);
   if (k_cache) {
@@ -267,14 +270,18 @@ int beam_attn_prefill(int kind, const beam_attn_params *p, int32_t B, int32_t T,
 
   if ((st = encode_fn())) return st;
   CUtensorMap tm_q, tm_k, tm_v;
-  if ((st = make_head_map(&tm_q, qn, kHq, T, B))) return st;
+  if ((st = make_head_map(&tm_q, q, kHq, T, B))) return st;
   if ((st = make_head_map(&tm_k, kn, kHkv, T, B))) return st;
   if ((st = make_head_map(&tm_v, v, kHkv, T, B))) return st;
   PrefillTcArgs fa;
+  fa.q_norm_w = q_norm_w;
+  fa.rope_tab = kind == BEAM_LOCAL ? rope_tab : nullptr;
+  fa.eps = p->rms_eps;
   fa.gate = static_cast<const uint16_t *>(gate);
   fa.gate_bias = gate_bias;
   fa.out = static_cast<uint16_t *>(out);
   fa.status = dev_status;
+  fa.B = B;
   fa.T = T;
   fa.kind = kind;
   fa.window = p->window;
@@ -282,8 +289,11 @@ int beam_attn_prefill(int kind, const beam_attn_params *p, int32_t B, int32_t T,
   fa.scale_log2 = p->softmax_scale * kLog2e;
   fa.ssmax_base = p->ssmax_base;
   fa.ssmax_exp = p->ssmax_exp;
-  if (fa.n_qblocks > 65535 || (int64_t)B * (kHq / 2) > INT32_MAX) return BEAM_ERR_UNSUPPORTED;
-  dim3 grid((unsigned)(B * (kHq / 2)), (unsigned)fa.n_qblocks);
+  const int64_t n_units = (int64_t)fa.n_qblocks * (kHq / 2) * B;
+  if (n_units > INT32_MAX) return BEAM_ERR_UNSUPPORTED;
+  fa.n_units = (int)n_units;
+  // persistent: one CTA per SM (the kernel's shared memory admits one per SM)
+  const int grid = (int)std::min<int64_t>(n_units, dev->sm_count);
   prefill_tc_kernel<<<grid, kTcThreads, kTcSmemBytes, s>>>(tm_q, tm_k, tm_v, fa);
   return launch_status();
 }

@@ -7,9 +7,13 @@
 // Y = O * sigmoid(G + b_h) per coordinate (section "Follow the tensors").  The global
 // layer's scalable-softmax factor a(t+1) multiplies each row's fp32 score scale.
 //
-// One CTA = 128 query rows x two query heads of one GQA group (two 128 x 128 Q tiles that
-// share every K/V tile), 384 threads in warp roles:
-//   warp 0      TMA producer: Q tiles once, then K and V tiles of 128 keys into a
+// Work unit: 128 query rows x two query heads of one GQA group -- two 128 x 128 Q tiles
+// that share every K/V tile.  The kernel is persistent: one CTA per SM walks the units
+// u = blockIdx.x, blockIdx.x + gridDim.x, ... in order of decreasing work (the causal
+// triangle's longest rows first), so the next unit's loads and first Q K^T overlap the
+// current unit's epilogue, and set-up (barriers, tensor memory) happens once.
+// 512 threads in warp roles:
+//   warp 0      TMA producer: Q tiles of each unit, then K and V tiles of 128 keys into a
 //               two-stage ring (128-byte swizzled boxes of 128 rows x 64 columns);
 //   warp 1      MMA issuer (one thread): S_t = Q_t K^T (both operands in shared memory)
 //               and O_t += P_t V (P from tensor memory, V in shared memory), t = 0, 1;
@@ -17,27 +21,33 @@
 //               S_0 [0,128) S_1 [128,256) O_0 [256,384) O_1 [384,512) (fp32), with P_t
 //               written as bf16 pairs over the first 64 columns of S_t;
 //   warps 2-3   idle;
+//   warps 12-15 Q preparation: once a unit's raw Q tiles have landed, RMSNorm (and RoPE
+//               with a per-position cos/sin table for a local layer) each row in place in
+//               shared memory, then release the tiles to the MMA issuer;
 //   warps 4-7   softmax of tile 0, warps 8-11 softmax of tile 1: one thread per query row
-//               (tensor-memory lane = row; warp % 4 picks the lane quarter a warp may use).  Each reads its S row, masks the window /
-//               causal edge, keeps the online max m and sum l in exp2 units, writes P and,
-//               only when the row max grew by more than 2^8, rescales its O row in tensor
-//               memory first (the stale max keeps every P <= 256, safe in fp32 and bf16).
-//               The last block's wait also serves as the epilogue: O/l * sigmoid(G + b).
-// MMAs issued by one thread run in issue order, so S_t(j+1), which overwrites P_t(j),
-// is issued after O_t += P_t(j) V_j; the commit that publishes S_t(j) also covers the
-// O_t update of block j-1, which lets the softmax rescale O_t without a further wait.
-// Key blocks entirely outside the window or the causal triangle are never loaded.
-// Every mbarrier wait is bounded; a wait that runs out sets BEAM_ERR_DEVICE_TIMEOUT in
-// the status word, raises an abort flag that the other roles also watch, and the CTA
-// still frees its tensor memory before it returns.
+//               (tensor-memory lane = row; warp % 4 picks the lane quarter a warp may use).
+//               Each reads its S row, masks the window / causal edge, keeps the online max
+//               m and sum l in exp2 units, writes P and, only when the row max grew by more
+//               than 2^8, rescales its O row in tensor memory (the stale max keeps every
+//               P <= 256, safe in fp32 and bf16).  After a unit's last block the same
+//               threads run the epilogue O/l * sigmoid(G + b) and release O.
+// MMAs issued by one thread run in issue order, so S_t(j+1), which overwrites P_t(j), is
+// issued after O_t += P_t(j) V_j; the commit that publishes S_t(j) also covers the O_t
+// update of block j-1, which lets the softmax rescale O_t without a further wait.  Key
+// blocks entirely outside the window or the causal triangle are never loaded.
+// Every mbarrier wait is bounded; a wait that runs out sets BEAM_ERR_DEVICE_TIMEOUT in the
+// status word, raises an abort flag that the other roles also watch, and the CTA still
+// frees its tensor memory before it returns.
 #pragma once
+
+#include <climits>
 
 #include "common.cuh"
 #include "tc_ptx.cuh"
 
 namespace beam {
 
-constexpr int kTcThreads = 384;
+constexpr int kTcThreads = 512;
 constexpr int kTcBM = 128;      // query rows per tile
 constexpr int kTcBN = 128;      // keys per block
 constexpr uint32_t kTcTileBytes = 128 * 128 * 2;   // 32 KiB: one 128 x 128 bf16 tile
@@ -50,18 +60,21 @@ constexpr uint32_t kTcSmemBytes = kTcSmemBar + 256 + 1024;  // + barriers + alig
 constexpr uint32_t kTcSpinLimit = 1u << 22;
 
 struct PrefillTcArgs {
+  const float *q_norm_w;  // [128]
+  const float *rope_tab;  // local: [T][128] cos then sin of position t; null for global
+  float eps;
   const uint16_t *gate;   // [B][T][48*128]
   const float *gate_bias; // [48]
   uint16_t *out;          // [B][T][48*128]
   int32_t *status;
-  int T, kind, window, n_qblocks;
+  int B, T, kind, window, n_qblocks, n_units;
   float scale_log2, ssmax_base, ssmax_exp;
 };
 
 namespace tcd {
 // barrier slots (8 bytes each) after kTcSmemBar
-constexpr int kQFull = 0, kKFull = 1, kVFull = 3, kKVEmpty = 5, kSFull = 7, kPFull = 9,
-              kOFull = 11, kNumBars = 13;
+constexpr int kQFull = 0, kQEmpty = 1, kKFull = 2, kVFull = 4, kKVEmpty = 6, kSFull = 8,
+              kPFull = 10, kOFull = 12, kOEmpty = 14, kQReady = 16, kNumBars = 17;
 constexpr uint32_t kTmemHolder = kNumBars * 8;      // u32: tensor-memory base address
 constexpr uint32_t kAbortFlag = kTmemHolder + 4;    // u32: set when a wait ran out
 }  // namespace tcd
@@ -69,6 +82,11 @@ constexpr uint32_t kAbortFlag = kTmemHolder + 4;    // u32: set when a wait ran 
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;\n" : "=f"(y) : "f"(x));
   return y;
 }
 
@@ -84,6 +102,24 @@ __device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity, volatile 
   return false;
 }
 
+// Work unit u -> (q block, head pair, sequence); units with more key blocks come first.
+struct TcUnit {
+  int qb, pair, b, q0, kb_lo, n_blk;
+};
+__device__ __forceinline__ TcUnit tc_unit(const PrefillTcArgs &a, int u) {
+  TcUnit w;
+  const int per_qb = (kHq / 2) * a.B;
+  const int idx = u / per_qb;
+  w.qb = a.n_qblocks - 1 - idx;
+  const int rem = u - idx * per_qb;
+  w.pair = rem % (kHq / 2);
+  w.b = rem / (kHq / 2);
+  w.q0 = w.qb * kTcBM;
+  w.kb_lo = a.kind == BEAM_LOCAL ? max(0, w.q0 - a.window + 1) / kTcBN : 0;
+  w.n_blk = w.qb - w.kb_lo + 1;  // the last visible key of the unit is in block qb
+  return w;
+}
+
 __global__ void __launch_bounds__(kTcThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
@@ -97,19 +133,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   auto bar = [&](int i) { return bars + 8u * (uint32_t)i; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int pair = blockIdx.x % (kHq / 2), b = blockIdx.x / (kHq / 2);
-  const int qb = a.n_qblocks - 1 - (int)blockIdx.y;  // longest rows first
-  const int h0 = 2 * pair, g = h0 / kGroup;
-  const int q0 = qb * kTcBM;
   const bool local = a.kind == BEAM_LOCAL;
-  const int kb_lo = local ? max(0, q0 - a.window + 1) / kTcBN : 0;
-  const int kb_hi = qb;  // q_last = min(T, q0 + 128) - 1 < (qb + 1) * 128
-  const int n_blk = kb_hi - kb_lo + 1;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < tcd::kNumBars; ++i) {
       uint32_t count = 1;
-      if (i == tcd::kPFull || i == tcd::kPFull + 1) count = 128;
+      if (i == tcd::kPFull || i == tcd::kPFull + 1 || i == tcd::kOEmpty || i == tcd::kOEmpty + 1 ||
+          i == tcd::kQReady)
+        count = 128;
       tc::mbar_init(bar(i), count);
     }
     *abort = 0u;
@@ -124,9 +155,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc::tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sgen + kTcSmemBar + tcd::kTmemHolder);
 
-  // Register split (per warpgroup): warps 0-3 (producer, MMA issuer, two idle) keep 56
-  // registers, the softmax warpgroups get 224: 4*56 + 8*224 = 12*168, what the CTA is
-  // launched with, and on every SM sub-partition 56 + 2*224 <= 512 registers per lane.
+  // Register split (per warpgroup) of the 512 x 128 registers the CTA is launched with:
+  // warps 0-3 (producer, MMA issuer, two idle) keep 56, the Q-preparation warpgroup
+  // (warps 12-15) 104, the two softmax warpgroups 176: 128*(56 + 104) + 256*176 = 65536,
+  // and on every SM sub-partition 56 + 104 + 2*176 = 512 registers per lane.
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     asm volatile("setmaxnreg.dec.sync.aligned.u32 56;\n" ::: "memory");
@@ -134,23 +166,32 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc::prefetch_tmap(&tm_q);
       tc::prefetch_tmap(&tm_k);
       tc::prefetch_tmap(&tm_v);
-      tc::mbar_expect_tx(bar(tcd::kQFull), 2 * kTcTileBytes);
-      for (int t = 0; t < 2; ++t)
-        for (int hf = 0; hf < 2; ++hf)
-          tc::tma_load_4d(sbase + kTcSmemQ + t * kTcTileBytes + hf * kTcHalfBytes, &tm_q,
-                          bar(tcd::kQFull), hf * 64, h0 + t, q0, b);
-      for (int j = 0; j < n_blk; ++j) {
-        const int s = j & 1;
-        if (j >= 2 && !tc_wait(bar(tcd::kKVEmpty + s), ((j >> 1) - 1) & 1, abort, a.status)) break;
-        const int key0 = (kb_lo + j) * kTcBN;
-        tc::mbar_expect_tx(bar(tcd::kKFull + s), kTcTileBytes);
-        for (int hf = 0; hf < 2; ++hf)
-          tc::tma_load_4d(sbase + kTcSmemK + s * kTcTileBytes + hf * kTcHalfBytes, &tm_k,
-                          bar(tcd::kKFull + s), hf * 64, g, key0, b);
-        tc::mbar_expect_tx(bar(tcd::kVFull + s), kTcTileBytes);
-        for (int hf = 0; hf < 2; ++hf)
-          tc::tma_load_4d(sbase + kTcSmemV + s * kTcTileBytes + hf * kTcHalfBytes, &tm_v,
-                          bar(tcd::kVFull + s), hf * 64, g, key0, b);
+      uint32_t it = 0;  // K/V blocks loaded so far (ring position)
+      bool ok = true;
+      for (int u = blockIdx.x, n = 0; ok && u < a.n_units; u += gridDim.x, ++n) {
+        const TcUnit w = tc_unit(a, u);
+        const int h0 = 2 * w.pair, g = h0 / kGroup;
+        if (n > 0 && !(ok = tc_wait(bar(tcd::kQEmpty), (n - 1) & 1, abort, a.status))) break;
+        tc::mbar_expect_tx(bar(tcd::kQFull), 2 * kTcTileBytes);
+        for (int t = 0; t < 2; ++t)
+          for (int hf = 0; hf < 2; ++hf)
+            tc::tma_load_4d(sbase + kTcSmemQ + t * kTcTileBytes + hf * kTcHalfBytes, &tm_q,
+                            bar(tcd::kQFull), hf * 64, h0 + t, w.q0, w.b);
+        for (int j = 0; j < w.n_blk; ++j, ++it) {
+          const uint32_t s = it & 1u;
+          if (it >= 2 &&
+              !(ok = tc_wait(bar(tcd::kKVEmpty + s), ((it >> 1) - 1) & 1u, abort, a.status)))
+            break;
+          const int key0 = (w.kb_lo + j) * kTcBN;
+          tc::mbar_expect_tx(bar(tcd::kKFull + s), kTcTileBytes);
+          for (int hf = 0; hf < 2; ++hf)
+            tc::tma_load_4d(sbase + kTcSmemK + s * kTcTileBytes + hf * kTcHalfBytes, &tm_k,
+                            bar(tcd::kKFull + s), hf * 64, g, key0, w.b);
+          tc::mbar_expect_tx(bar(tcd::kVFull + s), kTcTileBytes);
+          for (int hf = 0; hf < 2; ++hf)
+            tc::tma_load_4d(sbase + kTcSmemV + s * kTcTileBytes + hf * kTcHalfBytes, &tm_v,
+                            bar(tcd::kVFull + s), hf * 64, g, key0, w.b);
+        }
       }
     }
     __syncwarp();
@@ -166,184 +207,306 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       auto v_desc = [&](uint32_t tile, int kk) {  // MN-major: d halves 16 KiB apart
         return tc::sdesc_sw128(tile + kk * 2048, kTcHalfBytes, 1024);
       };
-      auto issue_pv = [&](int t, int jb) {
-        const uint32_t vt = sbase + kTcSmemV + (jb & 1) * kTcTileBytes;
+      // O_t += P_t V for K/V ring position `pos`; `first` overwrites O_t.
+      auto issue_pv = [&](int t, uint32_t pos, bool first) {
+        const uint32_t vt = sbase + kTcSmemV + (pos & 1u) * kTcTileBytes;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           tc::umma_ts(tmem + 256 + 128 * t, tmem + 128 * t + kk * 8, v_desc(vt, kk), idesc_pv,
-                      (jb > 0 || kk > 0) ? 1u : 0u);
+                      (!first || kk > 0) ? 1u : 0u);
       };
-      bool ok = tc_wait(bar(tcd::kQFull), 0, abort, a.status);
-      for (int j = 0; ok && j < n_blk; ++j) {
-        const int s = j & 1;
-        if (!(ok = tc_wait(bar(tcd::kKFull + s), (j >> 1) & 1, abort, a.status))) break;
-        tc::tc_fence_after();
-        const uint32_t kt = sbase + kTcSmemK + s * kTcTileBytes;
-        for (int t = 0; t < 2 && ok; ++t) {
-          if (j > 0) {
-            if (!(ok = tc_wait(bar(tcd::kPFull + t), (j - 1) & 1, abort, a.status))) break;
-            if (t == 0 &&
-                !(ok = tc_wait(bar(tcd::kVFull + ((j - 1) & 1)), ((j - 1) >> 1) & 1, abort, a.status)))
-              break;
-            tc::tc_fence_after();
-            issue_pv(t, j - 1);
-            if (t == 1) tc::umma_commit(bar(tcd::kKVEmpty + ((j - 1) & 1)));
-          }
-          const uint32_t qt = sbase + kTcSmemQ + t * kTcTileBytes;
+      uint32_t it = 0;  // K/V ring position of the current block
+      bool ok = true;
+      for (int u = blockIdx.x, n = 0; ok && u < a.n_units; u += gridDim.x, ++n) {
+        const TcUnit w = tc_unit(a, u);
+        if (!(ok = tc_wait(bar(tcd::kQReady), n & 1, abort, a.status))) break;
+        // step j: O_t += P_t(j-1) V(j-1) (j > 0), then S_t(j) = Q_t K(j)^T (j < n_blk)
+        for (int j = 0; ok && j <= w.n_blk; ++j) {
+          const bool has_s = j < w.n_blk;
+          const uint32_t s = it & 1u;
+          if (has_s && !(ok = tc_wait(bar(tcd::kKFull + s), (it >> 1) & 1u, abort, a.status)))
+            break;
+          tc::tc_fence_after();
+          const uint32_t kt = sbase + kTcSmemK + s * kTcTileBytes;
+          for (int t = 0; t < 2 && ok; ++t) {
+            if (j > 0) {
+              const uint32_t prev = it - 1;
+              if (!(ok = tc_wait(bar(tcd::kPFull + t), prev & 1u, abort, a.status))) break;
+              if (t == 0 && !(ok = tc_wait(bar(tcd::kVFull + (prev & 1u)), (prev >> 1) & 1u,
+                                           abort, a.status)))
+                break;
+              // the first P V of a unit overwrites O_t: the previous epilogue must be done
+              if (j == 1 && n > 0 &&
+                  !(ok = tc_wait(bar(tcd::kOEmpty + t), (n - 1) & 1, abort, a.status)))
+                break;
+              tc::tc_fence_after();
+              issue_pv(t, prev, j == 1);
+              if (t == 1) tc::umma_commit(bar(tcd::kKVEmpty + (prev & 1u)));
+              if (!has_s) tc::umma_commit(bar(tcd::kOFull + t));
+            }
+            if (has_s) {
+              const uint32_t qt = sbase + kTcSmemQ + t * kTcTileBytes;
 #pragma unroll
-          for (int ks = 0; ks < 8; ++ks)
-            tc::umma_ss(tmem + 128 * t, qk_desc(qt, ks), qk_desc(kt, ks), idesc_qk, ks > 0 ? 1u : 0u);
-          tc::umma_commit(bar(tcd::kSFull + t));
+              for (int ks = 0; ks < 8; ++ks)
+                tc::umma_ss(tmem + 128 * t, qk_desc(qt, ks), qk_desc(kt, ks), idesc_qk,
+                            ks > 0 ? 1u : 0u);
+              tc::umma_commit(bar(tcd::kSFull + t));
+              if (t == 1 && j == w.n_blk - 1) tc::umma_commit(bar(tcd::kQEmpty));
+            }
+          }
+          if (has_s) ++it;
         }
-      }
-      const int jl = n_blk - 1;
-      for (int t = 0; t < 2 && ok; ++t) {
-        if (!(ok = tc_wait(bar(tcd::kPFull + t), jl & 1, abort, a.status))) break;
-        if (t == 0 && !(ok = tc_wait(bar(tcd::kVFull + (jl & 1)), (jl >> 1) & 1, abort, a.status)))
-          break;
-        tc::tc_fence_after();
-        issue_pv(t, jl);
-        tc::umma_commit(bar(tcd::kOFull + t));
       }
     }
     __syncwarp();
   } else if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 56;\n" ::: "memory");
+  } else if (warp >= 12) {
+    // ------------------------------------------------------------ Q preparation
+    // RMSNorm of each raw Q row in shared memory (in place), then RoPE for a local layer;
+    // thread r owns row r of both tiles (same position, so the same angles).  The cos/sin
+    // values of a row are fetched ahead: chunks 0-1 before the Q tiles land, chunk c + 2
+    // as soon as chunk c is done.
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 104;\n" ::: "memory");
+    const int r = threadIdx.x - 384;
+    const float4 *w4 = reinterpret_cast<const float4 *>(a.q_norm_w);
+    bool ok = true;
+    for (int u = blockIdx.x, n = 0; ok && u < a.n_units; u += gridDim.x, ++n) {
+      const TcUnit w = tc_unit(a, u);
+      const int tok = w.q0 + r;
+      const float4 *tab =
+          local ? reinterpret_cast<const float4 *>(a.rope_tab + (size_t)min(tok, a.T - 1) * 128)
+                : nullptr;
+      float4 tb[8];   // per slot: cos lo, cos hi, sin lo, sin hi of one chunk of 8
+      auto tab_load = [&](int c, int slot) {
+        tb[4 * slot + 0] = __ldg(tab + 2 * c);
+        tb[4 * slot + 1] = __ldg(tab + 2 * c + 1);
+        tb[4 * slot + 2] = __ldg(tab + 16 + 2 * c);
+        tb[4 * slot + 3] = __ldg(tab + 16 + 2 * c + 1);
+      };
+      if (local) {
+        tab_load(0, 0);
+        tab_load(1, 1);
+      }
+      if (!(ok = tc_wait(bar(tcd::kQFull), n & 1, abort, a.status))) break;
+      auto chunk = [&](int t, int hf, int c) -> uint4 * {   // 8 bf16 at d = 64 hf + 8 c
+        return reinterpret_cast<uint4 *>(sgen + kTcSmemQ + t * kTcTileBytes + r * 128 +
+                                         hf * kTcHalfBytes + ((c ^ (r & 7)) << 4));
+      };
+      float inv[2];
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        float ss = 0.f;
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint4 v = *chunk(t, hf, c);
+            const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float x0 = bf16_lo(vw[e]), x1 = bf16_hi(vw[e]);
+              ss = fmaf(x0, x0, fmaf(x1, x1, ss));
+            }
+          }
+        inv[t] = rsqrtf(ss * (1.0f / kD) + a.eps);
+      }
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const int slot = c & 1;
+        const float4 wl0 = __ldg(w4 + 2 * c), wl1 = __ldg(w4 + 2 * c + 1);
+        const float4 wh0 = __ldg(w4 + 16 + 2 * c), wh1 = __ldg(w4 + 16 + 2 * c + 1);
+        const float wl[8] = {wl0.x, wl0.y, wl0.z, wl0.w, wl1.x, wl1.y, wl1.z, wl1.w};
+        const float wh[8] = {wh0.x, wh0.y, wh0.z, wh0.w, wh1.x, wh1.y, wh1.z, wh1.w};
+        float cv[8], sv[8];
+        if (local) {
+          const float4 c0 = tb[4 * slot], c1 = tb[4 * slot + 1];
+          const float4 s0 = tb[4 * slot + 2], s1 = tb[4 * slot + 3];
+          cv[0] = c0.x; cv[1] = c0.y; cv[2] = c0.z; cv[3] = c0.w;
+          cv[4] = c1.x; cv[5] = c1.y; cv[6] = c1.z; cv[7] = c1.w;
+          sv[0] = s0.x; sv[1] = s0.y; sv[2] = s0.z; sv[3] = s0.w;
+          sv[4] = s1.x; sv[5] = s1.y; sv[6] = s1.z; sv[7] = s1.w;
+          if (c < 6) tab_load(c + 2, slot);
+        }
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          const uint4 lo = *chunk(t, 0, c), hi = *chunk(t, 1, c);
+          const uint32_t lw[4] = {lo.x, lo.y, lo.z, lo.w}, hw[4] = {hi.x, hi.y, hi.z, hi.w};
+          float xl[8], xh[8];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            xl[2 * e] = bf16_lo(lw[e]) * inv[t] * wl[2 * e];
+            xl[2 * e + 1] = bf16_hi(lw[e]) * inv[t] * wl[2 * e + 1];
+            xh[2 * e] = bf16_lo(hw[e]) * inv[t] * wh[2 * e];
+            xh[2 * e + 1] = bf16_hi(hw[e]) * inv[t] * wh[2 * e + 1];
+          }
+          if (local) {  // rotate-half: coordinate i < 64 pairs with i + 64
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float a0 = xl[e], b0 = xh[e];
+              xl[e] = a0 * cv[e] - b0 * sv[e];
+              xh[e] = b0 * cv[e] + a0 * sv[e];
+            }
+          }
+          *chunk(t, 0, c) = make_uint4(pack_bf16(xl[0], xl[1]), pack_bf16(xl[2], xl[3]),
+                                       pack_bf16(xl[4], xl[5]), pack_bf16(xl[6], xl[7]));
+          *chunk(t, 1, c) = make_uint4(pack_bf16(xh[0], xh[1]), pack_bf16(xh[2], xh[3]),
+                                       pack_bf16(xh[4], xh[5]), pack_bf16(xh[6], xh[7]));
+        }
+      }
+      // generic-proxy writes -> visible to the tensor cores' async proxy, then publish
+      asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+      tc::mbar_arrive(bar(tcd::kQReady));
+    }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 224;\n" ::: "memory");
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 176;\n" ::: "memory");
     const int t = (warp - 4) >> 2;      // tile: 0 for warps 4-7, 1 for warps 8-11
     const int wq = warp & 3;            // tensor-memory lane quarter this warp may access
     const int r = wq * 32 + lane;       // query row within the tile
-    const int tok = q0 + r;
-    const int h = h0 + t;
-    float factor = a.scale_log2;
-    if (!local) factor *= ssmax_factor((int64_t)tok + 1, a.ssmax_base, a.ssmax_exp);
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const uint32_t t_s = tmem + lane_off + 128 * t;
     const uint32_t t_o = tmem + lane_off + 256 + 128 * t;
-    float m = -INFINITY, l = 0.f;
+    uint32_t it = 0;  // blocks processed so far (barrier phases)
     bool ok = true;
-    for (int j = 0; j < n_blk; ++j) {
-      if (!(ok = tc_wait(bar(tcd::kSFull + t), j & 1, abort, a.status))) break;
-      tc::tc_fence_after();
-      uint32_t sr[4][32];
+    for (int u = blockIdx.x, n = 0; ok && u < a.n_units; u += gridDim.x, ++n) {
+      const TcUnit w = tc_unit(a, u);
+      const int tok = w.q0 + r;
+      const int h = 2 * w.pair + t;
+      float factor = a.scale_log2;
+      if (!local) factor *= ssmax_factor((int64_t)tok + 1, a.ssmax_base, a.ssmax_exp);
+      float m = -INFINITY, l = 0.f;
+      for (int j = 0; j < w.n_blk; ++j, ++it) {
+        if (!(ok = tc_wait(bar(tcd::kSFull + t), it & 1u, abort, a.status))) break;
+        tc::tc_fence_after();
+        uint32_t sr[4][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tc::tmem_ld32(t_s + 32 * c, sr[c]);
-      tc::tmem_ld_wait();
-      const int kb = kb_lo + j;
-      const bool need_mask =
-          kb == qb || (local && (q0 + kTcBM - 1) - kb * kTcBN > a.window - 1);
-      if (need_mask) {
-        // key kb*128 + i is visible to row tok iff lo <= i <= hi
-        const int hi = tok - kb * kTcBN;
-        const int lo = local ? tok - a.window + 1 - kb * kTcBN : INT_MIN;
+        for (int c = 0; c < 4; ++c) tc::tmem_ld32(t_s + 32 * c, sr[c]);
+        tc::tmem_ld_wait();
+        const int kb = w.kb_lo + j;
+        const bool need_mask =
+            kb == w.qb || (local && (w.q0 + kTcBM - 1) - kb * kTcBN > a.window - 1);
+        if (need_mask) {
+          // key kb*128 + i is visible to row tok iff lo <= i <= hi
+          const int hi = tok - kb * kTcBN;
+          const int lo = local ? tok - a.window + 1 - kb * kTcBN : INT_MIN;
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int kk = c * 32 + i;
+              sr[c][i] = (kk >= lo && kk <= hi) ? sr[c][i] : 0xFF800000u;  // -inf
+            }
+        }
+        // row max of the raw scores: eight independent chains of 3-input max
+        float mc[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) mc[q] = __uint_as_float(sr[q >> 1][(q & 1) * 16]);
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int kk = c * 32 + i;
-            sr[c][i] = (kk >= lo && kk <= hi) ? sr[c][i] : 0xFF800000u;  // -inf
+          for (int i = 0; i < 32; i += 2) {
+            const int q = (c * 2 + (i >> 4)) & 7;
+            mc[q] = tc::max3f(mc[q], __uint_as_float(sr[c][i]), __uint_as_float(sr[c][i + 1]));
           }
-      }
-      // row max of the raw scores: eight independent chains of 3-input max
-      float mc[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) mc[q] = __uint_as_float(sr[q >> 1][(q & 1) * 16]);
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const int q = (c * 2 + (i >> 4)) & 7;
-          mc[q] = tc::max3f(mc[q], __uint_as_float(sr[c][i]), __uint_as_float(sr[c][i + 1]));
+        const float mx = tc::max3f(tc::max3f(mc[0], mc[1], mc[2]), tc::max3f(mc[3], mc[4], mc[5]),
+                                   fmaxf(mc[6], mc[7])) * factor;   // factor > 0
+        bool rescale;
+        float m_new;
+        if (j == 0) {
+          rescale = false;
+          m_new = mx;
+        } else {
+          rescale = mx > m + 8.0f;
+          m_new = rescale ? mx : m;
         }
-      const float mx = tc::max3f(tc::max3f(mc[0], mc[1], mc[2]), tc::max3f(mc[3], mc[4], mc[5]),
-                             fmaxf(mc[6], mc[7])) * factor;   // factor > 0
-      bool rescale;
-      float m_new;
-      if (j == 0) {
-        rescale = false;
-        m_new = mx;
-      } else {
-        rescale = mx > m + 8.0f;
-        m_new = rescale ? mx : m;
-      }
-      const float alpha = rescale ? ex2_approx(m - m_new) : 1.0f;
-      m = m_new;
-      const float m_use = m == -INFINITY ? 0.f : m;
-      // P = exp2(s * factor - m) in fp32 pairs; bf16 pairs over the first 64 columns of S
-      const uint64_t f2 = tc::f2_pack(factor, factor), nm2 = tc::f2_pack(-m_use, -m_use);
-      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float y0, y1;
-          tc::f2_unpack(tc::f2_fma(tc::f2_pack(__uint_as_float(sr[c][i]), __uint_as_float(sr[c][i + 1])),
-                                   f2, nm2), y0, y1);
-          const float p0 = ex2_approx(y0), p1 = ex2_approx(y1);
-          acc[(i >> 1) & 3] = tc::f2_add(acc[(i >> 1) & 3], tc::f2_pack(p0, p1));
-          pk[i >> 1] = pack_bf16(p0, p1);
-        }
-        tc::tmem_st16(t_s + 16 * c, pk);
-      }
-      {
-        float s0, s1, s2, s3, s4, s5, s6, s7;
-        tc::f2_unpack(acc[0], s0, s1);
-        tc::f2_unpack(acc[1], s2, s3);
-        tc::f2_unpack(acc[2], s4, s5);
-        tc::f2_unpack(acc[3], s6, s7);
-        l = l * alpha + (((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7)));
-      }
-      // O *= alpha for the rows whose max moved by more than 2^8 (O is final through
-      // the previous block: the commit that published S covers that MMA)
-      if (j > 0 && __any_sync(0xffffffffu, rescale)) {
+        const float alpha = rescale ? ex2_approx(m - m_new) : 1.0f;
+        m = m_new;
+        const float m_use = m == -INFINITY ? 0.f : m;
+        // P = exp2(s * factor - m) in fp32 pairs; bf16 pairs over the first 64 columns of S
+        const uint64_t f2 = tc::f2_pack(factor, factor), nm2 = tc::f2_pack(-m_use, -m_use);
+        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          uint32_t o[32];
-          tc::tmem_ld32(t_o + 32 * c, o);
-          tc::tmem_ld_wait();
+          uint32_t pk[16];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tc::tmem_st32(t_o + 32 * c, o);
+          for (int i = 0; i < 32; i += 2) {
+            float y0, y1;
+            tc::f2_unpack(tc::f2_fma(tc::f2_pack(__uint_as_float(sr[c][i]),
+                                                 __uint_as_float(sr[c][i + 1])),
+                                     f2, nm2),
+                          y0, y1);
+            const float p0 = ex2_approx(y0), p1 = ex2_approx(y1);
+            acc[(i >> 1) & 3] = tc::f2_add(acc[(i >> 1) & 3], tc::f2_pack(p0, p1));
+            pk[i >> 1] = pack_bf16(p0, p1);
+          }
+          tc::tmem_st16(t_s + 16 * c, pk);
         }
+        {
+          float s0, s1, s2, s3, s4, s5, s6, s7;
+          tc::f2_unpack(acc[0], s0, s1);
+          tc::f2_unpack(acc[1], s2, s3);
+          tc::f2_unpack(acc[2], s4, s5);
+          tc::f2_unpack(acc[3], s6, s7);
+          l = l * alpha + (((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7)));
+        }
+        // O *= alpha for the rows whose max moved by more than 2^8 (O is final through
+        // the previous block: the commit that published S covers that MMA)
+        if (j > 0 && __any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[32];
+            tc::tmem_ld32(t_o + 32 * c, o);
+            tc::tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tc::tmem_st32(t_o + 32 * c, o);
+          }
+        }
+        tc::tmem_st_wait();
+        tc::tc_fence_before();
+        tc::mbar_arrive(bar(tcd::kPFull + t));
       }
-      tc::tmem_st_wait();
-      tc::tc_fence_before();
-      tc::mbar_arrive(bar(tcd::kPFull + t));
-    }
-    if (ok) ok = tc_wait(bar(tcd::kOFull + t), 0, abort, a.status);
-    if (ok) {
-      tc::tc_fence_after();
-      const float inv = 1.0f / l;
-      const float bias = a.gate_bias[h];
+      if (!ok) break;
+      // ---- epilogue: Y = O / l * sigmoid(G + b_h), sigmoid(x) = (1 + tanh(x/2)) / 2.
+      // The gate row is fetched before the wait for the last P V, to hide its latency.
       const bool valid = tok < a.T;
-      const size_t row = ((size_t)b * a.T + (valid ? tok : 0)) * (kHq * kD) + (size_t)h * kD;
+      const size_t row = ((size_t)w.b * a.T + (valid ? tok : 0)) * (kHq * kD) + (size_t)h * kD;
+      uint4 gr[16];
+      {
+        const uint4 *gp = reinterpret_cast<const uint4 *>(a.gate + row);
+#pragma unroll
+        for (int q = 0; q < 16; ++q) gr[q] = valid ? __ldg(gp + q) : make_uint4(0u, 0u, 0u, 0u);
+      }
+      if (!(ok = tc_wait(bar(tcd::kOFull + t), n & 1, abort, a.status))) break;
+      tc::tc_fence_after();
+      const float inv = 0.5f / l;
+      const float hb = 0.5f * a.gate_bias[h];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t o[32];
         tc::tmem_ld32(t_o + 32 * c, o);
         tc::tmem_ld_wait();
         if (valid) {
-          const uint4 *gp = reinterpret_cast<const uint4 *>(a.gate + row + c * 32);
           uint4 *op = reinterpret_cast<uint4 *>(a.out + row + c * 32);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const uint4 gr = gp[q];
-            const uint32_t gw[4] = {gr.x, gr.y, gr.z, gr.w};
+            const uint4 g4 = gr[4 * c + q];
+            const uint32_t gw[4] = {g4.x, g4.y, g4.z, g4.w};
             uint32_t yw[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const float g0 = bf16_lo(gw[e]) + bias, g1 = bf16_hi(gw[e]) + bias;
-              const float y0 = __uint_as_float(o[q * 8 + 2 * e]) * inv / (1.0f + __expf(-g0));
-              const float y1 = __uint_as_float(o[q * 8 + 2 * e + 1]) * inv / (1.0f + __expf(-g1));
-              yw[e] = pack_bf16(y0, y1);
+              const float s0 = 1.0f + tanh_approx(fmaf(0.5f, bf16_lo(gw[e]), hb));
+              const float s1 = 1.0f + tanh_approx(fmaf(0.5f, bf16_hi(gw[e]), hb));
+              yw[e] = pack_bf16(__uint_as_float(o[q * 8 + 2 * e]) * inv * s0,
+                                __uint_as_float(o[q * 8 + 2 * e + 1]) * inv * s1);
             }
             op[q] = make_uint4(yw[0], yw[1], yw[2], yw[3]);
           }
         }
       }
+      tc::tc_fence_before();
+      tc::mbar_arrive(bar(tcd::kOEmpty + t));
     }
   }
 

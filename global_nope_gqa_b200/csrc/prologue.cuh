@@ -32,6 +32,7 @@ struct PrologueArgs {
   uint16_t *v_cache;
   int64_t stride_seq, stride_head, slots;
   const int64_t *pos0;   // device [B]: position of token 0 of each sequence, or null (= 0)
+  float *rope_tab;       // local layers, or null: [T][128] cos (64) then sin (64) of token i
   int32_t *status;
   int T;                 // tokens per sequence in this call
   int kind;
@@ -83,6 +84,15 @@ __global__ void __launch_bounds__(128) prologue_kernel(const PrologueArgs a) {
 
   float cs[8], sn[8];
   if (local) rope_angles(a, t < 0 ? 0 : t, l16 & 7, cs, sn);
+  if (local && a.rope_tab && b == 0 && warp == 0 && lane < 8) {
+    // the same angles serve every head and sequence (positions 0 .. T-1): one table row
+    float4 *c4 = reinterpret_cast<float4 *>(a.rope_tab + (size_t)i * 128 + lane * 8);
+    float4 *s4 = reinterpret_cast<float4 *>(a.rope_tab + (size_t)i * 128 + 64 + lane * 8);
+    c4[0] = make_float4(cs[0], cs[1], cs[2], cs[3]);
+    c4[1] = make_float4(cs[4], cs[5], cs[6], cs[7]);
+    s4[0] = make_float4(sn[0], sn[1], sn[2], sn[3]);
+    s4[1] = make_float4(sn[4], sn[5], sn[6], sn[7]);
+  }
 
   float wq[8], wk[8];
   {

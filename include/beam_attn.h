@@ -111,8 +111,9 @@ typedef struct {
 BEAM_API int beam_kv_layout(int kind, const beam_attn_params *p, int32_t batch, int64_t capacity_tokens,
                    beam_kv_layout_t *out);
 
-/* Workspace the prefill call needs for B sequences of T tokens (bytes; the
- * normalised Q and K in bf16).  16-byte aligned workspace required. */
+/* Workspace the prefill call needs for B sequences of T tokens (bytes): the
+ * normalised (local: rotated) keys in bf16 and a table of the RoPE cos/sin values
+ * of positions 0 .. T-1.  16-byte aligned workspace required. */
 BEAM_API size_t beam_prefill_workspace_bytes(const beam_attn_params *p, int32_t B, int32_t T);
 
 /* Prefill of one layer: B sequences of T new tokens at positions 0 .. T-1.
