@@ -13,14 +13,16 @@
 // triangle's longest rows first), so the next unit's loads and first Q K^T overlap the
 // current unit's epilogue, and set-up (barriers, tensor memory) happens once.
 // 512 threads in warp roles:
-//   warp 0      TMA producer: Q tiles of each unit, then K and V tiles of 128 keys into a
-//               two-stage ring (128-byte swizzled boxes of 128 rows x 64 columns);
+//   warp 0      K/V producer (TMA): K and V tiles of 128 keys into a three-slot ring
+//               (128-byte swizzled boxes of 128 rows x 64 columns);
 //   warp 1      MMA issuer (one thread): S_t = Q_t K^T (both operands in shared memory)
 //               and O_t += P_t V (P from tensor memory, V in shared memory), t = 0, 1;
 //               the whole warp also allocates and frees the 512 tensor-memory columns:
 //               S_0 [0,128) S_1 [128,256) O_0 [256,384) O_1 [384,512) (fp32), with P_t
 //               written as bf16 pairs over the first 64 columns of S_t;
-//   warps 2-3   idle;
+//   warp 2      Q producer (TMA): the raw Q tiles of unit n into Q set n % 2, so the next
+//               unit's Q is loaded and prepared while the current unit runs;
+//   warp 3      idle;
 //   warps 12-15 Q preparation: once a unit's raw Q tiles have landed, RMSNorm (and RoPE
 //               with a per-position cos/sin table for a local layer) each row in place in
 //               shared memory, then release the tiles to the MMA issuer;
@@ -52,11 +54,11 @@ constexpr int kTcBM = 128;      // query rows per tile
 constexpr int kTcBN = 128;      // keys per block
 constexpr uint32_t kTcTileBytes = 128 * 128 * 2;   // 32 KiB: one 128 x 128 bf16 tile
 constexpr uint32_t kTcHalfBytes = kTcTileBytes / 2;  // one 128 x 64 TMA box
-constexpr uint32_t kTcSmemQ = 0;                      // Q_0, Q_1
-constexpr uint32_t kTcSmemK = 2 * kTcTileBytes;       // K stage 0, 1
-constexpr uint32_t kTcSmemV = 4 * kTcTileBytes;       // V stage 0, 1
-constexpr uint32_t kTcSmemBar = 6 * kTcTileBytes;     // mbarriers
-constexpr uint32_t kTcSmemBytes = kTcSmemBar + 256 + 1024;  // + barriers + alignment slack
+constexpr uint32_t kTcSmemQ = 0;                      // Q: 2 sets (units n even / odd) x 2 tiles
+constexpr uint32_t kTcSmemKV = 4 * kTcTileBytes;      // K/V ring: 3 slots of one 128 x 128 tile
+constexpr uint32_t kTcKVSlots = 3;
+constexpr uint32_t kTcSmemBar = kTcSmemKV + kTcKVSlots * kTcTileBytes;  // mbarriers
+constexpr uint32_t kTcSmemBytes = kTcSmemBar + 256 + 1024;  // 230,656 B: barriers + alignment slack
 constexpr uint32_t kTcSpinLimit = 1u << 22;
 
 struct PrefillTcArgs {
@@ -73,8 +75,8 @@ struct PrefillTcArgs {
 
 namespace tcd {
 // barrier slots (8 bytes each) after kTcSmemBar
-constexpr int kQFull = 0, kQEmpty = 1, kKFull = 2, kVFull = 4, kKVEmpty = 6, kSFull = 8,
-              kPFull = 10, kOFull = 12, kOEmpty = 14, kQReady = 16, kNumBars = 17;
+constexpr int kQFull = 0, kQEmpty = 2, kQReady = 4, kKVFull = 6, kKVEmpty = 9, kSFull = 12,
+              kPFull = 14, kOFull = 16, kOEmpty = 18, kNumBars = 20;
 constexpr uint32_t kTmemHolder = kNumBars * 8;      // u32: tensor-memory base address
 constexpr uint32_t kAbortFlag = kTmemHolder + 4;    // u32: set when a wait ran out
 }  // namespace tcd
@@ -139,7 +141,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int i = 0; i < tcd::kNumBars; ++i) {
       uint32_t count = 1;
       if (i == tcd::kPFull || i == tcd::kPFull + 1 || i == tcd::kOEmpty || i == tcd::kOEmpty + 1 ||
-          i == tcd::kQReady)
+          i == tcd::kQReady || i == tcd::kQReady + 1)
         count = 128;
       tc::mbar_init(bar(i), count);
     }
@@ -156,41 +158,36 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sgen + kTcSmemBar + tcd::kTmemHolder);
 
   // Register split (per warpgroup) of the 512 x 128 registers the CTA is launched with:
-  // warps 0-3 (producer, MMA issuer, two idle) keep 56, the Q-preparation warpgroup
+  // warps 0-3 (two producers, MMA issuer, idle) keep 56, the Q-preparation warpgroup
   // (warps 12-15) 104, the two softmax warpgroups 176: 128*(56 + 104) + 256*176 = 65536,
   // and on every SM sub-partition 56 + 104 + 2*176 = 512 registers per lane.
+  // K/V ring: block i of the CTA's sequence of blocks loads K as load 2i and V as load
+  // 2i + 1; load L goes to slot L % 3 and may start once load L - 3 has been consumed.
+  auto kv_slot = [](uint32_t L) { return L % kTcKVSlots; };
+  auto kv_par = [](uint32_t L) { return (L / kTcKVSlots) & 1u; };
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------ K/V producer
     asm volatile("setmaxnreg.dec.sync.aligned.u32 56;\n" ::: "memory");
     if (lane == 0) {
-      tc::prefetch_tmap(&tm_q);
       tc::prefetch_tmap(&tm_k);
       tc::prefetch_tmap(&tm_v);
-      uint32_t it = 0;  // K/V blocks loaded so far (ring position)
+      uint32_t L = 0;
       bool ok = true;
-      for (int u = blockIdx.x, n = 0; ok && u < a.n_units; u += gridDim.x, ++n) {
+      for (int u = blockIdx.x; ok && u < a.n_units; u += gridDim.x) {
         const TcUnit w = tc_unit(a, u);
-        const int h0 = 2 * w.pair, g = h0 / kGroup;
-        if (n > 0 && !(ok = tc_wait(bar(tcd::kQEmpty), (n - 1) & 1, abort, a.status))) break;
-        tc::mbar_expect_tx(bar(tcd::kQFull), 2 * kTcTileBytes);
-        for (int t = 0; t < 2; ++t)
-          for (int hf = 0; hf < 2; ++hf)
-            tc::tma_load_4d(sbase + kTcSmemQ + t * kTcTileBytes + hf * kTcHalfBytes, &tm_q,
-                            bar(tcd::kQFull), hf * 64, h0 + t, w.q0, w.b);
-        for (int j = 0; j < w.n_blk; ++j, ++it) {
-          const uint32_t s = it & 1u;
-          if (it >= 2 &&
-              !(ok = tc_wait(bar(tcd::kKVEmpty + s), ((it >> 1) - 1) & 1u, abort, a.status)))
-            break;
+        const int g = (2 * w.pair) / kGroup;
+        for (int j = 0; ok && j < w.n_blk; ++j) {
           const int key0 = (w.kb_lo + j) * kTcBN;
-          tc::mbar_expect_tx(bar(tcd::kKFull + s), kTcTileBytes);
-          for (int hf = 0; hf < 2; ++hf)
-            tc::tma_load_4d(sbase + kTcSmemK + s * kTcTileBytes + hf * kTcHalfBytes, &tm_k,
-                            bar(tcd::kKFull + s), hf * 64, g, key0, w.b);
-          tc::mbar_expect_tx(bar(tcd::kVFull + s), kTcTileBytes);
-          for (int hf = 0; hf < 2; ++hf)
-            tc::tma_load_4d(sbase + kTcSmemV + s * kTcTileBytes + hf * kTcHalfBytes, &tm_v,
-                            bar(tcd::kVFull + s), hf * 64, g, key0, w.b);
+          for (int kv = 0; kv < 2; ++kv, ++L) {
+            const uint32_t slot = kv_slot(L);
+            if (L >= kTcKVSlots &&
+                !(ok = tc_wait(bar(tcd::kKVEmpty + slot), kv_par(L) ^ 1u, abort, a.status)))
+              break;
+            tc::mbar_expect_tx(bar(tcd::kKVFull + slot), kTcTileBytes);
+            for (int hf = 0; hf < 2; ++hf)
+              tc::tma_load_4d(sbase + kTcSmemKV + slot * kTcTileBytes + hf * kTcHalfBytes,
+                              kv ? &tm_v : &tm_k, bar(tcd::kKVFull + slot), hf * 64, g, key0, w.b);
+          }
         }
       }
     }
@@ -207,51 +204,56 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       auto v_desc = [&](uint32_t tile, int kk) {  // MN-major: d halves 16 KiB apart
         return tc::sdesc_sw128(tile + kk * 2048, kTcHalfBytes, 1024);
       };
-      // O_t += P_t V for K/V ring position `pos`; `first` overwrites O_t.
-      auto issue_pv = [&](int t, uint32_t pos, bool first) {
-        const uint32_t vt = sbase + kTcSmemV + (pos & 1u) * kTcTileBytes;
+      // O_t += P_t V with V in ring slot `slot`; `first` overwrites O_t.
+      auto issue_pv = [&](int t, uint32_t slot, bool first) {
+        const uint32_t vt = sbase + kTcSmemKV + slot * kTcTileBytes;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           tc::umma_ts(tmem + 256 + 128 * t, tmem + 128 * t + kk * 8, v_desc(vt, kk), idesc_pv,
                       (!first || kk > 0) ? 1u : 0u);
       };
-      uint32_t it = 0;  // K/V ring position of the current block
+      uint32_t it = 0;  // blocks of the CTA started so far
       bool ok = true;
       for (int u = blockIdx.x, n = 0; ok && u < a.n_units; u += gridDim.x, ++n) {
         const TcUnit w = tc_unit(a, u);
-        if (!(ok = tc_wait(bar(tcd::kQReady), n & 1, abort, a.status))) break;
+        const int qset = n & 1;
+        if (!(ok = tc_wait(bar(tcd::kQReady + qset), (n >> 1) & 1, abort, a.status))) break;
         // step j: O_t += P_t(j-1) V(j-1) (j > 0), then S_t(j) = Q_t K(j)^T (j < n_blk)
         for (int j = 0; ok && j <= w.n_blk; ++j) {
           const bool has_s = j < w.n_blk;
-          const uint32_t s = it & 1u;
-          if (has_s && !(ok = tc_wait(bar(tcd::kKFull + s), (it >> 1) & 1u, abort, a.status)))
+          const uint32_t LK = 2 * it;
+          if (has_s &&
+              !(ok = tc_wait(bar(tcd::kKVFull + kv_slot(LK)), kv_par(LK), abort, a.status)))
             break;
           tc::tc_fence_after();
-          const uint32_t kt = sbase + kTcSmemK + s * kTcTileBytes;
+          const uint32_t kt = sbase + kTcSmemKV + kv_slot(LK) * kTcTileBytes;
           for (int t = 0; t < 2 && ok; ++t) {
             if (j > 0) {
-              const uint32_t prev = it - 1;
-              if (!(ok = tc_wait(bar(tcd::kPFull + t), prev & 1u, abort, a.status))) break;
-              if (t == 0 && !(ok = tc_wait(bar(tcd::kVFull + (prev & 1u)), (prev >> 1) & 1u,
-                                           abort, a.status)))
+              const uint32_t LV = 2 * (it - 1) + 1;
+              if (!(ok = tc_wait(bar(tcd::kPFull + t), (it - 1) & 1u, abort, a.status))) break;
+              if (t == 0 &&
+                  !(ok = tc_wait(bar(tcd::kKVFull + kv_slot(LV)), kv_par(LV), abort, a.status)))
                 break;
               // the first P V of a unit overwrites O_t: the previous epilogue must be done
               if (j == 1 && n > 0 &&
                   !(ok = tc_wait(bar(tcd::kOEmpty + t), (n - 1) & 1, abort, a.status)))
                 break;
               tc::tc_fence_after();
-              issue_pv(t, prev, j == 1);
-              if (t == 1) tc::umma_commit(bar(tcd::kKVEmpty + (prev & 1u)));
+              issue_pv(t, kv_slot(LV), j == 1);
+              if (t == 1) tc::umma_commit(bar(tcd::kKVEmpty + kv_slot(LV)));
               if (!has_s) tc::umma_commit(bar(tcd::kOFull + t));
             }
             if (has_s) {
-              const uint32_t qt = sbase + kTcSmemQ + t * kTcTileBytes;
+              const uint32_t qt = sbase + kTcSmemQ + (qset * 2 + t) * kTcTileBytes;
 #pragma unroll
               for (int ks = 0; ks < 8; ++ks)
                 tc::umma_ss(tmem + 128 * t, qk_desc(qt, ks), qk_desc(kt, ks), idesc_qk,
                             ks > 0 ? 1u : 0u);
               tc::umma_commit(bar(tcd::kSFull + t));
-              if (t == 1 && j == w.n_blk - 1) tc::umma_commit(bar(tcd::kQEmpty));
+              if (t == 1) {
+                tc::umma_commit(bar(tcd::kKVEmpty + kv_slot(LK)));
+                if (j == w.n_blk - 1) tc::umma_commit(bar(tcd::kQEmpty + qset));
+              }
             }
           }
           if (has_s) ++it;
@@ -259,7 +261,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp < 4) {
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ Q producer
+    // Raw Q tiles of unit n into set n & 1, as soon as unit n - 2 has released the set.
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 56;\n" ::: "memory");
+    if (lane == 0) {
+      tc::prefetch_tmap(&tm_q);
+      bool ok = true;
+      for (int u = blockIdx.x, n = 0; ok && u < a.n_units; u += gridDim.x, ++n) {
+        const TcUnit w = tc_unit(a, u);
+        const int qset = n & 1;
+        if (n >= 2 &&
+            !(ok = tc_wait(bar(tcd::kQEmpty + qset), ((n >> 1) - 1) & 1, abort, a.status)))
+          break;
+        tc::mbar_expect_tx(bar(tcd::kQFull + qset), 2 * kTcTileBytes);
+        for (int t = 0; t < 2; ++t)
+          for (int hf = 0; hf < 2; ++hf)
+            tc::tma_load_4d(sbase + kTcSmemQ + (qset * 2 + t) * kTcTileBytes + hf * kTcHalfBytes,
+                            &tm_q, bar(tcd::kQFull + qset), hf * 64, 2 * w.pair + t, w.q0, w.b);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 3) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 56;\n" ::: "memory");
   } else if (warp >= 12) {
     // ------------------------------------------------------------ Q preparation
@@ -288,10 +311,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tab_load(0, 0);
         tab_load(1, 1);
       }
-      if (!(ok = tc_wait(bar(tcd::kQFull), n & 1, abort, a.status))) break;
+      const int qset = n & 1;
+      if (!(ok = tc_wait(bar(tcd::kQFull + qset), (n >> 1) & 1, abort, a.status))) break;
       auto chunk = [&](int t, int hf, int c) -> uint4 * {   // 8 bf16 at d = 64 hf + 8 c
-        return reinterpret_cast<uint4 *>(sgen + kTcSmemQ + t * kTcTileBytes + r * 128 +
-                                         hf * kTcHalfBytes + ((c ^ (r & 7)) << 4));
+        return reinterpret_cast<uint4 *>(sgen + kTcSmemQ + (qset * 2 + t) * kTcTileBytes +
+                                         r * 128 + hf * kTcHalfBytes + ((c ^ (r & 7)) << 4));
       };
       float inv[2];
 #pragma unroll
@@ -356,7 +380,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       // generic-proxy writes -> visible to the tensor cores' async proxy, then publish
       asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-      tc::mbar_arrive(bar(tcd::kQReady));
+      tc::mbar_arrive(bar(tcd::kQReady + qset));
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
