@@ -13,8 +13,8 @@
 // triangle's longest rows first), so the next unit's loads and first Q K^T overlap the
 // current unit's epilogue, and set-up (barriers, tensor memory) happens once.
 // 512 threads in warp roles:
-//   warp 0      K/V producer (TMA): K and V tiles of 128 keys into a three-slot ring
-//               (128-byte swizzled boxes of 128 rows x 64 columns);
+//   warp 0      K/V producer (TMA): K tiles of 128 keys into a two-slot ring running a
+//               block ahead, V tiles into one slot (128-byte swizzled 128 x 64 boxes);
 //   warp 1      MMA issuer (one thread): S_t = Q_t K^T (both operands in shared memory)
 //               and O_t += P_t V (P from tensor memory, V in shared memory), t = 0, 1;
 //               the whole warp also allocates and frees the 512 tensor-memory columns:
@@ -55,7 +55,7 @@ constexpr int kTcBN = 128;      // keys per block
 constexpr uint32_t kTcTileBytes = 128 * 128 * 2;   // 32 KiB: one 128 x 128 bf16 tile
 constexpr uint32_t kTcHalfBytes = kTcTileBytes / 2;  // one 128 x 64 TMA box
 constexpr uint32_t kTcSmemQ = 0;                      // Q: 2 sets (units n even / odd) x 2 tiles
-constexpr uint32_t kTcSmemKV = 4 * kTcTileBytes;      // K/V ring: 3 slots of one 128 x 128 tile
+constexpr uint32_t kTcSmemKV = 4 * kTcTileBytes;      // K ring (slots 0, 1) and V slot (2)
 constexpr uint32_t kTcKVSlots = 3;
 constexpr uint32_t kTcSmemBar = kTcSmemKV + kTcKVSlots * kTcTileBytes;  // mbarriers
 constexpr uint32_t kTcSmemBytes = kTcSmemBar + 256 + 1024;  // 230,656 B: barriers + alignment slack
@@ -90,6 +90,29 @@ __device__ __forceinline__ float tanh_approx(float x) {
   float y;
   asm("tanh.approx.f32 %0, %1;\n" : "=f"(y) : "f"(x));
   return y;
+}
+
+// exp2 of two values on the FMA and integer pipes, to take part of the exponentials off the
+// MUFU unit: 2^y = 2^k * 2^f with k = round(y) (found by adding 1.5 * 2^23, which leaves k
+// in the low mantissa bits), f = y - k in [-1/2, 1/2], 2^f from a cubic fitted for least
+// maximum relative error (7.5e-5, far below bf16's 2^-9; fit_exp2_poly.py), and 2^k
+// applied by adding k to the exponent field.  y is clamped at -120 first, so masked
+// (-inf) scores give 2^-120 instead of 0 -- negligible against the row's weights.
+constexpr int kTcEmuPairs = 0;  // pairs per 16 emulated in each 32-score chunk
+__device__ __forceinline__ void exp2_poly_pair(float y0, float y1, float &p0, float &p1) {
+  const uint64_t y = tc::f2_pack(fmaxf(y0, -120.0f), fmaxf(y1, -120.0f));
+  const uint64_t t = tc::f2_add(y, tc::f2_pack(12582912.0f, 12582912.0f));
+  const uint64_t kf = tc::f2_add(t, tc::f2_pack(-12582912.0f, -12582912.0f));
+  const uint64_t f = tc::f2_fma(kf, tc::f2_pack(-1.0f, -1.0f), y);
+  uint64_t q = tc::f2_fma(tc::f2_pack(5.517166853e-02f, 5.517166853e-02f), f,
+                          tc::f2_pack(2.426111251e-01f, 2.426111251e-01f));
+  q = tc::f2_fma(q, f, tc::f2_pack(6.932609677e-01f, 6.932609677e-01f));
+  q = tc::f2_fma(q, f, tc::f2_pack(9.999280572e-01f, 9.999280572e-01f));
+  float q0, q1, t0, t1;
+  tc::f2_unpack(q, q0, q1);
+  tc::f2_unpack(t, t0, t1);
+  p0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+  p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
 }
 
 // Bounded wait on an mbarrier phase; false when it ran out or another role aborted.
@@ -161,34 +184,67 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // warps 0-3 (two producers, MMA issuer, idle) keep 56, the Q-preparation warpgroup
   // (warps 12-15) 104, the two softmax warpgroups 176: 128*(56 + 104) + 256*176 = 65536,
   // and on every SM sub-partition 56 + 104 + 2*176 = 512 registers per lane.
-  // K/V ring: block i of the CTA's sequence of blocks loads K as load 2i and V as load
-  // 2i + 1; load L goes to slot L % 3 and may start once load L - 3 has been consumed.
-  auto kv_slot = [](uint32_t L) { return L % kTcKVSlots; };
-  auto kv_par = [](uint32_t L) { return (L / kTcKVSlots) & 1u; };
+  // K tiles of the CTA's block sequence go to a two-slot ring (block i in slot i % 2), V
+  // tiles to one slot; K runs a block ahead of V, so K(i+1) loads as soon as both Q K(i-1)^T
+  // are done, and V(i) once both P V(i-1) are.  Barrier slots kKVFull/kKVEmpty + 0, 1 are
+  // the K ring, + 2 the V slot.
   if (warp == 0) {
     // ------------------------------------------------------------ K/V producer
     asm volatile("setmaxnreg.dec.sync.aligned.u32 56;\n" ::: "memory");
     if (lane == 0) {
       tc::prefetch_tmap(&tm_k);
       tc::prefetch_tmap(&tm_v);
-      uint32_t L = 0;
-      bool ok = true;
-      for (int u = blockIdx.x; ok && u < a.n_units; u += gridDim.x) {
-        const TcUnit w = tc_unit(a, u);
-        const int g = (2 * w.pair) / kGroup;
-        for (int j = 0; ok && j < w.n_blk; ++j) {
-          const int key0 = (w.kb_lo + j) * kTcBN;
-          for (int kv = 0; kv < 2; ++kv, ++L) {
-            const uint32_t slot = kv_slot(L);
-            if (L >= kTcKVSlots &&
-                !(ok = tc_wait(bar(tcd::kKVEmpty + slot), kv_par(L) ^ 1u, abort, a.status)))
-              break;
-            tc::mbar_expect_tx(bar(tcd::kKVFull + slot), kTcTileBytes);
-            for (int hf = 0; hf < 2; ++hf)
-              tc::tma_load_4d(sbase + kTcSmemKV + slot * kTcTileBytes + hf * kTcHalfBytes,
-                              kv ? &tm_v : &tm_k, bar(tcd::kKVFull + slot), hf * 64, g, key0, w.b);
-          }
+      struct Cursor {  // walks (unit, block) in the order the MMA issuer consumes them
+        int u, j;
+        TcUnit w;
+        bool valid;
+      };
+      auto start = [&](Cursor &c) {
+        c.u = blockIdx.x;
+        c.j = 0;
+        c.valid = c.u < a.n_units;
+        if (c.valid) c.w = tc_unit(a, c.u);
+      };
+      auto advance = [&](Cursor &c) {
+        if (++c.j == c.w.n_blk) {
+          c.j = 0;
+          c.u += gridDim.x;
+          c.valid = c.u < a.n_units;
+          if (c.valid) c.w = tc_unit(a, c.u);
         }
+      };
+      auto load = [&](const Cursor &c, bool is_v, uint32_t slot) {
+        const int g = (2 * c.w.pair) / kGroup, key0 = (c.w.kb_lo + c.j) * kTcBN;
+        tc::mbar_expect_tx(bar(tcd::kKVFull + slot), kTcTileBytes);
+        for (int hf = 0; hf < 2; ++hf)
+          tc::tma_load_4d(sbase + kTcSmemKV + slot * kTcTileBytes + hf * kTcHalfBytes,
+                          is_v ? &tm_v : &tm_k, bar(tcd::kKVFull + slot), hf * 64, g, key0, c.w.b);
+      };
+      Cursor kc, vc;
+      start(kc);
+      start(vc);
+      uint32_t ik = 0, iv = 0;  // K and V tiles issued so far
+      bool ok = true;
+      if (kc.valid) {
+        load(kc, false, 0);
+        ++ik;
+        advance(kc);
+      }
+      while (ok && vc.valid) {
+        if (kc.valid) {
+          const uint32_t slot = ik & 1u;
+          if (ik >= 2 &&
+              !(ok = tc_wait(bar(tcd::kKVEmpty + slot), ((ik >> 1) - 1) & 1u, abort, a.status)))
+            break;
+          load(kc, false, slot);
+          ++ik;
+          advance(kc);
+        }
+        if (iv >= 1 && !(ok = tc_wait(bar(tcd::kKVEmpty + 2), (iv - 1) & 1u, abort, a.status)))
+          break;
+        load(vc, true, 2);
+        ++iv;
+        advance(vc);
       }
     }
     __syncwarp();
@@ -221,26 +277,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // step j: O_t += P_t(j-1) V(j-1) (j > 0), then S_t(j) = Q_t K(j)^T (j < n_blk)
         for (int j = 0; ok && j <= w.n_blk; ++j) {
           const bool has_s = j < w.n_blk;
-          const uint32_t LK = 2 * it;
+          const uint32_t ks_slot = it & 1u;
           if (has_s &&
-              !(ok = tc_wait(bar(tcd::kKVFull + kv_slot(LK)), kv_par(LK), abort, a.status)))
+              !(ok = tc_wait(bar(tcd::kKVFull + ks_slot), (it >> 1) & 1u, abort, a.status)))
             break;
           tc::tc_fence_after();
-          const uint32_t kt = sbase + kTcSmemKV + kv_slot(LK) * kTcTileBytes;
+          const uint32_t kt = sbase + kTcSmemKV + ks_slot * kTcTileBytes;
           for (int t = 0; t < 2 && ok; ++t) {
             if (j > 0) {
-              const uint32_t LV = 2 * (it - 1) + 1;
               if (!(ok = tc_wait(bar(tcd::kPFull + t), (it - 1) & 1u, abort, a.status))) break;
               if (t == 0 &&
-                  !(ok = tc_wait(bar(tcd::kKVFull + kv_slot(LV)), kv_par(LV), abort, a.status)))
+                  !(ok = tc_wait(bar(tcd::kKVFull + 2), (it - 1) & 1u, abort, a.status)))
                 break;
               // the first P V of a unit overwrites O_t: the previous epilogue must be done
               if (j == 1 && n > 0 &&
                   !(ok = tc_wait(bar(tcd::kOEmpty + t), (n - 1) & 1, abort, a.status)))
                 break;
               tc::tc_fence_after();
-              issue_pv(t, kv_slot(LV), j == 1);
-              if (t == 1) tc::umma_commit(bar(tcd::kKVEmpty + kv_slot(LV)));
+              issue_pv(t, 2, j == 1);
+              if (t == 1) tc::umma_commit(bar(tcd::kKVEmpty + 2));
               if (!has_s) tc::umma_commit(bar(tcd::kOFull + t));
             }
             if (has_s) {
@@ -251,7 +306,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                             ks > 0 ? 1u : 0u);
               tc::umma_commit(bar(tcd::kSFull + t));
               if (t == 1) {
-                tc::umma_commit(bar(tcd::kKVEmpty + kv_slot(LK)));
+                tc::umma_commit(bar(tcd::kKVEmpty + ks_slot));
                 if (j == w.n_blk - 1) tc::umma_commit(bar(tcd::kQEmpty + qset));
               }
             }
@@ -460,7 +515,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                                  __uint_as_float(sr[c][i + 1])),
                                      f2, nm2),
                           y0, y1);
-            const float p0 = ex2_approx(y0), p1 = ex2_approx(y1);
+            float p0, p1;
+            if ((i >> 1) < kTcEmuPairs) {
+              exp2_poly_pair(y0, y1, p0, p1);
+            } else {
+              p0 = ex2_approx(y0);
+              p1 = ex2_approx(y1);
+            }
             acc[(i >> 1) & 3] = tc::f2_add(acc[(i >> 1) & 3], tc::f2_pack(p0, p1));
             pk[i >> 1] = pack_bf16(p0, p1);
           }
