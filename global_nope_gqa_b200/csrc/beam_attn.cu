@@ -56,7 +56,11 @@ int device_info(DeviceInfo **out) {
     if ((st = cuda_status(cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev),
                           "SM count")))
       return st;
-    if ((st = cuda_status(cudaFuncSetAttribute(decode_splitk_kernel,
+    if ((st = cuda_status(cudaFuncSetAttribute(decode_attn_kernel<false>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem),
+                          "decode shared-memory opt-in")))
+      return st;
+    if ((st = cuda_status(cudaFuncSetAttribute(decode_attn_kernel<true>,
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem),
                           "decode shared-memory opt-in")))
       return st;
@@ -133,12 +137,17 @@ int make_head_map(CUtensorMap *map, const void *base, int heads, int T, int B) {
   return r == CUDA_SUCCESS ? BEAM_OK : BEAM_ERR_CUDA;
 }
 
-// Decode split size: cache slots per CTA.  A local ring is one split; a global
+// Decode split size: cache slots per CTA.  A local ring is cut into at most four
+// splits (one thread-block cluster); a global
 // cache is cut so that the grid holds several waves of the SMs at its largest
 // context, in runs of at least 512 slots (the partial results are then well
 // under 1% of the bytes streamed).
 int decode_split(int kind, const beam_attn_params *p, int32_t B, int64_t slots, int sm_count) {
-  if (kind == BEAM_LOCAL) return (int)round_up((size_t)p->window, kDecTile);
+  if (kind == BEAM_LOCAL) {  // the ring: one split, or up to 4 (a cluster) for small batches
+    const size_t ring = round_up((size_t)p->window, kDecTile);
+    if ((int64_t)B * kHkv >= 2 * sm_count) return (int)ring;
+    return (int)std::max<size_t>(kDecTile, round_up(((size_t)p->window + 3) / 4, kDecTile));
+  }
   const int64_t target_ctas = (int64_t)sm_count * 2 * 8;  // ~8 waves at 2 CTAs per SM
   int64_t split = 512;
   while (split < 16384 && (int64_t)B * kHkv * ((slots + split - 1) / split) > target_ctas)
@@ -376,6 +385,56 @@ int beam_attn_decode(int kind, const beam_attn_params *p, int32_t B, const void 
   if (n_split_max > 65535) return BEAM_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
 
+  DecodeArgs da;
+  memset(&da, 0, sizeof da);
+  da.qn = w.qn;
+  da.k_cache = static_cast<uint16_t *>(k_cache);
+  da.v_cache = static_cast<uint16_t *>(v_cache);
+  da.stride_seq = layout->stride_seq;
+  da.stride_head = layout->stride_head;
+  da.slots = layout->slots_per_seq;
+  da.pos = pos;
+  da.kind = kind;
+  da.window = p->window;
+  da.split = split;
+  da.n_split_max = n_split_max;
+  da.scale_log2 = p->softmax_scale * kLog2e;
+  da.ssmax_base = p->ssmax_base;
+  da.ssmax_exp = p->ssmax_exp;
+  da.part_o = w.part_o;
+  da.part_ml = w.part_ml;
+  dim3 grid(n_split_max, kHkv, B);
+
+  if (kind == BEAM_LOCAL) {
+    // one launch: the ring's splits form a cluster that normalises, appends, attends,
+    // merges through distributed shared memory and gates
+    da.q_raw = static_cast<const uint16_t *>(q);
+    da.k_raw = static_cast<const uint16_t *>(k);
+    da.v_raw = static_cast<const uint16_t *>(v);
+    da.gate = static_cast<const uint16_t *>(gate);
+    da.qw = q_norm_w;
+    da.kw = k_norm_w;
+    da.gate_bias = gate_bias;
+    da.out = static_cast<uint16_t *>(out);
+    da.status = dev_status;
+    da.eps = p->rms_eps;
+    fill_inv_freq(da.inv_freq, p->rope_theta);
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof cfg);
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kDecThreads);
+    cfg.dynamicSmemBytes = kDecSmem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)n_split_max;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cuda_status(cudaLaunchKernelEx(&cfg, decode_attn_kernel<true>, da), "ring decode launch");
+  }
+
   PrologueArgs pa;
   memset(&pa, 0, sizeof pa);
   pa.q = static_cast<const uint16_t *>(q);
@@ -399,26 +458,7 @@ int beam_attn_decode(int kind, const beam_attn_params *p, int32_t B, const void 
   fill_inv_freq(pa.inv_freq, p->rope_theta);
   prologue_kernel<<<(unsigned)B, 128, 0, s>>>(pa);
   if ((st = launch_status())) return st;
-
-  DecodeArgs da;
-  da.qn = w.qn;
-  da.k_cache = static_cast<const uint16_t *>(k_cache);
-  da.v_cache = static_cast<const uint16_t *>(v_cache);
-  da.stride_seq = layout->stride_seq;
-  da.stride_head = layout->stride_head;
-  da.slots = layout->slots_per_seq;
-  da.pos = pos;
-  da.kind = kind;
-  da.window = p->window;
-  da.split = split;
-  da.n_split_max = n_split_max;
-  da.scale_log2 = p->softmax_scale * kLog2e;
-  da.ssmax_base = p->ssmax_base;
-  da.ssmax_exp = p->ssmax_exp;
-  da.part_o = w.part_o;
-  da.part_ml = w.part_ml;
-  dim3 grid(n_split_max, kHkv, B);
-  decode_splitk_kernel<<<grid, kDecThreads, kDecSmem, s>>>(da);
+  decode_attn_kernel<false><<<grid, kDecThreads, kDecSmem, s>>>(da);
   if ((st = launch_status())) return st;
 
   CombineArgs ca;

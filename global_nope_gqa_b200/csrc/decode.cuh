@@ -7,7 +7,7 @@
 // and the time goes into streaming the global caches, 4 KiB per token per
 // layer (section "KV memory").
 //
-// decode_splitk_kernel: grid (split, KV head, sequence), 128 threads.  A CTA
+// decode_attn_kernel: grid (split, KV head, sequence), 128 threads.  A CTA
 // streams a contiguous run of `split` cache slots of one (sequence, KV head) --
 // keys and values are contiguous in the head-major cache -- through a 3-stage
 // cp.async ring of 64-slot tiles (16-byte coalesced loads, XOR-swizzled rows).
@@ -22,7 +22,10 @@
 // with the log-sum-exp rule and applies Y = O/l * sigmoid(G + b_h).
 #pragma once
 
+#include <cooperative_groups.h>
+
 #include "common.cuh"
+#include "prologue.cuh"
 
 namespace beam {
 
@@ -33,9 +36,9 @@ constexpr int kDecTileBytes = kDecTile * kD * 2;                   // 16 KiB
 constexpr int kDecSmem = kDecStages * 2 * kDecTileBytes;
 
 struct DecodeArgs {
-  const uint16_t *qn;       // [B][48][128] prepared queries
-  const uint16_t *k_cache;
-  const uint16_t *v_cache;
+  const uint16_t *qn;       // [B][48][128] prepared queries (split-K path)
+  uint16_t *k_cache;
+  uint16_t *v_cache;
   int64_t stride_seq, stride_head, slots;
   const int64_t *pos;       // [B] 0-based position of the new token
   int kind, window;
@@ -45,6 +48,13 @@ struct DecodeArgs {
   float ssmax_base, ssmax_exp;
   float *part_o;            // [B][8][n_split_max][6][128]
   float *part_ml;           // [B][8][n_split_max][6][2]  (running max in log2 units, sum)
+  // single-kernel path (one split covers every visible slot): raw inputs and the output
+  const uint16_t *q_raw, *k_raw, *v_raw, *gate;  // [B][48*128], [B][8*128] x 2, [B][48*128]
+  const float *qw, *kw, *gate_bias;
+  uint16_t *out;            // [B][48*128]
+  int32_t *status;
+  float eps;
+  double inv_freq[64];
 };
 
 // Number of visible slots of sequence b (0 when the position is invalid).
@@ -54,39 +64,34 @@ __device__ __forceinline__ int64_t decode_visible(const DecodeArgs &a, int64_t t
   return t < a.slots ? t + 1 : 0;
 }
 
-__global__ void __launch_bounds__(kDecThreads) decode_splitk_kernel(const DecodeArgs a) {
+// kFused = false: one split of the keys, partials to the workspace (combined afterwards).
+// kFused = true: the whole step of a local layer in one launch.  The splits of a
+// (sequence, KV head) form one thread-block cluster (gridDim.x CTAs, at most 4 of 128+
+// ring slots each); every CTA normalises and rotates the six queries of its group, the CTA
+// whose slots hold position t also writes the new key and value there, each CTA attends
+// over its slots, and rank 0 merges the CTAs' partials through distributed shared memory
+// and writes Y = O/l * sigmoid(G + b).
+template <bool kFused>
+__global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const DecodeArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
+  __shared__ __align__(16) uint16_t q_prep[kFused ? kGroup * kD : 8];
   const int s_idx = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int64_t t = a.pos[b];
+  if (kFused && t < 0) {
+    if (threadIdx.x == 0) set_status(a.status, BEAM_ERR_CAPACITY);
+    return;
+  }
   const int64_t n_vis = decode_visible(a, t);
   const int64_t key_lo = (int64_t)s_idx * a.split;
-  if (key_lo >= n_vis) return;
+  if (!kFused && key_lo >= n_vis) return;   // a fused CTA stays: its cluster merges below
   const int64_t key_hi = min(n_vis, key_lo + a.split);
-  const int n_keys = (int)(key_hi - key_lo);
+  const int n_keys = key_hi > key_lo ? (int)(key_hi - key_lo) : 0;
   const int n_tiles = (n_keys + kDecTile - 1) / kDecTile;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const size_t head_off = (size_t)b * a.stride_seq + (size_t)g * a.stride_head;
   const uint16_t *kbase = a.k_cache + head_off;
   const uint16_t *vbase = a.v_cache + head_off;
-
-  float factor = a.scale_log2;
-  if (a.kind == BEAM_GLOBAL) factor *= ssmax_factor(t + 1, a.ssmax_base, a.ssmax_exp);
-
-  // Query fragments: A rows = heads (lane/4 < 6 valid), 8 k-steps over d.
-  uint32_t qa[8][2];
-  {
-    const int h = lane >> 2;
-    const uint16_t *qrow = a.qn + ((size_t)b * kHq + g * kGroup + (h < kGroup ? h : 0)) * kD;
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      const int d0 = ks * 16 + (lane & 3) * 2;
-      uint32_t lo = *reinterpret_cast<const uint32_t *>(qrow + d0);
-      uint32_t hi = *reinterpret_cast<const uint32_t *>(qrow + d0 + 8);
-      qa[ks][0] = h < kGroup ? lo : 0u;
-      qa[ks][1] = h < kGroup ? hi : 0u;
-    }
-  }
 
   auto load_tile = [&](int tile, int stage) {
     uint8_t *ks = smem + stage * 2 * kDecTileBytes;
@@ -103,11 +108,74 @@ __global__ void __launch_bounds__(kDecThreads) decode_splitk_kernel(const Decode
       cp_async16(smem_u32(vs + off), vbase + row * kD + c * 8, valid);
     }
   };
-
+  // The first tiles are requested before anything else (in the fused kernel, before the
+  // new row is written: a prefetched tile holding that slot is patched in shared memory).
 #pragma unroll
   for (int st = 0; st < kDecStages - 1; ++st) {
     if (st < n_tiles) load_tile(st, st);
     cp_async_commit();
+  }
+
+  int patch_tile = -1, patch_row = 0;  // fused: prefetched tile and row of the new slot
+  uint4 patch_val = make_uint4(0u, 0u, 0u, 0u);
+  float gate6[kGroup];                 // fused, rank 0: gate logits + bias of its outputs
+  if (kFused) {
+    if (s_idx == 0) {
+#pragma unroll
+      for (int i = 0; i < kGroup; ++i) {
+        const int h = g * kGroup + i;
+        gate6[i] = __uint_as_float((uint32_t)a.gate[((size_t)b * kHq + h) * kD + tid] << 16) +
+                   a.gate_bias[h];
+      }
+    }
+    // rows: 6 queries, the new key, the new value; a half-warp per row
+    const int half = lane >> 4, l16 = lane & 15, row = warp * 2 + half;
+    const unsigned half_mask = 0xFFFFu << (half * 16);
+    const bool rope = a.kind == BEAM_LOCAL;
+    float cs[8], sn[8];
+    if (rope) rope_angles(a.inv_freq, t, l16 & 7, cs, sn);
+    float w[8];
+    load_weights8(row < kGroup ? a.qw : a.kw, l16, w);
+    const uint16_t *src = row < kGroup ? a.q_raw + ((size_t)b * kHq + g * kGroup + row) * kD
+                                       : (row == kGroup ? a.k_raw : a.v_raw) +
+                                             ((size_t)b * kHkv + g) * kD;
+    const uint4 raw = *reinterpret_cast<const uint4 *>(src + l16 * 8);
+    const uint4 res = row == kGroup + 1 ? raw
+                                        : norm_rope_row(raw, w, rope, cs, sn, l16, half_mask, a.eps);
+    const int64_t slot = a.kind == BEAM_LOCAL ? t % a.window : t;
+    if (row < kGroup) {
+      *reinterpret_cast<uint4 *>(q_prep + row * kD + l16 * 8) = res;
+    } else if (slot / a.split == s_idx) {
+      uint16_t *cache = row == kGroup ? a.k_cache : a.v_cache;
+      *reinterpret_cast<uint4 *>(cache + head_off + (size_t)slot * kD + l16 * 8) = res;
+      const int rel = (int)(slot - key_lo);
+      if (rel / kDecTile < kDecStages - 1) {
+        patch_tile = rel / kDecTile;
+        patch_row = rel % kDecTile;
+        patch_val = res;
+      }
+    }
+    __threadfence();  // the new row reaches L2 before the later tiles stream it (cp.async.cg)
+    __syncthreads();  // the queries are in shared memory
+  }
+
+  float factor = a.scale_log2;
+  if (a.kind == BEAM_GLOBAL) factor *= ssmax_factor(t + 1, a.ssmax_base, a.ssmax_exp);
+
+  // Query fragments: A rows = heads (lane/4 < 6 valid), 8 k-steps over d.
+  uint32_t qa[8][2];
+  {
+    const int h = lane >> 2;
+    const uint16_t *qrow = kFused ? q_prep + (h < kGroup ? h : 0) * kD
+                                  : a.qn + ((size_t)b * kHq + g * kGroup + (h < kGroup ? h : 0)) * kD;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const int d0 = ks * 16 + (lane & 3) * 2;
+      uint32_t lo = *reinterpret_cast<const uint32_t *>(qrow + d0);
+      uint32_t hi = *reinterpret_cast<const uint32_t *>(qrow + d0 + 8);
+      qa[ks][0] = h < kGroup ? lo : 0u;
+      qa[ks][1] = h < kGroup ? hi : 0u;
+    }
   }
 
   float m_run = -INFINITY;   // running max (log2 units) of head lane/4
@@ -116,9 +184,19 @@ __global__ void __launch_bounds__(kDecThreads) decode_splitk_kernel(const Decode
 #pragma unroll
   for (int nb = 0; nb < 16; ++nb) o[nb][0] = o[nb][1] = o[nb][2] = o[nb][3] = 0.f;
 
+  const bool any_patch = kFused && __syncthreads_or(patch_tile >= 0);
   for (int tile = 0; tile < n_tiles; ++tile) {
     cp_async_wait<kDecStages - 2>();
     __syncthreads();
+    if (kFused && any_patch && tile < kDecStages - 1) {
+      // the new key / value row, written after this tile was requested
+      if (patch_tile == tile) {
+        uint8_t *ks = smem + (tile % kDecStages) * 2 * kDecTileBytes;
+        uint8_t *dst = (warp * 2 + (lane >> 4) == kGroup) ? ks : ks + kDecTileBytes;
+        *reinterpret_cast<uint4 *>(dst + swz256(patch_row, lane & 15)) = patch_val;
+      }
+      __syncthreads();
+    }
     {  // refill the stage that the previous iteration finished with
       const int nt = tile + kDecStages - 1;
       if (nt < n_tiles) load_tile(nt, nt % kDecStages);
@@ -225,11 +303,50 @@ __global__ void __launch_bounds__(kDecThreads) decode_splitk_kernel(const Decode
       acc += sc * sm_o[(w * kGroup + hh) * kD + d];
       L += sc * sm_l[w * kGroup + hh];
     }
-    a.part_o[part * (kGroup * kD) + idx] = acc;
-    if (d == 0) {
-      a.part_ml[(part * kGroup + hh) * 2 + 0] = M;
-      a.part_ml[(part * kGroup + hh) * 2 + 1] = L;
+    if (kFused) {
+      float *cl = reinterpret_cast<float *>(smem + 16384);  // this CTA's partial
+      cl[idx] = acc;
+      if (d == 0) {
+        cl[kGroup * kD + hh] = M;
+        cl[kGroup * kD + kGroup + hh] = L;
+      }
+    } else {
+      a.part_o[part * (kGroup * kD) + idx] = acc;
+      if (d == 0) {
+        a.part_ml[(part * kGroup + hh) * 2 + 0] = M;
+        a.part_ml[(part * kGroup + hh) * 2 + 1] = L;
+      }
     }
+  }
+  if (kFused) {
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    cluster.sync();
+    if (cluster.block_rank() == 0) {
+      float *cl = reinterpret_cast<float *>(smem + 16384);
+      const int n_rank = (int)cluster.num_blocks();
+      for (int idx = tid; idx < kGroup * kD; idx += kDecThreads) {
+        const int hh = idx / kD;
+        float M = -INFINITY;
+        for (int r = 0; r < n_rank; ++r)
+          M = fmaxf(M, cluster.map_shared_rank(cl, r)[kGroup * kD + hh]);
+        const float Mu = M == -INFINITY ? 0.f : M;
+        float acc = 0.f, L = 0.f;
+        for (int r = 0; r < n_rank; ++r) {
+          const float *rc = cluster.map_shared_rank(cl, r);
+          const float sc = exp2f(rc[kGroup * kD + hh] - Mu);
+          acc += sc * rc[idx];
+          L += sc * rc[kGroup * kD + kGroup + hh];
+        }
+        const int h = g * kGroup + hh;
+        const size_t o = ((size_t)b * kHq + h) * kD + (idx - hh * kD);
+        float gl = gate6[0];  // idx = tid + 128 * hh: this thread's d is tid for every head
+#pragma unroll
+        for (int i = 1; i < kGroup; ++i) gl = hh == i ? gate6[i] : gl;
+        a.out[o] = (uint16_t)(pack_bf16(acc / L / (1.0f + expf(-gl)), 0.f) & 0xFFFFu);
+      }
+    }
+    cluster.sync();  // the other CTAs' shared memory stays alive until rank 0 is done
   }
 }
 

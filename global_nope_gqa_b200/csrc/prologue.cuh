@@ -41,17 +41,60 @@ struct PrologueArgs {
   double inv_freq[64];   // theta^(-2i/128), formed on the host in double
 };
 
-__device__ __forceinline__ void rope_angles(const PrologueArgs &a, int64_t t, int sub,
+// cos / sin of the angles t * f_i, i = 8 sub .. 8 sub + 7, formed and reduced to [-pi, pi]
+// in fp64, then evaluated in fp32.
+__device__ __forceinline__ void rope_angles(const double *inv_freq, int64_t t, int sub,
                                             float (&cs)[8], float (&sn)[8]) {
   const double two_pi = 6.283185307179586;
   const double inv_two_pi = 0.15915494309189535;
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
-    double phi = (double)t * a.inv_freq[sub * 8 + e];
+    double phi = (double)t * inv_freq[sub * 8 + e];
     double n = rint(phi * inv_two_pi);
     double r = fma(-n, two_pi, phi);  // |r| <= pi (+ rounding)
     sincosf((float)r, &sn[e], &cs[e]);
   }
+}
+
+// RMSNorm of one 128-wide row held by a half-warp (lane l16 holds coordinates
+// 8 l16 .. 8 l16 + 7 as eight bf16 in `raw`), times the weights w, then -- for a local
+// layer -- rotate-half RoPE with the angles' cos / sin (the partner of coordinate c < 64 is
+// c + 64, held by lane l16 ^ 8).  Returns the eight results as bf16.
+__device__ __forceinline__ uint4 norm_rope_row(uint4 raw, const float (&w)[8], bool rope,
+                                               const float (&cs)[8], const float (&sn)[8],
+                                               int l16, unsigned half_mask, float eps) {
+  float x[8];
+  x[0] = bf16_lo(raw.x); x[1] = bf16_hi(raw.x); x[2] = bf16_lo(raw.y); x[3] = bf16_hi(raw.y);
+  x[4] = bf16_lo(raw.z); x[5] = bf16_hi(raw.z); x[6] = bf16_lo(raw.w); x[7] = bf16_hi(raw.w);
+  float ss = 0.f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
+#pragma unroll
+  for (int off = 1; off < 16; off <<= 1) ss += __shfl_xor_sync(half_mask, ss, off);
+  const float inv_rms = rsqrtf(ss * (1.0f / kD) + eps);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) x[e] = x[e] * inv_rms * w[e];
+  if (rope) {
+    float y[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      float partner = __shfl_xor_sync(half_mask, x[e], 8);
+      y[e] = (l16 < 8) ? (x[e] * cs[e] - partner * sn[e]) : (x[e] * cs[e] + partner * sn[e]);
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) x[e] = y[e];
+  }
+  uint4 res;
+  res.x = pack_bf16(x[0], x[1]); res.y = pack_bf16(x[2], x[3]);
+  res.z = pack_bf16(x[4], x[5]); res.w = pack_bf16(x[6], x[7]);
+  return res;
+}
+
+__device__ __forceinline__ void load_weights8(const float *w, int l16, float (&out)[8]) {
+  const float4 *w4 = reinterpret_cast<const float4 *>(w) + l16 * 2;
+  const float4 x0 = w4[0], x1 = w4[1];
+  out[0] = x0.x; out[1] = x0.y; out[2] = x0.z; out[3] = x0.w;
+  out[4] = x1.x; out[5] = x1.y; out[6] = x1.z; out[7] = x1.w;
 }
 
 __global__ void __launch_bounds__(128) prologue_kernel(const PrologueArgs a) {
@@ -83,7 +126,7 @@ __global__ void __launch_bounds__(128) prologue_kernel(const PrologueArgs a) {
   }
 
   float cs[8], sn[8];
-  if (local) rope_angles(a, t < 0 ? 0 : t, l16 & 7, cs, sn);
+  if (local) rope_angles(a.inv_freq, t < 0 ? 0 : t, l16 & 7, cs, sn);
   if (local && a.rope_tab && b == 0 && warp == 0 && lane < 8) {
     // the same angles serve every head and sequence (positions 0 .. T-1): one table row
     float4 *c4 = reinterpret_cast<float4 *>(a.rope_tab + (size_t)i * 128 + lane * 8);
@@ -95,15 +138,8 @@ __global__ void __launch_bounds__(128) prologue_kernel(const PrologueArgs a) {
   }
 
   float wq[8], wk[8];
-  {
-    const float4 *q4 = reinterpret_cast<const float4 *>(a.qw) + l16 * 2;
-    const float4 *k4 = reinterpret_cast<const float4 *>(a.kw) + l16 * 2;
-    float4 x0 = q4[0], x1 = q4[1], y0 = k4[0], y1 = k4[1];
-    wq[0] = x0.x; wq[1] = x0.y; wq[2] = x0.z; wq[3] = x0.w;
-    wq[4] = x1.x; wq[5] = x1.y; wq[6] = x1.z; wq[7] = x1.w;
-    wk[0] = y0.x; wk[1] = y0.y; wk[2] = y0.z; wk[3] = y0.w;
-    wk[4] = y1.x; wk[5] = y1.y; wk[6] = y1.z; wk[7] = y1.w;
-  }
+  load_weights8(a.qw, l16, wq);
+  load_weights8(a.kw, l16, wk);
 
   const unsigned half_mask = 0xFFFFu << (half * 16);  // shuffles stay inside the half-warp
   const int n_rows = kHq + kHkv + kHkv;  // q heads, k heads, v heads
@@ -118,34 +154,8 @@ __global__ void __launch_bounds__(128) prologue_kernel(const PrologueArgs a) {
     const uint16_t *src = is_q ? a.q + (size_t)tok * (kHq * kD) + head * kD
                                : (is_k ? a.k : a.v) + (size_t)tok * (kHkv * kD) + head * kD;
     uint4 raw = *reinterpret_cast<const uint4 *>(src + l16 * 8);
-    uint4 res = raw;
-    if (!is_v) {
-      float x[8];
-      x[0] = bf16_lo(raw.x); x[1] = bf16_hi(raw.x); x[2] = bf16_lo(raw.y); x[3] = bf16_hi(raw.y);
-      x[4] = bf16_lo(raw.z); x[5] = bf16_hi(raw.z); x[6] = bf16_lo(raw.w); x[7] = bf16_hi(raw.w);
-      float ss = 0.f;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
-#pragma unroll
-      for (int off = 1; off < 16; off <<= 1) ss += __shfl_xor_sync(half_mask, ss, off);
-      const float inv_rms = rsqrtf(ss * (1.0f / kD) + a.eps);
-      const float *w = is_q ? wq : wk;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) x[e] = x[e] * inv_rms * w[e];
-      if (local) {
-        // rotate-half: coordinate c < 64 pairs with c + 64, held by lane l16 ^ 8
-        float y[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          float partner = __shfl_xor_sync(half_mask, x[e], 8);
-          y[e] = (l16 < 8) ? (x[e] * cs[e] - partner * sn[e]) : (x[e] * cs[e] + partner * sn[e]);
-        }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) x[e] = y[e];
-      }
-      res.x = pack_bf16(x[0], x[1]); res.y = pack_bf16(x[2], x[3]);
-      res.z = pack_bf16(x[4], x[5]); res.w = pack_bf16(x[6], x[7]);
-    }
+    const uint4 res = is_v ? raw : norm_rope_row(raw, is_q ? wq : wk, local, cs, sn, l16,
+                                                 half_mask, a.eps);
     if (is_q) {
       *reinterpret_cast<uint4 *>(a.q_out + (size_t)tok * (kHq * kD) + head * kD + l16 * 8) = res;
     } else {
