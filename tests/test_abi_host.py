@@ -123,7 +123,7 @@ def test_host_validation_rejects_before_launch(beam):
     P = ctypes.byref(p)
     A = 1 << 20  # a fake, 16-byte aligned device address: never dereferenced on the host
     ws = beam.beam_prefill_workspace_bytes(p, 1, 16)
-    assert ws == 16 * 48 * 128 * 2 + 16 * 8 * 128 * 2
+    assert ws == 16 * 8 * 128 * 2 + 16 * 128 * 4   # prepared keys + RoPE cos/sin table
     args = lambda **kw: [kw.get("kind", 0), kw.get("P", P), kw.get("B", 1), kw.get("T", 16),
                          kw.get("q", A), A, A, A, A, A, A, kw.get("out", A), kw.get("kc", None),
                          kw.get("vc", None), kw.get("layout", None), kw.get("ws", A),
