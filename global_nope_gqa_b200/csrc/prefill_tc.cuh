@@ -127,18 +127,19 @@ __device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity, volatile 
   return false;
 }
 
-// Work unit u -> (q block, head pair, sequence); units with more key blocks come first.
+// Work unit u -> (sequence, q block, head pair): sequence-major, so the CTAs share one
+// sequence's K/V (8 heads x T x 512 B, 32 MiB at T = 8192) while it stays in L2, and within
+// a sequence the units with more key blocks come first.
 struct TcUnit {
   int qb, pair, b, q0, kb_lo, n_blk;
 };
 __device__ __forceinline__ TcUnit tc_unit(const PrefillTcArgs &a, int u) {
   TcUnit w;
-  const int per_qb = (kHq / 2) * a.B;
-  const int idx = u / per_qb;
-  w.qb = a.n_qblocks - 1 - idx;
-  const int rem = u - idx * per_qb;
+  const int per_b = (kHq / 2) * a.n_qblocks;
+  w.b = u / per_b;
+  const int rem = u - w.b * per_b;
+  w.qb = a.n_qblocks - 1 - rem / (kHq / 2);
   w.pair = rem % (kHq / 2);
-  w.b = rem / (kHq / 2);
   w.q0 = w.qb * kTcBM;
   w.kb_lo = a.kind == BEAM_LOCAL ? max(0, w.q0 - a.window + 1) / kTcBN : 0;
   w.n_blk = w.qb - w.kb_lo + 1;  // the last visible key of the unit is in block qb
