@@ -57,6 +57,27 @@ def _jsonable(o):
     raise TypeError(type(o))
 
 
+def measured_traffic():
+    """DRAM traffic (read + write bytes) of one global-layer attention launch of the batched
+    prefill, from the committed ncu summary -- only while the kernel source it was taken on
+    is unchanged (its hash is recorded beside the figure)."""
+    import hashlib
+    try:
+        src = os.path.join(ROOT, "global_nope_gqa_b200", "csrc", "prefill_tc.cuh")
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        fields = {}
+        with open(os.path.join(ROOT, "profiles", "prefill_tc_global_b2.md")) as f:
+            for line in f:
+                if ":" in line and not line.startswith(("#", " ", "|")):
+                    key, _, val = line.partition(":")
+                    fields[key.strip()] = val.strip()
+        if fields.get("kernel_source_sha256_16") == sha:
+            return int(fields["traffic_bytes_per_launch_batched_prefill_global"])
+    except Exception:
+        pass
+    return None
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -472,7 +493,10 @@ def run_gpu(args):
         "pct_of_bf16_peak": round(100 * value / world / pk["bf16_tflops"], 2),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": pk["bf16_tflops"],
                      "unit": "TFLOP/s", "frac": round(achieved / pk["bf16_tflops"], 4),
-                     "traffic": None, "kernel": "global-layer prefill call (prologue + attention)",
+                     "traffic": measured_traffic() if (w.B, w.T, has_global) == (4, 8192, True)
+                     else None,
+                     "kernel": "global-layer prefill call: K prologue + prefill_tc_kernel "
+                               "(traffic: prefill_tc_kernel, ncu)",
                      "peak_source": pk["source"] + " burst bf16"},
         "e2e": None if args.no_e2e else {
             "value": round(aggregate(flops_step, world, e2e_sec) / 1e12, 3), "unit": "TFLOP/s",
