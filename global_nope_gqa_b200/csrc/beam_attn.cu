@@ -298,6 +298,13 @@ int beam_attn_prefill(int kind, const beam_attn_params *p, int32_t B, int32_t T,
   fa.scale_log2 = p->softmax_scale * kLog2e;
   fa.ssmax_base = p->ssmax_base;
   fa.ssmax_exp = p->ssmax_exp;
+  // Fault injection for tests of the device-timeout path: with BEAM_FAULT_INJECT set to
+  // prefill_wait_stall, the attention kernel's MMA issuer waits on a barrier that nothing
+  // arrives at, so the wait runs out and the call reports BEAM_ERR_DEVICE_TIMEOUT.
+  {
+    const char *f = std::getenv("BEAM_FAULT_INJECT");
+    fa.fault_stall = f != nullptr && std::strcmp(f, "prefill_wait_stall") == 0;
+  }
   const int64_t n_units = (int64_t)fa.n_qblocks * (kHq / 2) * B;
   if (n_units > INT32_MAX) return BEAM_ERR_UNSUPPORTED;
   fa.n_units = (int)n_units;

@@ -37,9 +37,12 @@
 // issued after O_t += P_t(j) V_j; the commit that publishes S_t(j) also covers the O_t
 // update of block j-1, which lets the softmax rescale O_t without a further wait.  Key
 // blocks entirely outside the window or the causal triangle are never loaded.
-// Every mbarrier wait is bounded; a wait that runs out sets BEAM_ERR_DEVICE_TIMEOUT in the
-// status word, raises an abort flag that the other roles also watch, and the CTA still
-// frees its tensor memory before it returns.
+// Every mbarrier wait is bounded (about a second of device time); a wait that runs out sets
+// BEAM_ERR_DEVICE_TIMEOUT in the status word and raises an abort flag that the other roles
+// also watch.  Before the CTA returns, each producer waits (bounded again) for the tiles it
+// issued to land and the MMA issuer for its MMAs to finish, so nothing writes shared or
+// tensor memory after the CTA has freed it.  For tests of that path a launch may ask the
+// MMA issuer to start with a wait on a barrier that nothing arrives at.
 #pragma once
 
 #include <climits>
@@ -59,7 +62,9 @@ constexpr uint32_t kTcSmemKV = 4 * kTcTileBytes;      // K ring (slots 0, 1) and
 constexpr uint32_t kTcKVSlots = 3;
 constexpr uint32_t kTcSmemBar = kTcSmemKV + kTcKVSlots * kTcTileBytes;  // mbarriers
 constexpr uint32_t kTcSmemBytes = kTcSmemBar + 256 + 1024;  // 230,656 B: barriers + alignment slack
-constexpr uint32_t kTcSpinLimit = 1u << 22;
+constexpr uint64_t kTcWaitNs = 1000000000ull;  // give up a wait after 1 s of device time
+constexpr uint32_t kTcSpinLimit = 1u << 25;     // backstop on the polls of one wait
+constexpr uint32_t kTcDrainLimit = 1u << 22;    // polls for in-flight work after an abort
 
 struct PrefillTcArgs {
   const float *q_norm_w;  // [128]
@@ -71,12 +76,13 @@ struct PrefillTcArgs {
   int32_t *status;
   int B, T, kind, window, n_qblocks, n_units;
   float scale_log2, ssmax_base, ssmax_exp;
+  int fault_stall;        // tests only: the MMA issuer first waits on a barrier never arrived at
 };
 
 namespace tcd {
 // barrier slots (8 bytes each) after kTcSmemBar
 constexpr int kQFull = 0, kQEmpty = 2, kQReady = 4, kKVFull = 6, kKVEmpty = 9, kSFull = 12,
-              kPFull = 14, kOFull = 16, kOEmpty = 18, kNumBars = 20;
+              kPFull = 14, kOFull = 16, kOEmpty = 18, kDrain = 20, kStall = 21, kNumBars = 22;
 constexpr uint32_t kTmemHolder = kNumBars * 8;      // u32: tensor-memory base address
 constexpr uint32_t kAbortFlag = kTmemHolder + 4;    // u32: set when a wait ran out
 }  // namespace tcd
@@ -115,16 +121,38 @@ __device__ __forceinline__ void exp2_poly_pair(float y0, float y1, float &p0, fl
   p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
 }
 
-// Bounded wait on an mbarrier phase; false when it ran out or another role aborted.
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
+  return t;
+}
+
+// Bounded wait on an mbarrier phase; false when it ran out or another role aborted.  The
+// clock is read every 1024 polls only, so a wait that succeeds soon never reads it.
 __device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity, volatile uint32_t *abort,
                                         int32_t *status) {
+  uint64_t t0 = 0;
   for (uint32_t i = 0; i < kTcSpinLimit; ++i) {
     if (tc::mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
+    if ((i & 1023u) == 1023u) {
+      const uint64_t t = globaltimer_ns();
+      if (t0 == 0) t0 = t;
+      else if (t - t0 > kTcWaitNs) break;
+    }
   }
   set_status(status, BEAM_ERR_DEVICE_TIMEOUT);
   *abort = 1u;
   return false;
+}
+
+// Wait for the `count`-th completion (count >= 1) of a barrier that only its own producer
+// arms: in-flight copies must land before the CTA returns, whether or not it aborted.
+__device__ __forceinline__ void tc_drain(uint32_t bar, uint32_t count, int32_t *status) {
+  if (count == 0) return;
+  for (uint32_t i = 0; i < kTcDrainLimit; ++i)
+    if (tc::mbar_try_wait(bar, (count - 1) & 1u)) return;
+  set_status(status, BEAM_ERR_DEVICE_TIMEOUT);
 }
 
 // Work unit u -> (sequence, q block, head pair): sequence-major, so the CTAs share one
@@ -247,6 +275,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         ++iv;
         advance(vc);
       }
+      // K slot 0 took loads 0, 2, 4, ..., slot 1 loads 1, 3, ...; V slot 2 all iv
+      tc_drain(bar(tcd::kKVFull + 0), (ik + 1) >> 1, a.status);
+      tc_drain(bar(tcd::kKVFull + 1), ik >> 1, a.status);
+      tc_drain(bar(tcd::kKVFull + 2), iv, a.status);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -270,7 +302,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                       (!first || kk > 0) ? 1u : 0u);
       };
       uint32_t it = 0;  // blocks of the CTA started so far
-      bool ok = true;
+      bool ok = !a.fault_stall || tc_wait(bar(tcd::kStall), 0u, abort, a.status);
       for (int u = blockIdx.x, n = 0; ok && u < a.n_units; u += gridDim.x, ++n) {
         const TcUnit w = tc_unit(a, u);
         const int qset = n & 1;
@@ -315,6 +347,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (has_s) ++it;
         }
       }
+      // every MMA issued so far must be done before the tensor memory is freed
+      tc::umma_commit(bar(tcd::kDrain));
+      tc_drain(bar(tcd::kDrain), 1, a.status);
     }
     __syncwarp();
   } else if (warp == 2) {
@@ -324,6 +359,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (lane == 0) {
       tc::prefetch_tmap(&tm_q);
       bool ok = true;
+      int nq = 0;   // units whose Q tiles were issued (set n & 1 took units n, n + 2, ...)
       for (int u = blockIdx.x, n = 0; ok && u < a.n_units; u += gridDim.x, ++n) {
         const TcUnit w = tc_unit(a, u);
         const int qset = n & 1;
@@ -335,7 +371,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int hf = 0; hf < 2; ++hf)
             tc::tma_load_4d(sbase + kTcSmemQ + (qset * 2 + t) * kTcTileBytes + hf * kTcHalfBytes,
                             &tm_q, bar(tcd::kQFull + qset), hf * 64, 2 * w.pair + t, w.q0, w.b);
+        nq = n + 1;
       }
+      tc_drain(bar(tcd::kQFull + 0), (nq + 1) >> 1, a.status);
+      tc_drain(bar(tcd::kQFull + 1), nq >> 1, a.status);
     }
     __syncwarp();
   } else if (warp == 3) {

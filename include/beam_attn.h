@@ -126,7 +126,13 @@ BEAM_API size_t beam_prefill_workspace_bytes(const beam_attn_params *p, int32_t 
  *     min(T, window) tokens at slot t mod window.  A global cache must hold T
  *     slots (else BEAM_ERR_CAPACITY before any launch).
  *   workspace : device buffer of at least beam_prefill_workspace_bytes().
- * B = 0 or T = 0 is a no-op that returns BEAM_OK. */
+ * B = 0 or T = 0 is a no-op that returns BEAM_OK.
+ * Every wait inside the attention kernel gives up after about one second of
+ * device time: it then writes BEAM_ERR_DEVICE_TIMEOUT to dev_status, lets its
+ * in-flight copies and MMAs finish, leaves that part of `out` unwritten and
+ * returns, so the CUDA context stays usable.  For tests of that path only, the
+ * environment variable BEAM_FAULT_INJECT=prefill_wait_stall (read at each call)
+ * makes the kernel start with a wait that nothing satisfies. */
 BEAM_API int beam_attn_prefill(int kind, const beam_attn_params *p, int32_t B, int32_t T,
                       const void *q, const void *k, const void *v, const void *gate,
                       const float *q_norm_w, const float *k_norm_w, const float *gate_bias,
