@@ -92,6 +92,11 @@ def lib():
         L.oracle_decode.restype = ctypes.c_int
         L.oracle_decode.argtypes = [ctypes.c_int, pp, ctypes.c_int, u16p, u16p, u16p, u16p, fp, fp,
                                     fp, i64p, u16p, u16p, ctypes.c_int64, dp, ctypes.c_int]
+        L.oracle_prefill_chunk_rows.restype = ctypes.c_int
+        L.oracle_prefill_chunk_rows.argtypes = [
+            ctypes.c_int, pp, ctypes.c_int, ctypes.c_int, u16p, u16p, u16p, u16p, fp, fp, fp,
+            ctypes.POINTER(ctypes.c_int64), u16p, u16p, ctypes.c_int64, ctypes.c_int64,
+            ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64), dp, ctypes.c_int]
         L.oracle_kv_row.restype = None
         L.oracle_kv_row.argtypes = [ctypes.c_int, pp, u16p, u16p, fp, ctypes.c_int64, u16p, u16p]
         _lib = L
@@ -232,6 +237,44 @@ def decode(kind, P: Params, q, k, v, gate, q_norm_w, k_norm_w, gate_bias, pos, k
     if rc != 0:
         raise ValueError("oracle_decode rejected its arguments")
     return out
+
+
+def prefill_chunk_rows(kind, P: Params, q, k, v, gate, q_norm_w, k_norm_w, gate_bias, pos0,
+                       k_cache, v_cache, rows_b, rows_i, n_threads: int | None = None) -> np.ndarray:
+    """Chunked prefill against an existing cache, for the listed (b, new token i) rows:
+    [n_rows, Hq, d] float64.  q, gate: [B, T, Hq*d]; k, v: [B, T, Hkv*d] (bf16 bits);
+    pos0: [B] positions of each sequence's first new token; caches [B, Hkv, slots, d]
+    bf16 bits as they were before the call."""
+    q, k, v, gate = _u16(q), _u16(k), _u16(v), _u16(gate)
+    k_cache, v_cache = _u16(k_cache), _u16(v_cache)
+    B, T = q.shape[0], q.shape[1]
+    slots = k_cache.shape[2]
+    pos0 = np.ascontiguousarray(pos0, dtype=np.int64)
+    rows_b = np.ascontiguousarray(rows_b, dtype=np.int64)
+    rows_i = np.ascontiguousarray(rows_i, dtype=np.int64)
+    qw, kw, bias = _f32(q_norm_w), _f32(k_norm_w), _f32(gate_bias)
+    out = np.empty((rows_b.size, P.n_q_heads, P.head_dim), dtype=np.float64)
+    i64 = ctypes.c_int64
+    rc = lib().oracle_prefill_chunk_rows(
+        kind, ctypes.byref(P), B, T, _ptr(q, ctypes.c_uint16), _ptr(k, ctypes.c_uint16),
+        _ptr(v, ctypes.c_uint16), _ptr(gate, ctypes.c_uint16), _ptr(qw, ctypes.c_float),
+        _ptr(kw, ctypes.c_float), _ptr(bias, ctypes.c_float), _ptr(pos0, i64),
+        _ptr(k_cache, ctypes.c_uint16), _ptr(v_cache, ctypes.c_uint16), slots, rows_b.size,
+        _ptr(rows_b, i64), _ptr(rows_i, i64), _ptr(out, ctypes.c_double),
+        n_threads or n_threads_default())
+    if rc != 0:
+        raise ValueError("oracle_prefill_chunk_rows rejected its arguments")
+    return out
+
+
+def prefill_chunk(kind, P: Params, q, k, v, gate, q_norm_w, k_norm_w, gate_bias, pos0, k_cache,
+                  v_cache, n_threads: int | None = None) -> np.ndarray:
+    """All rows of a chunk: [B, T, Hq, d] float64."""
+    B, T = q.shape[0], q.shape[1]
+    bb, ii = np.meshgrid(np.arange(B), np.arange(T), indexing="ij")
+    out = prefill_chunk_rows(kind, P, q, k, v, gate, q_norm_w, k_norm_w, gate_bias, pos0,
+                             k_cache, v_cache, bb.ravel(), ii.ravel(), n_threads)
+    return out.reshape(B, T, P.n_q_heads, P.head_dim)
 
 
 def kv_row(kind, P: Params, k_token, v_token, k_norm_w, j):

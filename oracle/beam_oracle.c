@@ -421,6 +421,117 @@ int oracle_decode(int kind, const oracle_params *P, int B, const uint16_t *q, co
   return 0;
 }
 
+/* --------------------------------------------------------- chunked prefill */
+
+/* Prefill of one chunk against an existing cache: sequence b adds T new
+ * tokens at 0-based positions pos0[b] .. pos0[b] + T - 1 after pos0[b] earlier
+ * tokens (section "KV memory": a call that continues a sequence reads the
+ * earlier keys from the global cache or the local ring).  New token i of
+ * sequence b is the query at t = pos0[b] + i.  Its visible keys j
+ * (oracle_visible) come from two places: j < pos0[b] from the cache as it was
+ * before the call (slot oracle_cache_slot(kind, j, slots), keys already
+ * prepared), j >= pos0[b] from the chunk's own new token j - pos0[b], prepared
+ * here exactly, the way decode treats its one new token.  q, k, v, gate are
+ * token-major [B][T][heads][d] as in oracle_prefill_rows; the caches are
+ * head-major [B][Hkv][slots][d].  Only the listed rows (b = rows_b[r], new
+ * token i = rows_i[r]) are computed; out is [n_rows][Hq][d] doubles. */
+typedef struct {
+  int kind;
+  const oracle_params *P;
+  int B, T;
+  const uint16_t *q, *k, *v, *gate;
+  const double *qw, *kw;
+  const float *bias;
+  const int64_t *pos0;
+  const uint16_t *k_cache, *v_cache;
+  int64_t slots;
+  const int64_t *rows_b, *rows_i;
+  double *out;
+} chunk_ctx;
+
+typedef struct {
+  const chunk_ctx *c;
+  int64_t b, g, lo;
+  const double *k_new, *v_new;  /* [T][d]: the chunk's prepared keys and values, head g */
+} chunk_view;
+
+static void chunk_row(const void *vctx, int64_t idx, double *k_row, double *v_row) {
+  const chunk_view *r = (const chunk_view *)vctx;
+  const chunk_ctx *c = r->c;
+  int d = c->P->head_dim;
+  int64_t j = r->lo + idx, p0 = c->pos0[r->b];
+  if (j >= p0) {
+    memcpy(k_row, r->k_new + (size_t)(j - p0) * d, sizeof(double) * d);
+    memcpy(v_row, r->v_new + (size_t)(j - p0) * d, sizeof(double) * d);
+    return;
+  }
+  int64_t s = oracle_cache_slot(c->kind, j, c->slots);
+  size_t off = (((size_t)r->b * c->P->n_kv_heads + r->g) * c->slots + s) * d;
+  for (int i = 0; i < d; ++i) {
+    k_row[i] = oracle_bf16_to_double(c->k_cache[off + i]);
+    v_row[i] = oracle_bf16_to_double(c->v_cache[off + i]);
+  }
+}
+
+static void chunk_job(void *vctx, int64_t r) {
+  chunk_ctx *c = (chunk_ctx *)vctx;
+  const oracle_params *P = c->P;
+  int d = P->head_dim, Hq = P->n_q_heads, Hkv = P->n_kv_heads, G = Hq / Hkv;
+  int64_t b = c->rows_b[r], i = c->rows_i[r];
+  int64_t t = c->pos0[b] + i;
+  int64_t lo = 0;
+  while (!oracle_visible(c->kind, t, lo, P->window)) ++lo;
+  int64_t n = t - lo + 1;
+  /* the new tokens m0 .. i of this sequence that are visible, prepared at their own
+   * positions (rows below m0 are never read) */
+  int64_t m0 = lo > c->pos0[b] ? lo - c->pos0[b] : 0;
+  double *kv_new = (double *)malloc(sizeof(double) * 2 * (size_t)(i + 1) * d);
+  double *scores = (double *)malloc(sizeof(double) * n);
+  double *q = (double *)malloc(sizeof(double) * d);
+  for (int h = 0; h < Hq; ++h) {
+    int g = h / G;
+    if (h % G == 0) {
+      for (int64_t m = m0; m <= i; ++m) {
+        size_t in_off = (((size_t)b * c->T + m) * Hkv + g) * d;
+        prepare_key(c->kind, P, c->k + in_off, c->kw, c->pos0[b] + m, kv_new + (size_t)m * d);
+        for (int e = 0; e < d; ++e)
+          kv_new[(size_t)(i + 1) * d + (size_t)m * d + e] = oracle_bf16_to_double(c->v[in_off + e]);
+      }
+    }
+    chunk_view view = {c, b, g, lo, kv_new, kv_new + (size_t)(i + 1) * d};
+    size_t q_off = (((size_t)b * c->T + i) * Hq + h) * d;
+    prepare_query(c->kind, P, c->q + q_off, c->qw, t, q);
+    attend_one(P, q, n, chunk_row, &view, c->gate + q_off, (double)c->bias[h], scores,
+               c->out + ((size_t)r * Hq + h) * d);
+  }
+  free(kv_new); free(scores); free(q);
+}
+
+int oracle_prefill_chunk_rows(int kind, const oracle_params *P, int B, int T,
+                              const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                              const uint16_t *gate, const float *q_norm_w, const float *k_norm_w,
+                              const float *gate_bias, const int64_t *pos0,
+                              const uint16_t *k_cache, const uint16_t *v_cache, int64_t slots,
+                              int64_t n_rows, const int64_t *rows_b, const int64_t *rows_i,
+                              double *out, int n_threads) {
+  if (!P || P->n_kv_heads <= 0 || P->n_q_heads % P->n_kv_heads) return -1;
+  for (int b = 0; b < B; ++b) {
+    if (pos0[b] < 0) return -1;
+    if (kind == ORACLE_GLOBAL && pos0[b] + T > slots) return -1;
+    if (kind == ORACLE_LOCAL && slots < P->window) return -1;
+  }
+  for (int64_t r = 0; r < n_rows; ++r)
+    if (rows_b[r] < 0 || rows_b[r] >= B || rows_i[r] < 0 || rows_i[r] >= T) return -1;
+  int d = P->head_dim;
+  double *qw = (double *)malloc(sizeof(double) * d), *kw = (double *)malloc(sizeof(double) * d);
+  for (int i = 0; i < d; ++i) { qw[i] = q_norm_w[i]; kw[i] = k_norm_w[i]; }
+  chunk_ctx c = {kind, P, B, T, q, k, v, gate, qw, kw, gate_bias, pos0, k_cache, v_cache, slots,
+                 rows_b, rows_i, out};
+  run_parallel(chunk_job, &c, n_rows, n_threads);
+  free(qw); free(kw);
+  return 0;
+}
+
 /* Expected cache rows written for one token at position j: the prepared key
  * rounded to the nearest bf16 and the raw value bits, one row per KV head
  * ([Hkv][d] each).  Tests compare these with what the device wrote at slot

@@ -340,6 +340,81 @@ def test_decode_after_cache_fill_matches_prefill(orc, kind, T):
         assert np.max(np.abs(bad - ref)) > 0.05
 
 
+# ---------------------------------------------------------------- chunked prefill
+def _small_chunk_problem(B, T, seed, d=16, Hq=6, Hkv=2):
+    q, gate = _rand((B, T, Hq * d), seed, "q"), _rand((B, T, Hq * d), seed, "g")
+    k, v = _rand((B, T, Hkv * d), seed, "k"), _rand((B, T, Hkv * d), seed, "v")
+    qw, kw = wl.norm_weight(seed, "qw")[:d], wl.norm_weight(seed, "kw")[:d]
+    bias = np.linspace(-0.5, 0.5, Hq).astype(np.float32)
+    return q, k, v, gate, qw, kw, bias
+
+
+@pytest.mark.parametrize("kind", [0, 1])
+def test_chunk_of_one_token_equals_decode(orc, kind):
+    """A chunk of one new token is a decode step: same visible keys, same cache
+    slots, the new key prepared exactly.  Decode itself is pinned above."""
+    d, Hq, Hkv, W = 16, 6, 2, 8
+    P = orc.params(n_q_heads=Hq, n_kv_heads=Hkv, head_dim=d, window=W)
+    pos = np.array([0, 3, 8, 29], np.int64)
+    B, slots = pos.size, (W if kind == orc.LOCAL else 40)
+    q, k, v, gate, qw, kw, bias = _small_chunk_problem(B, 1, 21)
+    kc = _rand((B, Hkv, slots, d), 21, "kc")
+    vc = _rand((B, Hkv, slots, d), 21, "vc")
+    got = orc.prefill_chunk(kind, P, q, k, v, gate, qw, kw, bias, pos, kc, vc)[:, 0]
+    ref = orc.decode(kind, P, q[:, 0], k[:, 0], v[:, 0], gate[:, 0], qw, kw, bias, pos, kc, vc)
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("kind", [0, 1])
+def test_chunk_at_position_zero_equals_prefill_and_reads_no_cache(orc, kind):
+    """With pos0 = 0 nothing is cached yet: the chunk is a plain prefill, whatever
+    the cache buffer holds."""
+    d, Hq, Hkv, W = 16, 6, 2, 8
+    P = orc.params(n_q_heads=Hq, n_kv_heads=Hkv, head_dim=d, window=W)
+    B, T = 2, 19
+    q, k, v, gate, qw, kw, bias = _small_chunk_problem(B, T, 22)
+    slots = W if kind == orc.LOCAL else T
+    kc = np.full((B, Hkv, slots, d), _bf16([1e30])[0], np.uint16)   # poison
+    vc = kc.copy()
+    got = orc.prefill_chunk(kind, P, q, k, v, gate, qw, kw, bias, np.zeros(B, np.int64), kc, vc)
+    ref = orc.prefill(kind, P, q, k, v, gate, qw, kw, bias)
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("kind", [0, 1])
+def test_chunk_after_cache_fill_matches_prefill(orc, kind):
+    """Sequence b's first P_b tokens go into the cache as the oracle's own rows
+    (bf16), then the remaining tokens arrive as one chunk: every chunk row equals
+    the one-shot prefill row at the same position, up to the bf16 rounding of the
+    cached keys.  The ring at the wrong slot, or the chunk's positions off by
+    one, differ by far more."""
+    d, Hq, Hkv, W = 16, 6, 2, 8
+    P = orc.params(n_q_heads=Hq, n_kv_heads=Hkv, head_dim=d, window=W)
+    B, Ttot = 2, 27
+    pos0 = np.array([5, 13], np.int64)            # chunk lengths 22 and 14: use T = 14
+    T = 14
+    q, k, v, gate, qw, kw, bias = _small_chunk_problem(B, Ttot, 23)
+    ref = orc.prefill(kind, P, q, k, v, gate, qw, kw, bias)
+    slots = W if kind == orc.LOCAL else Ttot + 1   # room for the shifted call below
+    kc = np.zeros((B, Hkv, slots, d), np.uint16)
+    vc = np.zeros_like(kc)
+    for b in range(B):
+        for j in range(pos0[b]):
+            kr, vr = orc.kv_row(kind, P, k[b, j], v[b, j], kw, j)
+            s = orc.cache_slot(kind, j, slots)
+            kc[b, :, s], vc[b, :, s] = kr, vr
+    sl = [np.stack([x[b, pos0[b]:pos0[b] + T] for b in range(B)]) for x in (q, k, v, gate)]
+    got = orc.prefill_chunk(kind, P, *sl, qw, kw, bias, pos0, kc, vc)
+    want = np.stack([ref[b, pos0[b]:pos0[b] + T] for b in range(B)])
+    np.testing.assert_allclose(got, want, rtol=2e-2, atol=2e-2)
+    if kind == orc.LOCAL:
+        bad = orc.prefill_chunk(kind, P, *sl, qw, kw, bias, pos0, np.roll(kc, 1, axis=2),
+                                np.roll(vc, 1, axis=2))
+        assert np.max(np.abs(bad[:, 0] - want[:, 0])) > 0.05
+    shifted = orc.prefill_chunk(kind, P, *sl, qw, kw, bias, pos0 + 1, kc, vc)
+    assert np.max(np.abs(shifted - want)) > 0.05
+
+
 # ---------------------------------------------------------------- bf16
 def test_bf16_rounding_ties_to_even(orc):
     cases = {1.0 + 2.0 ** -8: 0x3F80, 1.0 + 3 * 2.0 ** -8: 0x3F82, -2.5: 0xC020,

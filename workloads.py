@@ -165,6 +165,42 @@ def decode_inputs(kind: int, ctx: np.ndarray, slots: int, seed: int, layer: str 
     return di
 
 
+@dataclass
+class ChunkInputs:
+    """One chunked-prefill call: T new tokens per sequence at positions pos0[b] ..
+    pos0[b] + T - 1, plus the cache as it was before the call (rows of earlier
+    positions; same layout and meaning as DecodeInputs' caches)."""
+    B: int
+    T: int
+    kind: int
+    pos0: np.ndarray    # [B] int64
+    q: np.ndarray       # [B, T, 48*128]
+    k: np.ndarray       # [B, T, 8*128]
+    v: np.ndarray
+    gate: np.ndarray
+    q_norm_w: np.ndarray
+    k_norm_w: np.ndarray
+    gate_bias: np.ndarray
+    slots: int
+    k_cache: np.ndarray | None = None  # [B, 8, slots, 128] uint16
+    v_cache: np.ndarray | None = None
+
+
+def chunk_inputs(kind: int, T: int, pos0, slots: int, seed: int, layer: str = "L",
+                 with_cache: bool = True) -> ChunkInputs:
+    pos0 = np.asarray(pos0, dtype=np.int64)
+    B = int(pos0.shape[0])
+    p = prefill_inputs(B, T, seed, layer=f"chunk/{layer}")
+    ci = ChunkInputs(B=B, T=T, kind=kind, pos0=pos0, q=p.q, k=p.k, v=p.v, gate=p.gate,
+                     q_norm_w=p.q_norm_w, k_norm_w=p.k_norm_w, gate_bias=p.gate_bias,
+                     slots=int(slots))
+    if with_cache:
+        shape = (B, N_KV_HEADS, int(slots), HEAD_DIM)
+        ci.k_cache = normal_bf16(shape, seed, f"chunk/{layer}/kcache")
+        ci.v_cache = normal_bf16(shape, seed, f"chunk/{layer}/vcache")
+    return ci
+
+
 def device_normal_bf16_(tensor, seed: int, tag: str):
     """Fill a CUDA bf16 tensor in place with seeded N(0,1) draws (torch Philox).
 
