@@ -27,7 +27,7 @@ STATUS = {
 EXPORTS = (
     "beam_default_params", "beam_kv_layout", "beam_prefill_workspace_bytes", "beam_attn_prefill",
     "beam_kv_append", "beam_decode_workspace_bytes", "beam_attn_decode", "beam_status_string",
-    "beam_attn_decode_noalloc",
+    "beam_attn_decode_noalloc", "beam_prefill_chunk_workspace_bytes", "beam_attn_prefill_chunk",
 )
 
 
@@ -77,6 +77,11 @@ def lib() -> ctypes.CDLL:
         L.beam_attn_prefill.restype = ctypes.c_int
         L.beam_attn_prefill.argtypes = [ctypes.c_int, pp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp,
                                         vp, vp, lp, vp, sz, vp, vp]
+        L.beam_prefill_chunk_workspace_bytes.restype = sz
+        L.beam_prefill_chunk_workspace_bytes.argtypes = [ctypes.c_int, pp, i32, i32]
+        L.beam_attn_prefill_chunk.restype = ctypes.c_int
+        L.beam_attn_prefill_chunk.argtypes = [ctypes.c_int, pp, i32, i32, vp, vp, vp, vp, vp, vp, vp,
+                                              vp, vp, vp, vp, lp, vp, sz, vp, vp]
         L.beam_kv_append.restype = ctypes.c_int
         L.beam_kv_append.argtypes = [ctypes.c_int, pp, i32, i32, vp, vp, vp, vp, vp, vp, lp, vp, vp]
         L.beam_decode_workspace_bytes.restype = sz
@@ -161,6 +166,28 @@ def beam_attn_prefill(kind, params, q, k, v, gate, q_norm_w, k_norm_w, gate_bias
         ctypes.byref(layout) if layout is not None else None, _ptr(workspace), ws_bytes,
         _ptr(dev_status), _stream(stream))
     _check("beam_attn_prefill", rc)
+    return out
+
+
+def beam_prefill_chunk_workspace_bytes(kind: int, params: Params, B: int, T: int) -> int:
+    return lib().beam_prefill_chunk_workspace_bytes(kind, ctypes.byref(params), B, T)
+
+
+def beam_attn_prefill_chunk(kind, params, q, k, v, gate, q_norm_w, k_norm_w, gate_bias, pos0, out,
+                            k_cache, v_cache, layout: KVLayout, workspace=None, dev_status=None,
+                            stream=None):
+    """Chunked prefill: q, gate [B, T, 6144]; k, v [B, T, 1024] bf16; pos0 [B] int64 on the
+    device (position of each sequence's first new token); caches as for decode."""
+    B, T = q.shape[0], q.shape[1]
+    need = beam_prefill_chunk_workspace_bytes(kind, params, B, T)
+    if workspace is None and need:
+        workspace = _workspace(need, q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib().beam_attn_prefill_chunk(
+        kind, ctypes.byref(params), B, T, _ptr(q), _ptr(k), _ptr(v), _ptr(gate), _ptr(q_norm_w),
+        _ptr(k_norm_w), _ptr(gate_bias), _ptr(pos0), _ptr(out), _ptr(k_cache), _ptr(v_cache),
+        ctypes.byref(layout), _ptr(workspace), ws_bytes, _ptr(dev_status), _stream(stream))
+    _check("beam_attn_prefill_chunk", rc)
     return out
 
 

@@ -137,6 +137,53 @@ int make_head_map(CUtensorMap *map, const void *base, int heads, int T, int B) {
   return r == CUDA_SUCCESS ? BEAM_OK : BEAM_ERR_CUDA;
 }
 
+// 4-D bf16 map over a head-major cache [B][8][slots][128] with the layout's strides:
+// coordinates (d, slot, head, b), the same boxes; slots past the capacity read as zeros.
+int make_cache_map(CUtensorMap *map, const void *base, const beam_kv_layout_t *L, int B) {
+  const cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)L->slots_per_seq, (cuuint64_t)kHkv,
+                              (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)L->stride_slot * 2, (cuuint64_t)L->stride_head * 2,
+                                 (cuuint64_t)L->stride_seq * 2};
+  const cuuint32_t box[4] = {64, (cuuint32_t)kTcBN, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = g_encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base),
+                              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? BEAM_OK : BEAM_ERR_CUDA;
+}
+
+// The persistent tcgen05 attention kernel over B sequences of T query rows.  The caller
+// fills the pointers and the chunk fields of `fa`; the shape and scale fields are set here.
+int launch_prefill_attention(int kind, const beam_attn_params *p, int32_t B, int32_t T,
+                             const CUtensorMap &tm_q, const CUtensorMap &tm_k,
+                             const CUtensorMap &tm_v, PrefillTcArgs fa, const DeviceInfo *dev,
+                             cudaStream_t s) {
+  fa.eps = p->rms_eps;
+  fa.B = B;
+  fa.T = T;
+  fa.kind = kind;
+  fa.window = p->window;
+  fa.n_qblocks = (T + kTcBM - 1) / kTcBM;
+  fa.scale_log2 = p->softmax_scale * kLog2e;
+  fa.ssmax_base = p->ssmax_base;
+  fa.ssmax_exp = p->ssmax_exp;
+  // Fault injection for tests of the device-timeout path: with BEAM_FAULT_INJECT set to
+  // prefill_wait_stall, the attention kernel's MMA issuer waits on a barrier that nothing
+  // arrives at, so the wait runs out and the call reports BEAM_ERR_DEVICE_TIMEOUT.
+  {
+    const char *f = std::getenv("BEAM_FAULT_INJECT");
+    fa.fault_stall = f != nullptr && std::strcmp(f, "prefill_wait_stall") == 0;
+  }
+  const int64_t n_units = (int64_t)fa.n_qblocks * (kHq / 2) * B;
+  if (n_units > INT32_MAX) return BEAM_ERR_UNSUPPORTED;
+  fa.n_units = (int)n_units;
+  // persistent: one CTA per SM (the kernel's shared memory admits one per SM)
+  const int grid = (int)std::min<int64_t>(n_units, dev->sm_count);
+  prefill_tc_kernel<<<grid, kTcThreads, kTcSmemBytes, s>>>(tm_q, tm_k, tm_v, fa);
+  return launch_status();
+}
+
 // Decode split size: cache slots per CTA.  A local ring is cut into at most four
 // splits (one thread-block cluster); a global
 // cache is cut so that the grid holds several waves of the SMs at its largest
@@ -283,35 +330,140 @@ int beam_attn_prefill(int kind, const beam_attn_params *p, int32_t B, int32_t T,
   if ((st = make_head_map(&tm_k, kn, kHkv, T, B))) return st;
   if ((st = make_head_map(&tm_v, v, kHkv, T, B))) return st;
   PrefillTcArgs fa;
+  memset(&fa, 0, sizeof fa);
   fa.q_norm_w = q_norm_w;
   fa.rope_tab = kind == BEAM_LOCAL ? rope_tab : nullptr;
-  fa.eps = p->rms_eps;
   fa.gate = static_cast<const uint16_t *>(gate);
   fa.gate_bias = gate_bias;
   fa.out = static_cast<uint16_t *>(out);
   fa.status = dev_status;
-  fa.B = B;
-  fa.T = T;
-  fa.kind = kind;
-  fa.window = p->window;
-  fa.n_qblocks = (T + kTcBM - 1) / kTcBM;
-  fa.scale_log2 = p->softmax_scale * kLog2e;
-  fa.ssmax_base = p->ssmax_base;
-  fa.ssmax_exp = p->ssmax_exp;
-  // Fault injection for tests of the device-timeout path: with BEAM_FAULT_INJECT set to
-  // prefill_wait_stall, the attention kernel's MMA issuer waits on a barrier that nothing
-  // arrives at, so the wait runs out and the call reports BEAM_ERR_DEVICE_TIMEOUT.
-  {
-    const char *f = std::getenv("BEAM_FAULT_INJECT");
-    fa.fault_stall = f != nullptr && std::strcmp(f, "prefill_wait_stall") == 0;
+  return launch_prefill_attention(kind, p, B, T, tm_q, tm_k, tm_v, fa, dev, s);
+}
+
+size_t beam_prefill_chunk_workspace_bytes(int kind, const beam_attn_params *p, int32_t B,
+                                          int32_t T) {
+  if (!p || B <= 0 || T <= 0 || p->window < 1) return 0;
+  if (kind != BEAM_LOCAL) return 0;  // a global chunk reads and writes the cache itself
+  const size_t rows = (size_t)B * ((size_t)p->window - 1 + T);
+  // keys and values [B][window - 1 + T][8][128] bf16, then the RoPE table [B][T][128] fp32
+  return 2 * round_up(rows * kHkv * kD * 2, 256) + round_up((size_t)B * T * 128 * 4, 256);
+}
+
+int beam_attn_prefill_chunk(int kind, const beam_attn_params *p, int32_t B, int32_t T,
+                            const void *q, const void *k, const void *v, const void *gate,
+                            const float *q_norm_w, const float *k_norm_w, const float *gate_bias,
+                            const int64_t *pos0, void *out, void *k_cache, void *v_cache,
+                            const beam_kv_layout_t *layout, void *workspace,
+                            size_t workspace_bytes, int32_t *dev_status, beam_stream_t stream) {
+  int st = check_params(kind, p);
+  if (st) return st;
+  if (B < 0 || T < 0) return BEAM_ERR_INVALID_ARG;
+  if (B == 0 || T == 0) return BEAM_OK;
+  if (!q || !k || !v || !gate || !q_norm_w || !k_norm_w || !gate_bias || !pos0 || !out ||
+      !k_cache || !v_cache)
+    return BEAM_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(gate) || !aligned16(out) ||
+      !aligned16(q_norm_w) || !aligned16(k_norm_w) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      !aligned16(workspace) || (reinterpret_cast<uintptr_t>(pos0) & 7u))
+    return BEAM_ERR_ALIGNMENT;
+  if ((st = check_layout(kind, p, layout))) return st;
+  const bool local = kind == BEAM_LOCAL;
+  if (!local && layout->slots_per_seq < T) return BEAM_ERR_CAPACITY;
+  if (!local && layout->slots_per_seq > INT32_MAX - kTcBN) return BEAM_ERR_UNSUPPORTED;
+  const size_t need = beam_prefill_chunk_workspace_bytes(kind, p, B, T);
+  if (need && (!workspace || workspace_bytes < need)) return BEAM_ERR_WORKSPACE;
+  const int64_t ext_rows = local ? (int64_t)p->window - 1 + T : T;
+  if ((int64_t)B * ext_rows > INT32_MAX) return BEAM_ERR_UNSUPPORTED;
+  DeviceInfo *dev = nullptr;
+  if ((st = device_info(&dev))) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+  const size_t ext_bytes = round_up((size_t)B * ext_rows * kHkv * kD * 2, 256);
+  uint16_t *k_ext = local ? static_cast<uint16_t *>(workspace) : nullptr;
+  uint16_t *v_ext = local ? reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(workspace) +
+                                                         ext_bytes)
+                          : nullptr;
+  float *rope_tab = local ? reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
+                                                      2 * ext_bytes)
+                          : nullptr;
+  const int prefix = local ? p->window - 1 : 0;
+
+  // 1. the ring rows the chunk still sees (local), or the value padding (global)
+  ChunkPrepArgs ca;
+  ca.pos0 = pos0;
+  ca.k_cache = static_cast<const uint16_t *>(k_cache);
+  ca.v_cache = static_cast<uint16_t *>(v_cache);
+  ca.stride_seq = layout->stride_seq;
+  ca.stride_head = layout->stride_head;
+  ca.slots = layout->slots_per_seq;
+  ca.k_ext = k_ext;
+  ca.v_ext = v_ext;
+  ca.ext_rows = (int)ext_rows;
+  ca.prefix = prefix;
+  ca.T = T;
+  ca.window = p->window;
+  ca.kind = kind;
+  const int64_t prep_ctas = (int64_t)B * (local ? prefix : kChunkPadRows);
+  if (prep_ctas > 0) {
+    chunk_prep_kernel<<<(unsigned)prep_ctas, 128, 0, s>>>(ca);
+    if ((st = launch_status())) return st;
   }
-  const int64_t n_units = (int64_t)fa.n_qblocks * (kHq / 2) * B;
-  if (n_units > INT32_MAX) return BEAM_ERR_UNSUPPORTED;
-  fa.n_units = (int)n_units;
-  // persistent: one CTA per SM (the kernel's shared memory admits one per SM)
-  const int grid = (int)std::min<int64_t>(n_units, dev->sm_count);
-  prefill_tc_kernel<<<grid, kTcThreads, kTcSmemBytes, s>>>(tm_q, tm_k, tm_v, fa);
-  return launch_status();
+
+  // 2. prepared keys (and raw values) of the new tokens: into the cache and, for a local
+  //    layer, behind the earlier rows; the RoPE table at each sequence's own positions
+  PrologueArgs pa;
+  memset(&pa, 0, sizeof pa);
+  pa.k = static_cast<const uint16_t *>(k);
+  pa.v = static_cast<const uint16_t *>(v);
+  pa.qw = q_norm_w;
+  pa.kw = k_norm_w;
+  pa.k_out = k_ext;
+  pa.v_out = v_ext;
+  pa.out_rows = (int)ext_rows;
+  pa.out_row0 = prefix;
+  pa.k_cache = static_cast<uint16_t *>(k_cache);
+  pa.v_cache = static_cast<uint16_t *>(v_cache);
+  pa.stride_seq = layout->stride_seq;
+  pa.stride_head = layout->stride_head;
+  pa.slots = layout->slots_per_seq;
+  pa.pos0 = pos0;
+  pa.rope_tab = rope_tab;
+  pa.rope_per_seq = 1;
+  pa.whole_seq = 1;
+  pa.status = dev_status;
+  pa.T = T;
+  pa.kind = kind;
+  pa.window = p->window;
+  pa.eps = p->rms_eps;
+  fill_inv_freq(pa.inv_freq, p->rope_theta);
+  prologue_kernel<<<(unsigned)((size_t)B * T), 128, 0, s>>>(pa);
+  if ((st = launch_status())) return st;
+
+  // 3. attention of the new rows over the earlier and the new keys
+  if ((st = encode_fn())) return st;
+  CUtensorMap tm_q, tm_k, tm_v;
+  if ((st = make_head_map(&tm_q, q, kHq, T, B))) return st;
+  if (local) {
+    if ((st = make_head_map(&tm_k, k_ext, kHkv, (int)ext_rows, B))) return st;
+    if ((st = make_head_map(&tm_v, v_ext, kHkv, (int)ext_rows, B))) return st;
+  } else {
+    if ((st = make_cache_map(&tm_k, k_cache, layout, B))) return st;
+    if ((st = make_cache_map(&tm_v, v_cache, layout, B))) return st;
+  }
+  PrefillTcArgs fa;
+  memset(&fa, 0, sizeof fa);
+  fa.q_norm_w = q_norm_w;
+  fa.rope_tab = rope_tab;
+  fa.rope_rows = T;
+  fa.gate = static_cast<const uint16_t *>(gate);
+  fa.gate_bias = gate_bias;
+  fa.out = static_cast<uint16_t *>(out);
+  fa.status = dev_status;
+  fa.pos0 = pos0;
+  fa.slots = layout->slots_per_seq;
+  fa.ext_prefix = prefix;
+  fa.kv_slot_major = local ? 0 : 1;
+  return launch_prefill_attention(kind, p, B, T, tm_q, tm_k, tm_v, fa, dev, s);
 }
 
 int beam_kv_append(int kind, const beam_attn_params *p, int32_t B, int32_t T, const void *k,

@@ -77,6 +77,12 @@ struct PrefillTcArgs {
   int B, T, kind, window, n_qblocks, n_units;
   float scale_log2, ssmax_base, ssmax_exp;
   int fault_stall;        // tests only: the MMA issuer first waits on a barrier never arrived at
+  // Chunked prefill (new tokens after pos0[b] cached ones); pos0 == null for a plain prefill.
+  const int64_t *pos0;    // [B] position of each sequence's first new token
+  int64_t slots;          // global: cache slots per sequence (the K/V maps cover the cache)
+  int ext_prefix;         // local: rows of earlier keys in front of the new ones (window - 1)
+  int kv_slot_major;      // K/V maps take coordinates (d, slot, head, b), not (d, head, t, b)
+  int rope_rows;          // rows per sequence in rope_tab (0: one table for all sequences)
 };
 
 namespace tcd {
@@ -158,8 +164,17 @@ __device__ __forceinline__ void tc_drain(uint32_t bar, uint32_t count, int32_t *
 // Work unit u -> (sequence, q block, head pair): sequence-major, so the CTAs share one
 // sequence's K/V (8 heads x T x 512 B, 32 MiB at T = 8192) while it stays in L2, and within
 // a sequence the units with more key blocks come first.
+// Keys are addressed by their coordinate in the K/V maps: query row r of the unit has its
+// own key at kq + r and sees the coordinates max(kq + r - window + 1, kmin) .. kq + r
+// (local) or 0 .. kq + r (global).  A plain prefill has kq = q0, kmin = 0.  A chunk of a
+// global layer reads the cache itself (coordinate = slot = position, kq = pos0 + q0); a
+// chunk of a local layer reads keys laid out as window - 1 earlier rows, then the new ones
+// (kq = window - 1 + q0; rows below kmin precede the sequence's first token).  t0 is the
+// position of row 0 (for a(p)); `bad` marks a sequence whose pos0 is out of range: its
+// rows are computed on clamped coordinates and not written.
 struct TcUnit {
-  int qb, pair, b, q0, kb_lo, n_blk;
+  int qb, pair, b, q0, kb_lo, n_blk, kq, kmin, t0;
+  bool bad;
 };
 __device__ __forceinline__ TcUnit tc_unit(const PrefillTcArgs &a, int u) {
   TcUnit w;
@@ -169,8 +184,32 @@ __device__ __forceinline__ TcUnit tc_unit(const PrefillTcArgs &a, int u) {
   w.qb = a.n_qblocks - 1 - rem / (kHq / 2);
   w.pair = rem % (kHq / 2);
   w.q0 = w.qb * kTcBM;
-  w.kb_lo = a.kind == BEAM_LOCAL ? max(0, w.q0 - a.window + 1) / kTcBN : 0;
-  w.n_blk = w.qb - w.kb_lo + 1;  // the last visible key of the unit is in block qb
+  w.kq = w.q0;
+  w.kmin = 0;
+  w.t0 = w.q0;
+  w.bad = false;
+  const bool local = a.kind == BEAM_LOCAL;
+  if (a.pos0) {
+    int64_t p0 = a.pos0[w.b];
+    if (p0 < 0) {
+      w.bad = true;
+      p0 = 0;
+    }
+    if (local) {
+      w.kq = a.ext_prefix + w.q0;
+      w.kmin = a.ext_prefix - (int)min(p0, (int64_t)a.ext_prefix);
+    } else {
+      if (p0 > a.slots - a.T) {
+        w.bad = true;
+        p0 = a.slots - a.T;   // >= 0: the host checks T <= slots
+      }
+      w.kq = (int)p0 + w.q0;
+      w.t0 = w.kq;
+    }
+  }
+  w.kb_lo = local ? max(w.kmin, w.kq - a.window + 1) / kTcBN : 0;
+  // the last visible key of the unit is the own key of its last row below T
+  w.n_blk = (w.kq + min(kTcBM - 1, a.T - 1 - w.q0)) / kTcBN - w.kb_lo + 1;
   return w;
 }
 
@@ -224,30 +263,44 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc::prefetch_tmap(&tm_k);
       tc::prefetch_tmap(&tm_v);
       struct Cursor {  // walks (unit, block) in the order the MMA issuer consumes them
-        int u, j;
-        TcUnit w;
+        int u, j, b, g, kb_lo, n_blk;
         bool valid;
+      };
+      auto set_unit = [&](Cursor &c) {
+        c.valid = c.u < a.n_units;
+        if (c.valid) {
+          const TcUnit w = tc_unit(a, c.u);
+          c.b = w.b;
+          c.g = (2 * w.pair) / kGroup;
+          c.kb_lo = w.kb_lo;
+          c.n_blk = w.n_blk;
+        }
       };
       auto start = [&](Cursor &c) {
         c.u = blockIdx.x;
         c.j = 0;
-        c.valid = c.u < a.n_units;
-        if (c.valid) c.w = tc_unit(a, c.u);
+        set_unit(c);
       };
       auto advance = [&](Cursor &c) {
-        if (++c.j == c.w.n_blk) {
+        if (++c.j == c.n_blk) {
           c.j = 0;
           c.u += gridDim.x;
-          c.valid = c.u < a.n_units;
-          if (c.valid) c.w = tc_unit(a, c.u);
+          set_unit(c);
         }
       };
       auto load = [&](const Cursor &c, bool is_v, uint32_t slot) {
-        const int g = (2 * c.w.pair) / kGroup, key0 = (c.w.kb_lo + c.j) * kTcBN;
+        const int g = c.g, key0 = (c.kb_lo + c.j) * kTcBN;
         tc::mbar_expect_tx(bar(tcd::kKVFull + slot), kTcTileBytes);
-        for (int hf = 0; hf < 2; ++hf)
-          tc::tma_load_4d(sbase + kTcSmemKV + slot * kTcTileBytes + hf * kTcHalfBytes,
-                          is_v ? &tm_v : &tm_k, bar(tcd::kKVFull + slot), hf * 64, g, key0, c.w.b);
+        const uint32_t dst = sbase + kTcSmemKV + slot * kTcTileBytes;
+        const CUtensorMap *map = is_v ? &tm_v : &tm_k;
+        for (int hf = 0; hf < 2; ++hf) {
+          if (a.kv_slot_major)
+            tc::tma_load_4d(dst + hf * kTcHalfBytes, map, bar(tcd::kKVFull + slot), hf * 64, key0, g,
+                            c.b);
+          else
+            tc::tma_load_4d(dst + hf * kTcHalfBytes, map, bar(tcd::kKVFull + slot), hf * 64, g, key0,
+                            c.b);
+        }
       };
       Cursor kc, vc;
       start(kc);
@@ -393,7 +446,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const TcUnit w = tc_unit(a, u);
       const int tok = w.q0 + r;
       const float4 *tab =
-          local ? reinterpret_cast<const float4 *>(a.rope_tab + (size_t)min(tok, a.T - 1) * 128)
+          local ? reinterpret_cast<const float4 *>(
+                      a.rope_tab + ((size_t)w.b * a.rope_rows + min(tok, a.T - 1)) * 128)
                 : nullptr;
       float4 tb[8];   // per slot: cos lo, cos hi, sin lo, sin hi of one chunk of 8
       auto tab_load = [&](int c, int slot) {
@@ -490,10 +544,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     bool ok = true;
     for (int u = blockIdx.x, n = 0; ok && u < a.n_units; u += gridDim.x, ++n) {
       const TcUnit w = tc_unit(a, u);
-      const int tok = w.q0 + r;
+      // the row's visible key coordinates are lo_base .. hi_base; rows of a sequence whose
+      // pos0 is out of range count as past T (computed, not written)
+      const int hi_base = w.kq + r;
+      const int lo_base = local ? max(hi_base - a.window + 1, w.kmin) : -(1 << 30);
+      const int tok = w.bad ? a.T : w.q0 + r;
       const int h = 2 * w.pair + t;
       float factor = a.scale_log2;
-      if (!local) factor *= ssmax_factor((int64_t)tok + 1, a.ssmax_base, a.ssmax_exp);
+      if (!local) factor *= ssmax_factor((int64_t)w.t0 + r + 1, a.ssmax_base, a.ssmax_exp);
       float m = -INFINITY, l = 0.f;
       for (int j = 0; j < w.n_blk; ++j, ++it) {
         if (!(ok = tc_wait(bar(tcd::kSFull + t), it & 1u, abort, a.status))) break;
@@ -502,13 +560,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c) tc::tmem_ld32(t_s + 32 * c, sr[c]);
         tc::tmem_ld_wait();
-        const int kb = w.kb_lo + j;
-        const bool need_mask =
-            kb == w.qb || (local && (w.q0 + kTcBM - 1) - kb * kTcBN > a.window - 1);
-        if (need_mask) {
-          // key kb*128 + i is visible to row tok iff lo <= i <= hi
-          const int hi = tok - kb * kTcBN;
-          const int lo = local ? tok - a.window + 1 - kb * kTcBN : INT_MIN;
+        const int k0 = (w.kb_lo + j) * kTcBN;
+        // masked only where the block holds a key outside this row's range (a warp whose
+        // rows disagree takes the masking path)
+        if (k0 + kTcBN - 1 > hi_base || k0 < lo_base) {
+          // key k0 + i is visible to row r iff lo <= i <= hi
+          const int hi = hi_base - k0;
+          const int lo = lo_base - k0;
 #pragma unroll
           for (int c = 0; c < 4; ++c)
 #pragma unroll

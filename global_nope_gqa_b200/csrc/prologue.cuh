@@ -27,12 +27,17 @@ struct PrologueArgs {
   const float *qw;       // [128]
   const float *kw;       // [128]
   uint16_t *q_out;       // [tokens][48*128] prepared queries, or null
-  uint16_t *k_out;       // [tokens][8*128] prepared keys, or null
+  uint16_t *k_out;       // prepared keys [B][out_rows][8*128], or null
+  uint16_t *v_out;       // raw values copied to [B][out_rows][8*128], or null
+  int out_rows;          // rows per sequence in k_out / v_out (0: T)
+  int out_row0;          // row of token 0 there (the rows before it hold earlier keys)
   uint16_t *k_cache;     // layer caches, or null
   uint16_t *v_cache;
   int64_t stride_seq, stride_head, slots;
   const int64_t *pos0;   // device [B]: position of token 0 of each sequence, or null (= 0)
-  float *rope_tab;       // local layers, or null: [T][128] cos (64) then sin (64) of token i
+  float *rope_tab;       // local layers, or null: cos (64) then sin (64) of each token's angles
+  int rope_per_seq;      // rope_tab is [B][T][128] (own positions) rather than [T][128] (0 .. T-1)
+  int whole_seq;         // a sequence whose tokens do not all fit is not written at all
   int32_t *status;
   int T;                 // tokens per sequence in this call
   int kind;
@@ -109,6 +114,13 @@ __global__ void __launch_bounds__(128) prologue_kernel(const PrologueArgs a) {
   // Cache target of this token.
   bool write_cache = a.k_cache != nullptr;
   int64_t slot = 0;
+  if (write_cache && a.whole_seq) {
+    const int64_t p0 = a.pos0 ? a.pos0[b] : 0;
+    if (p0 < 0 || (!local && p0 + a.T > a.slots)) {
+      if (threadIdx.x == 0 && i == 0) set_status(a.status, BEAM_ERR_CAPACITY);
+      write_cache = false;
+    }
+  }
   if (write_cache) {
     if (t < 0) {
       set_status(a.status, BEAM_ERR_CAPACITY);
@@ -127,10 +139,11 @@ __global__ void __launch_bounds__(128) prologue_kernel(const PrologueArgs a) {
 
   float cs[8], sn[8];
   if (local) rope_angles(a.inv_freq, t < 0 ? 0 : t, l16 & 7, cs, sn);
-  if (local && a.rope_tab && b == 0 && warp == 0 && lane < 8) {
-    // the same angles serve every head and sequence (positions 0 .. T-1): one table row
-    float4 *c4 = reinterpret_cast<float4 *>(a.rope_tab + (size_t)i * 128 + lane * 8);
-    float4 *s4 = reinterpret_cast<float4 *>(a.rope_tab + (size_t)i * 128 + 64 + lane * 8);
+  if (local && a.rope_tab && (a.rope_per_seq || b == 0) && warp == 0 && lane < 8) {
+    // the angles serve every head (and, at positions 0 .. T-1, every sequence)
+    const size_t trow = (size_t)(a.rope_per_seq ? tok : i) * 128;
+    float4 *c4 = reinterpret_cast<float4 *>(a.rope_tab + trow + lane * 8);
+    float4 *s4 = reinterpret_cast<float4 *>(a.rope_tab + trow + 64 + lane * 8);
     c4[0] = make_float4(cs[0], cs[1], cs[2], cs[3]);
     c4[1] = make_float4(cs[4], cs[5], cs[6], cs[7]);
     s4[0] = make_float4(sn[0], sn[1], sn[2], sn[3]);
@@ -149,7 +162,7 @@ __global__ void __launch_bounds__(128) prologue_kernel(const PrologueArgs a) {
     const bool is_v = row >= kHq + kHkv;
     if (is_q && (a.q == nullptr || a.q_out == nullptr)) continue;
     if (is_k && a.k_out == nullptr && !write_cache) continue;
-    if (is_v && !write_cache) continue;
+    if (is_v && !write_cache && a.v_out == nullptr) continue;
     const int head = is_q ? row : (is_k ? row - kHq : row - kHq - kHkv);
     const uint16_t *src = is_q ? a.q + (size_t)tok * (kHq * kD) + head * kD
                                : (is_k ? a.k : a.v) + (size_t)tok * (kHkv * kD) + head * kD;
@@ -159,14 +172,62 @@ __global__ void __launch_bounds__(128) prologue_kernel(const PrologueArgs a) {
     if (is_q) {
       *reinterpret_cast<uint4 *>(a.q_out + (size_t)tok * (kHq * kD) + head * kD + l16 * 8) = res;
     } else {
-      if (is_k && a.k_out)
-        *reinterpret_cast<uint4 *>(a.k_out + (size_t)tok * (kHkv * kD) + head * kD + l16 * 8) = res;
+      uint16_t *dst = is_k ? a.k_out : a.v_out;
+      if (dst) {
+        const size_t orow = (size_t)b * (a.out_rows ? a.out_rows : a.T) + a.out_row0 + i;
+        *reinterpret_cast<uint4 *>(dst + orow * (kHkv * kD) + head * kD + l16 * 8) = res;
+      }
       if (write_cache) {
         uint16_t *cache = is_k ? a.k_cache : a.v_cache;
         size_t off = (size_t)b * a.stride_seq + (size_t)head * a.stride_head + (size_t)slot * kD;
         *reinterpret_cast<uint4 *>(cache + off + l16 * 8) = res;
       }
     }
+  }
+}
+
+// Before the prologue of a chunked prefill (positions pos0[b] .. pos0[b] + T - 1 after
+// pos0[b] cached tokens).  Local layer: rows e = 0 .. L-1 (L = window - 1) of each
+// sequence's key and value buffers get the ring's rows of positions pos0[b] - L + e, i.e.
+// the earlier keys still inside the window of the chunk's first token, zeros before
+// position 0; this must run before the prologue overwrites ring slots.  Global layer: the
+// value slots from pos0[b] + T up to the next multiple of 128 (within the capacity) are
+// zeroed: the attention kernel reads whole 128-key blocks, and a masked key's weight is
+// exactly 0 but 0 times a non-finite stale value would not be.  One CTA of 128 threads
+// per row; thread x moves 8 coordinates of head x / 16.
+constexpr int kChunkPadRows = 128;  // global: CTAs per sequence (at most 127 slots to zero)
+
+struct ChunkPrepArgs {
+  const int64_t *pos0;
+  const uint16_t *k_cache;
+  uint16_t *v_cache;
+  int64_t stride_seq, stride_head, slots;
+  uint16_t *k_ext, *v_ext;   // local: [B][ext_rows][8*128]
+  int ext_rows, prefix, T, window, kind;
+};
+
+__global__ void __launch_bounds__(128) chunk_prep_kernel(const ChunkPrepArgs a) {
+  const int per_b = a.kind == BEAM_LOCAL ? a.prefix : kChunkPadRows;
+  const int b = blockIdx.x / per_b, e = blockIdx.x - b * per_b;
+  const int head = threadIdx.x >> 4, c = (threadIdx.x & 15) * 8;
+  const int64_t p0 = a.pos0[b];
+  const size_t cache_row = (size_t)b * a.stride_seq + (size_t)head * a.stride_head;
+  if (a.kind == BEAM_LOCAL) {
+    const int64_t j = p0 - a.prefix + e;
+    uint4 kv = make_uint4(0u, 0u, 0u, 0u), vv = kv;
+    if (p0 >= 0 && j >= 0) {
+      const size_t off = cache_row + (size_t)(j % a.window) * kD + c;
+      kv = *reinterpret_cast<const uint4 *>(a.k_cache + off);
+      vv = *reinterpret_cast<const uint4 *>(a.v_cache + off);
+    }
+    const size_t dst = ((size_t)b * a.ext_rows + e) * (kHkv * kD) + head * kD + c;
+    *reinterpret_cast<uint4 *>(a.k_ext + dst) = kv;
+    *reinterpret_cast<uint4 *>(a.v_ext + dst) = vv;
+  } else {
+    const int64_t end = p0 + a.T, slot = end + e;
+    if (p0 < 0 || end > a.slots || slot >= a.slots || slot >= (end + 127) / 128 * 128) return;
+    *reinterpret_cast<uint4 *>(a.v_cache + cache_row + (size_t)slot * kD + c) =
+        make_uint4(0u, 0u, 0u, 0u);
   }
 }
 

@@ -164,5 +164,26 @@ def test_host_validation_rejects_before_launch(beam):
 
     assert L.beam_kv_append(1, P, 1, 4, A, A, A, None, A, A, ctypes.byref(glob), None, None) == -1
     assert L.beam_kv_append(1, P, 1, 0, A, A, A, A, A, A, ctypes.byref(glob), None, None) == 0
+    # chunked prefill: the cache is required, pos0 is a device int64 array
+    ring = beam.beam_kv_layout(beam.LOCAL, p, 1, 0)
+    cws = beam.beam_prefill_chunk_workspace_bytes(beam.LOCAL, p, 1, 16)
+    assert cws == 2 * (511 + 16) * 8 * 128 * 2 + 16 * 128 * 4   # earlier + new K/V rows, RoPE table
+    assert beam.beam_prefill_chunk_workspace_bytes(beam.GLOBAL, p, 1, 16) == 0
+    cargs = lambda **kw: [kw.get("kind", 0), P, kw.get("B", 1), kw.get("T", 16), A, A, A, A, A, A,
+                          A, kw.get("pos0", A), A, kw.get("kc", A), A,
+                          kw.get("layout", ctypes.byref(ring)), kw.get("ws", A),
+                          kw.get("ws_bytes", cws), None, None]
+    assert L.beam_attn_prefill_chunk(*cargs(T=0)) == 0
+    assert L.beam_attn_prefill_chunk(*cargs(pos0=None)) == -1
+    assert L.beam_attn_prefill_chunk(*cargs(pos0=A + 4)) == -7
+    assert L.beam_attn_prefill_chunk(*cargs(kc=None)) == -1
+    assert L.beam_attn_prefill_chunk(*cargs(layout=None)) == -1
+    assert L.beam_attn_prefill_chunk(*cargs(ws_bytes=cws - 1)) == -6
+    assert L.beam_attn_prefill_chunk(*cargs(ws=None)) == -6
+    small = beam.beam_kv_layout(beam.GLOBAL, p, 1, 15)
+    assert L.beam_attn_prefill_chunk(*cargs(kind=1, layout=ctypes.byref(small), ws=None,
+                                            ws_bytes=0)) == -5          # T = 16 > 15 slots
+    assert L.beam_attn_prefill_chunk(*cargs(kind=0, layout=ctypes.byref(small))) == -1
+
     for s in (0, -1, -2, -3, -4, -5, -6, -7, -8, 99):
         assert isinstance(beam.beam_status_string(s), str)
