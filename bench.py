@@ -4,9 +4,10 @@ One step = the prefill of one local and one global attention layer of the
 batched-prefill workload (4 sequences x 8192 tokens, 48 query / 8 KV heads,
 head_dim 128), including the fused KV-cache append, through the C ABI.  The
 headline value is algorithmic TFLOP/s (visible (query, key) pairs x 4 x 128 x 48).
-Two decode measurements ride along on the same line: the 1M-context decode step
-across the 52-layer schedule (KV-read GB/s, tokens/s) and the batched decode step
-(64 sequences, contexts in [1024, 32768]).
+Three more measurements ride along on the same line: the 1M-context decode step
+across the 52-layer schedule (KV-read GB/s, tokens/s), the batched decode step
+(64 sequences, contexts in [1024, 32768]) and the chunked prefill (8192 new tokens
+after 57,344 cached ones, one local and one global layer; TFLOP/s).
 
 Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl beam|reference]
 N > 1 runs under torch.distributed.run, one process per GPU; every rank processes
@@ -340,6 +341,57 @@ def bench_decode_batched(torch, beam, steps, warmup, seed):
     return res
 
 
+def bench_prefill_chunk(torch, beam, steps, warmup, seed):
+    """The chunked-prefill workload: one local and one global layer call of 8192 new
+    tokens after 57,344 cached ones (cache contents drawn on the device)."""
+    w = wl.workload("chunked_prefill", seed)
+    p0 = w.extra["pos0"]
+    params = beam.default_params()
+    dev = "cuda"
+    x = {}
+    for name, width in (("q", 6144), ("k", 1024), ("v", 1024), ("gate", 6144)):
+        t = torch.empty((w.B, w.T, width), dtype=torch.bfloat16, device=dev)
+        wl.device_normal_bf16_(t, seed, f"chunk/{name}")
+        x[name] = t
+    inp = wl.prefill_inputs(1, 1, seed, layer="chunk")
+    qw = torch.from_numpy(inp.q_norm_w).to(dev)
+    kw = torch.from_numpy(inp.k_norm_w).to(dev)
+    bias = torch.from_numpy(inp.gate_bias).to(dev)
+    out = torch.empty_like(x["q"])
+    pos0 = torch.full((w.B,), p0, dtype=torch.int64, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    calls, res = [], {"workload": f"chunked_prefill: B={w.B}, T={w.T} new tokens after {p0} "
+                                  "cached (global cache 65536 slots; local 512-slot ring)"}
+    for kind in (wl.LOCAL, wl.GLOBAL):
+        slots = w.extra["global_slots"] if kind == wl.GLOBAL else wl.WINDOW
+        layout = beam.beam_kv_layout(kind, params, w.B, slots)
+        kc = torch.empty(layout.bytes_k // 2, dtype=torch.bfloat16, device=dev)
+        vc = torch.empty_like(kc)
+        wl.device_normal_bf16_(kc, seed, f"chunk/kc{kind}")
+        wl.device_normal_bf16_(vc, seed, f"chunk/vc{kind}")
+        ws = torch.empty(max(16, beam.beam_prefill_chunk_workspace_bytes(kind, params, w.B, w.T)),
+                         dtype=torch.uint8, device=dev)
+
+        def call(kind=kind, layout=layout, kc=kc, vc=vc, ws=ws):
+            # the same position every step: the call appends the same rows again
+            beam.beam_attn_prefill_chunk(kind, params, x["q"], x["k"], x["v"], x["gate"], qw, kw,
+                                         bias, pos0, out, kc, vc, layout, workspace=ws,
+                                         dev_status=status)
+        sec = time_loop(torch, call, steps, warmup)
+        flops = w.B * wl.chunk_visible_pairs(w.T, p0, wl.WINDOW if kind == wl.LOCAL else None) \
+            * HEAD_FLOPS_PER_PAIR
+        name = "local" if kind == wl.LOCAL else "global"
+        res[f"{name}_ms"] = sec * 1e3
+        res[f"{name}_tflops"] = flops / sec / 1e12
+        calls.append((sec, flops))
+    assert int(status.item()) == 0, "device status set during the chunked-prefill bench"
+    res["tflops"] = sum(f for _, f in calls) / sum(s for s, _ in calls) / 1e12
+    res["gpu_launches_per_step"] = 6   # per layer: ring copy or value padding, prologue, attention
+    del x, out
+    torch.cuda.empty_cache()
+    return res
+
+
 _CPU_INPUTS = {}
 
 
@@ -513,6 +565,9 @@ def run_gpu(args):
         db = bench_decode_batched(torch, beam, args.steps, args.warmup, args.seed)
         db["pct_of_hbm"] = round(100 * db["kv_read_GBps"] / pk["hbm_gbs"], 2)
         result["decode_batched"] = db
+        pc = bench_prefill_chunk(torch, beam, args.steps, args.warmup, args.seed)
+        pc["pct_of_bf16_peak"] = round(100 * pc["tflops"] / pk["bf16_tflops"], 2)
+        result["prefill_chunk"] = pc
     if rank == 0 and world == 1 and not args.no_cpu:
         result["cpu_baseline"] = cpu_baseline_prefill(seed=args.seed)
     if rank == 0:

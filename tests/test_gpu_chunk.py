@@ -118,6 +118,26 @@ def test_long_global_history_sampled_rows(env):
 
 
 @pytest.mark.parametrize("kind", [wl.GLOBAL, wl.LOCAL])
+def test_chunked_prefill_workload_sampled_rows(env, kind):
+    """The chunked-prefill workload at full size, in the call the bench times: 8192
+    new tokens after 57,344 cached ones; sampled rows against the oracle."""
+    torch, beam, orc = env
+    params = beam.default_params()
+    w = wl.workload("chunked_prefill")
+    slots = w.extra["global_slots"] if kind == wl.GLOBAL else wl.WINDOW
+    ci = wl.chunk_inputs(kind, w.T, [w.extra["pos0"]] * w.B, slots, w.seed, layer=f"full{kind}")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, *_ = run_chunk(torch, beam, ci, params, status)
+    assert int(status.item()) == 0
+    rng = wl.rng(w.seed, f"rows{kind}")
+    ri = np.unique(np.concatenate([[0, 127, 128, 4095, w.T - 1], rng.integers(0, w.T, 7)]))
+    rb = np.zeros_like(ri)
+    ref = oracle_chunk(orc, beam, ci, params, (rb, ri))
+    got = host_bits(out).reshape(w.B, w.T, 48, 128)[0, ri]
+    assert_close(got, ref, f"chunked_prefill kind={kind}")
+
+
+@pytest.mark.parametrize("kind", [wl.GLOBAL, wl.LOCAL])
 def test_prefill_then_chunk_equals_one_shot(env, kind):
     """The GPU's own prefill fills the cache with the first T1 tokens, then one chunk
     adds T2 more: the chunk rows equal the oracle's one-shot prefill rows T1 ..

@@ -243,11 +243,22 @@ def workload(name: str, seed: int = 1234) -> Workload:
                         seed=seed, extra={"global_slots": 32768})
     if name == "long_global_prefill":
         return Workload(name, "prefill", B=1, T=131072, layers=(GLOBAL,), seed=seed)
+    if name == "chunked_prefill":
+        # the last 8192-token chunk of a 65,536-token prompt: 57,344 tokens already cached
+        return Workload(name, "prefill", B=1, T=8192, layers=(LOCAL, GLOBAL), seed=seed,
+                        extra={"pos0": 57344, "global_slots": 65536})
     if name == "decode_1m":
         kinds = tuple(layer_kind(i) for i in range(1, N_LAYERS + 1))
         return Workload(name, "decode", B=1, layers=kinds, ctx=(MAX_CONTEXT,), seed=seed,
                         extra={"global_slots": MAX_CONTEXT})
     raise KeyError(name)
+
+
+def chunk_visible_pairs(T: int, pos0: int, window: int | None) -> int:
+    """(query, key) pairs the mask admits for queries pos0 .. pos0+T-1 over keys 0 ..."""
+    if window is None:
+        return T * pos0 + T * (T + 1) // 2
+    return sum(min(window, pos0 + i + 1) for i in range(T))
 
 
 def visible_pairs(T: int, window: int | None) -> int:
