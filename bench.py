@@ -247,8 +247,8 @@ class DecodeLayer:
                               dtype=torch.uint8, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         self.bytes = decode_kv_bytes(ctx, kind)
-        # a ring layer is one launch; a global layer is prologue + split-K + combine
-        self.launches_per_call = 1 if kind == wl.LOCAL else 3
+        # a ring layer is one launch; a global layer is split-K + combine
+        self.launches_per_call = 1 if kind == wl.LOCAL else 2
 
     def run(self):
         self.beam.beam_attn_decode(self.kind, self.params, self.q, self.k, self.v, self.gate,

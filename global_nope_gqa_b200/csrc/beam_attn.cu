@@ -203,7 +203,6 @@ int decode_split(int kind, const beam_attn_params *p, int32_t B, int64_t slots, 
 }
 
 struct DecodeWorkspace {
-  uint16_t *qn;
   float *part_o;
   float *part_ml;
   size_t bytes;
@@ -213,8 +212,6 @@ DecodeWorkspace decode_workspace(void *base, int32_t B, int n_split_max) {
   DecodeWorkspace w;
   uint8_t *p = static_cast<uint8_t *>(base);
   size_t off = 0;
-  w.qn = reinterpret_cast<uint16_t *>(p + off);
-  off += round_up((size_t)B * kHq * kD * 2, 256);
   w.part_o = reinterpret_cast<float *>(p + off);
   off += round_up((size_t)B * kHkv * n_split_max * kGroup * kD * 4, 256);
   w.part_ml = reinterpret_cast<float *>(p + off);
@@ -546,7 +543,6 @@ int beam_attn_decode(int kind, const beam_attn_params *p, int32_t B, const void 
 
   DecodeArgs da;
   memset(&da, 0, sizeof da);
-  da.qn = w.qn;
   da.k_cache = static_cast<uint16_t *>(k_cache);
   da.v_cache = static_cast<uint16_t *>(v_cache);
   da.stride_seq = layout->stride_seq;
@@ -563,21 +559,23 @@ int beam_attn_decode(int kind, const beam_attn_params *p, int32_t B, const void 
   da.part_o = w.part_o;
   da.part_ml = w.part_ml;
   dim3 grid(n_split_max, kHkv, B);
+  // every CTA normalises (local: rotates) its group's queries; the owner of the new
+  // token's slot also appends its key and value
+  da.q_raw = static_cast<const uint16_t *>(q);
+  da.k_raw = static_cast<const uint16_t *>(k);
+  da.v_raw = static_cast<const uint16_t *>(v);
+  da.gate = static_cast<const uint16_t *>(gate);
+  da.qw = q_norm_w;
+  da.kw = k_norm_w;
+  da.gate_bias = gate_bias;
+  da.out = static_cast<uint16_t *>(out);
+  da.status = dev_status;
+  da.eps = p->rms_eps;
+  fill_inv_freq(da.inv_freq, p->rope_theta);
 
   if (kind == BEAM_LOCAL) {
-    // one launch: the ring's splits form a cluster that normalises, appends, attends,
-    // merges through distributed shared memory and gates
-    da.q_raw = static_cast<const uint16_t *>(q);
-    da.k_raw = static_cast<const uint16_t *>(k);
-    da.v_raw = static_cast<const uint16_t *>(v);
-    da.gate = static_cast<const uint16_t *>(gate);
-    da.qw = q_norm_w;
-    da.kw = k_norm_w;
-    da.gate_bias = gate_bias;
-    da.out = static_cast<uint16_t *>(out);
-    da.status = dev_status;
-    da.eps = p->rms_eps;
-    fill_inv_freq(da.inv_freq, p->rope_theta);
+    // one launch: the ring's splits form a cluster that also merges through distributed
+    // shared memory and gates
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof cfg);
     cfg.gridDim = grid;
@@ -594,29 +592,6 @@ int beam_attn_decode(int kind, const beam_attn_params *p, int32_t B, const void 
     return cuda_status(cudaLaunchKernelEx(&cfg, decode_attn_kernel<true>, da), "ring decode launch");
   }
 
-  PrologueArgs pa;
-  memset(&pa, 0, sizeof pa);
-  pa.q = static_cast<const uint16_t *>(q);
-  pa.k = static_cast<const uint16_t *>(k);
-  pa.v = static_cast<const uint16_t *>(v);
-  pa.qw = q_norm_w;
-  pa.kw = k_norm_w;
-  pa.q_out = w.qn;
-  pa.k_out = nullptr;
-  pa.k_cache = static_cast<uint16_t *>(k_cache);
-  pa.v_cache = static_cast<uint16_t *>(v_cache);
-  pa.stride_seq = layout->stride_seq;
-  pa.stride_head = layout->stride_head;
-  pa.slots = layout->slots_per_seq;
-  pa.pos0 = pos;
-  pa.status = dev_status;
-  pa.T = 1;
-  pa.kind = kind;
-  pa.window = p->window;
-  pa.eps = p->rms_eps;
-  fill_inv_freq(pa.inv_freq, p->rope_theta);
-  prologue_kernel<<<(unsigned)B, 128, 0, s>>>(pa);
-  if ((st = launch_status())) return st;
   decode_attn_kernel<false><<<grid, kDecThreads, kDecSmem, s>>>(da);
   if ((st = launch_status())) return st;
 

@@ -7,7 +7,10 @@
 // and the time goes into streaming the global caches, 4 KiB per token per
 // layer (section "KV memory").
 //
-// decode_attn_kernel: grid (split, KV head, sequence), 128 threads.  A CTA
+// decode_attn_kernel: grid (split, KV head, sequence), 128 threads.  Every CTA first
+// normalises (and, in a local layer, rotates) the six queries of its group itself; the
+// CTA whose run holds the new token's slot also prepares and writes the new key and value
+// there.  A CTA then
 // streams a contiguous run of `split` cache slots of one (sequence, KV head) --
 // keys and values are contiguous in the head-major cache -- through a 3-stage
 // cp.async ring of 64-slot tiles (16-byte coalesced loads, XOR-swizzled rows).
@@ -15,9 +18,10 @@
 // (rows 6..15 are zero): S = Q K^T and O += P V.  The MMAs exist to take the
 // 6 x 128 x 2 multiply-adds per cached row off the FP32 pipe, which would
 // otherwise bound the kernel below HBM speed.  Each warp keeps its own online
-// softmax over a quarter of every tile; the four warps merge in shared memory and
-// the CTA writes one partial (m, l, o[128]) per head.
-//
+// softmax over a quarter of every tile; the four warps merge in shared memory.  Then
+// either the CTAs of a local ring (one thread-block cluster) merge through distributed
+// shared memory and gate the output, or each CTA writes one partial (m, l, o[128]) per
+// head and
 // decode_combine_kernel: one CTA per (sequence, query head) merges the partials
 // with the log-sum-exp rule and applies Y = O/l * sigmoid(G + b_h).
 #pragma once
@@ -36,7 +40,6 @@ constexpr int kDecTileBytes = kDecTile * kD * 2;                   // 16 KiB
 constexpr int kDecSmem = kDecStages * 2 * kDecTileBytes;
 
 struct DecodeArgs {
-  const uint16_t *qn;       // [B][48][128] prepared queries (split-K path)
   uint16_t *k_cache;
   uint16_t *v_cache;
   int64_t stride_seq, stride_head, slots;
@@ -46,12 +49,11 @@ struct DecodeArgs {
   int n_split_max;          // partial slots reserved per (sequence, KV head)
   float scale_log2;         // softmax_scale * log2(e)
   float ssmax_base, ssmax_exp;
-  float *part_o;            // [B][8][n_split_max][6][128]
-  float *part_ml;           // [B][8][n_split_max][6][2]  (running max in log2 units, sum)
-  // single-kernel path (one split covers every visible slot): raw inputs and the output
+  float *part_o;            // global: [B][8][n_split_max][6][128]
+  float *part_ml;           // global: [B][8][n_split_max][6][2]  (max in log2 units, sum)
   const uint16_t *q_raw, *k_raw, *v_raw, *gate;  // [B][48*128], [B][8*128] x 2, [B][48*128]
   const float *qw, *kw, *gate_bias;
-  uint16_t *out;            // [B][48*128]
+  uint16_t *out;            // local: [B][48*128] (a global layer's combine writes it)
   int32_t *status;
   float eps;
   double inv_freq[64];
@@ -64,26 +66,24 @@ __device__ __forceinline__ int64_t decode_visible(const DecodeArgs &a, int64_t t
   return t < a.slots ? t + 1 : 0;
 }
 
-// kFused = false: one split of the keys, partials to the workspace (combined afterwards).
-// kFused = true: the whole step of a local layer in one launch.  The splits of a
-// (sequence, KV head) form one thread-block cluster (gridDim.x CTAs, at most 4 of 128+
-// ring slots each); every CTA normalises and rotates the six queries of its group, the CTA
-// whose slots hold position t also writes the new key and value there, each CTA attends
-// over its slots, and rank 0 merges the CTAs' partials through distributed shared memory
-// and writes Y = O/l * sigmoid(G + b).
-template <bool kFused>
+// kCluster = false (global cache): one split of the keys, partials to the workspace,
+// merged by decode_combine_kernel.  kCluster = true (local ring): the whole step in one
+// launch -- the splits of a (sequence, KV head) form one thread-block cluster (gridDim.x
+// CTAs, at most 4 of 128+ ring slots each), and rank 0 merges the CTAs' partials through
+// distributed shared memory and writes Y = O/l * sigmoid(G + b).
+template <bool kCluster>
 __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const DecodeArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  __shared__ __align__(16) uint16_t q_prep[kFused ? kGroup * kD : 8];
+  __shared__ __align__(16) uint16_t q_prep[kGroup * kD];
   const int s_idx = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int64_t t = a.pos[b];
-  if (kFused && t < 0) {
-    if (threadIdx.x == 0) set_status(a.status, BEAM_ERR_CAPACITY);
+  const int64_t n_vis = decode_visible(a, t);
+  if (n_vis == 0) {   // a position outside the cache: nothing is written (a whole cluster
+    if (threadIdx.x == 0 && s_idx == 0) set_status(a.status, BEAM_ERR_CAPACITY);  // leaves)
     return;
   }
-  const int64_t n_vis = decode_visible(a, t);
   const int64_t key_lo = (int64_t)s_idx * a.split;
-  if (!kFused && key_lo >= n_vis) return;   // a fused CTA stays: its cluster merges below
+  if (!kCluster && key_lo >= n_vis) return;   // a cluster CTA stays: its cluster merges below
   const int64_t key_hi = min(n_vis, key_lo + a.split);
   const int n_keys = key_hi > key_lo ? (int)(key_hi - key_lo) : 0;
   const int n_tiles = (n_keys + kDecTile - 1) / kDecTile;
@@ -116,11 +116,11 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const DecodeAr
     cp_async_commit();
   }
 
-  int patch_tile = -1, patch_row = 0;  // fused: prefetched tile and row of the new slot
+  int patch_tile = -1, patch_row = 0;  // prefetched tile and row of the new slot
   uint4 patch_val = make_uint4(0u, 0u, 0u, 0u);
-  float gate6[kGroup];                 // fused, rank 0: gate logits + bias of its outputs
-  if (kFused) {
-    if (s_idx == 0) {
+  float gate6[kGroup];                 // cluster rank 0: gate logits + bias of its outputs
+  {
+    if (kCluster && s_idx == 0) {
 #pragma unroll
       for (int i = 0; i < kGroup; ++i) {
         const int h = g * kGroup + i;
@@ -166,8 +166,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const DecodeAr
   uint32_t qa[8][2];
   {
     const int h = lane >> 2;
-    const uint16_t *qrow = kFused ? q_prep + (h < kGroup ? h : 0) * kD
-                                  : a.qn + ((size_t)b * kHq + g * kGroup + (h < kGroup ? h : 0)) * kD;
+    const uint16_t *qrow = q_prep + (h < kGroup ? h : 0) * kD;
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
       const int d0 = ks * 16 + (lane & 3) * 2;
@@ -184,11 +183,11 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const DecodeAr
 #pragma unroll
   for (int nb = 0; nb < 16; ++nb) o[nb][0] = o[nb][1] = o[nb][2] = o[nb][3] = 0.f;
 
-  const bool any_patch = kFused && __syncthreads_or(patch_tile >= 0);
+  const bool any_patch = __syncthreads_or(patch_tile >= 0);
   for (int tile = 0; tile < n_tiles; ++tile) {
     cp_async_wait<kDecStages - 2>();
     __syncthreads();
-    if (kFused && any_patch && tile < kDecStages - 1) {
+    if (any_patch && tile < kDecStages - 1) {
       // the new key / value row, written after this tile was requested
       if (patch_tile == tile) {
         uint8_t *ks = smem + (tile % kDecStages) * 2 * kDecTileBytes;
@@ -303,7 +302,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const DecodeAr
       acc += sc * sm_o[(w * kGroup + hh) * kD + d];
       L += sc * sm_l[w * kGroup + hh];
     }
-    if (kFused) {
+    if (kCluster) {
       float *cl = reinterpret_cast<float *>(smem + 16384);  // this CTA's partial
       cl[idx] = acc;
       if (d == 0) {
@@ -318,7 +317,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const DecodeAr
       }
     }
   }
-  if (kFused) {
+  if (kCluster) {
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
     cluster.sync();

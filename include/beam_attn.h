@@ -181,8 +181,8 @@ BEAM_API int beam_kv_append(int kind, const beam_attn_params *p, int32_t B, int3
                    void *v_cache, const beam_kv_layout_t *layout, int32_t *dev_status,
                    beam_stream_t stream);
 
-/* Workspace of one decode call (bytes): the prepared queries and the split-K
- * partial results, sized from the layout's slots per sequence. */
+/* Workspace of one decode call (bytes): the split-K partial results, sized from
+ * the layout's slots per sequence. */
 BEAM_API size_t beam_decode_workspace_bytes(int kind, const beam_attn_params *p, int32_t B,
                                    const beam_kv_layout_t *layout);
 
@@ -212,7 +212,7 @@ BEAM_API int beam_attn_decode(int kind, const beam_attn_params *p, int32_t B, co
  * pre-partitions all device memory into its own pools, or a latency-critical
  * loop in which an allocation (and the device synchronisation that cudaMalloc
  * and cudaFree can imply) is not acceptable -- yet beam_attn_decode needs a
- * workspace for the prepared queries and the split-K partial results.
+ * workspace for the split-K partial results.
  *
  * This entry point computes exactly what beam_attn_decode computes, with the
  * same arguments minus the workspace.  Its scratch is a fixed array of
