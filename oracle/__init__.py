@@ -97,6 +97,19 @@ def lib():
             ctypes.c_int, pp, ctypes.c_int, ctypes.c_int, u16p, u16p, u16p, u16p, fp, fp, fp,
             ctypes.POINTER(ctypes.c_int64), u16p, u16p, ctypes.c_int64, ctypes.c_int64,
             ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64), dp, ctypes.c_int]
+        u8p = ctypes.POINTER(ctypes.c_uint8)
+        L.oracle_e4m3_decode.restype = ctypes.c_double
+        L.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+        L.oracle_e4m3_encode.restype = ctypes.c_uint8
+        L.oracle_e4m3_encode.argtypes = [ctypes.c_double]
+        L.oracle_decode_fp8.restype = ctypes.c_int
+        L.oracle_decode_fp8.argtypes = [
+            ctypes.c_int, pp, ctypes.c_int, u16p, u16p, u16p, u16p, fp, fp, fp,
+            ctypes.POINTER(ctypes.c_int64), u8p, u8p, ctypes.c_int64, ctypes.c_double,
+            ctypes.c_double, dp, ctypes.c_int]
+        L.oracle_kv_row_fp8.restype = None
+        L.oracle_kv_row_fp8.argtypes = [ctypes.c_int, pp, u16p, u16p, fp, ctypes.c_int64,
+                                        ctypes.c_double, ctypes.c_double, u8p, u8p]
         L.oracle_kv_row.restype = None
         L.oracle_kv_row.argtypes = [ctypes.c_int, pp, u16p, u16p, fp, ctypes.c_int64, u16p, u16p]
         _lib = L
@@ -275,6 +288,50 @@ def prefill_chunk(kind, P: Params, q, k, v, gate, q_norm_w, k_norm_w, gate_bias,
     out = prefill_chunk_rows(kind, P, q, k, v, gate, q_norm_w, k_norm_w, gate_bias, pos0,
                              k_cache, v_cache, bb.ravel(), ii.ravel(), n_threads)
     return out.reshape(B, T, P.n_q_heads, P.head_dim)
+
+
+def e4m3_decode(code: int) -> float:
+    return lib().oracle_e4m3_decode(int(code))
+
+
+def e4m3_encode(x: float) -> int:
+    return int(lib().oracle_e4m3_encode(float(x)))
+
+
+def decode_fp8(kind, P: Params, q, k, v, gate, q_norm_w, k_norm_w, gate_bias, pos, k_codes,
+               v_codes, k_scale: float, v_scale: float, n_threads: int | None = None) -> np.ndarray:
+    """One decode step over FP8 E4M3 caches ([B, Hkv, slots, d] uint8 codes, one scale per
+    cache tensor): [B, Hq, d] float64."""
+    q, k, v, gate = _u16(q), _u16(k), _u16(v), _u16(gate)
+    k_codes = np.ascontiguousarray(k_codes, dtype=np.uint8)
+    v_codes = np.ascontiguousarray(v_codes, dtype=np.uint8)
+    B = q.shape[0]
+    slots = k_codes.shape[2]
+    pos = np.ascontiguousarray(pos, dtype=np.int64)
+    qw, kw, bias = _f32(q_norm_w), _f32(k_norm_w), _f32(gate_bias)
+    out = np.empty((B, P.n_q_heads, P.head_dim), dtype=np.float64)
+    u8 = ctypes.c_uint8
+    rc = lib().oracle_decode_fp8(
+        kind, ctypes.byref(P), B, _ptr(q, ctypes.c_uint16), _ptr(k, ctypes.c_uint16),
+        _ptr(v, ctypes.c_uint16), _ptr(gate, ctypes.c_uint16), _ptr(qw, ctypes.c_float),
+        _ptr(kw, ctypes.c_float), _ptr(bias, ctypes.c_float), _ptr(pos, ctypes.c_int64),
+        _ptr(k_codes, u8), _ptr(v_codes, u8), slots, float(k_scale), float(v_scale),
+        _ptr(out, ctypes.c_double), n_threads or n_threads_default())
+    if rc != 0:
+        raise ValueError("oracle_decode_fp8 rejected its arguments")
+    return out
+
+
+def kv_row_fp8(kind, P: Params, k_token, v_token, k_norm_w, j, k_scale: float, v_scale: float):
+    """Expected FP8 cache codes for one token at position j: (k_codes, v_codes), [Hkv, d]."""
+    k_token, v_token, kw = _u16(k_token), _u16(v_token), _f32(k_norm_w)
+    kr = np.empty((P.n_kv_heads, P.head_dim), dtype=np.uint8)
+    vr = np.empty_like(kr)
+    u8 = ctypes.c_uint8
+    lib().oracle_kv_row_fp8(kind, ctypes.byref(P), _ptr(k_token, ctypes.c_uint16),
+                            _ptr(v_token, ctypes.c_uint16), _ptr(kw, ctypes.c_float), int(j),
+                            float(k_scale), float(v_scale), _ptr(kr, u8), _ptr(vr, u8))
+    return kr, vr
 
 
 def kv_row(kind, P: Params, k_token, v_token, k_norm_w, j):

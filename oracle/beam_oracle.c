@@ -532,6 +532,146 @@ int oracle_prefill_chunk_rows(int kind, const oracle_params *P, int B, int T,
   return 0;
 }
 
+/* ------------------------------------------------------------ FP8 cache */
+
+/* FP8 E4M3 as the KV-cache element (section "KV memory": 18 KiB per token
+ * over the nine global layers instead of 36 KiB in BF16).  The page names the
+ * format only; its definition here is the OCP 8-bit floating-point E4M3 one
+ * without infinities: sign bit, 4 exponent bits with bias 7, 3 mantissa bits;
+ * exponent 0 holds the subnormals m * 2^-9; S.1111.111 is NaN, so the largest
+ * finite magnitude is 1.75 * 2^8 = 448.  A cache element stores
+ * code = E4M3(x / scale) with one float scale per cache tensor of a layer, and
+ * reads back as E4M3^-1(code) * scale. */
+double oracle_e4m3_decode(uint8_t code) {
+  int s = code >> 7, e = (code >> 3) & 15, m = code & 7;
+  if (e == 15 && m == 7) return NAN;
+  double mag = e == 0 ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, e - 7);
+  return s ? -mag : mag;
+}
+
+/* Nearest code, ties to the even mantissa; magnitudes past 448 saturate to
+ * +-448 (the conversion the cache write uses), NaN stays NaN. */
+uint8_t oracle_e4m3_encode(double x) {
+  if (isnan(x)) return 0x7F;
+  uint8_t s = signbit(x) ? 0x80 : 0x00;
+  double a = fabs(x);
+  if (a >= 448.0) return s | 0x7E;
+  int e2;
+  frexp(a, &e2);          /* a = f * 2^e2, f in [0.5, 1) */
+  int e = e2 - 1;         /* a in [2^e, 2^(e+1)) */
+  if (a == 0.0 || e < -6) {
+    double m = nearbyint(ldexp(a, 9));   /* subnormal steps of 2^-9; 8 -> smallest normal */
+    return s | (uint8_t)m;
+  }
+  double m = nearbyint((ldexp(a, -e) - 1.0) * 8.0);   /* 0 .. 8 */
+  if (m == 8.0) { m = 0.0; ++e; }
+  if (e > 8 || (e == 8 && m > 6.0)) return s | 0x7E;
+  return s | (uint8_t)(((e + 7) << 3) | (int)m);
+}
+
+/* One decode step over FP8 caches: as oracle_decode, but every cached row is
+ * E4M3^-1(code) * scale, and the new token's key and value are first written
+ * as codes (append first, then attend), so the query sees them read back from
+ * the cache too.  Caches are head-major [B][Hkv][slots][d] codes. */
+typedef struct {
+  decode_ctx base;
+  const uint8_t *k_codes, *v_codes;
+  double k_scale, v_scale;
+} decode8_ctx;
+
+typedef struct {
+  const decode8_ctx *c;
+  int64_t b, g, lo, t;
+  const double *k_new, *v_new;
+} decode8_view;
+
+static void decode8_row(const void *vctx, int64_t idx, double *k_row, double *v_row) {
+  const decode8_view *r = (const decode8_view *)vctx;
+  const decode8_ctx *c = r->c;
+  int d = c->base.P->head_dim;
+  int64_t j = r->lo + idx;
+  if (j == r->t) {
+    memcpy(k_row, r->k_new, sizeof(double) * d);
+    memcpy(v_row, r->v_new, sizeof(double) * d);
+    return;
+  }
+  int64_t s = oracle_cache_slot(c->base.kind, j, c->base.slots);
+  size_t off = (((size_t)r->b * c->base.P->n_kv_heads + r->g) * c->base.slots + s) * d;
+  for (int i = 0; i < d; ++i) {
+    k_row[i] = oracle_e4m3_decode(c->k_codes[off + i]) * c->k_scale;
+    v_row[i] = oracle_e4m3_decode(c->v_codes[off + i]) * c->v_scale;
+  }
+}
+
+static void decode8_job(void *vctx, int64_t item) {
+  decode8_ctx *c8 = (decode8_ctx *)vctx;
+  const decode_ctx *c = &c8->base;
+  const oracle_params *P = c->P;
+  int d = P->head_dim, Hq = P->n_q_heads, Hkv = P->n_kv_heads, G = Hq / Hkv;
+  int64_t b = item / Hq;
+  int h = (int)(item % Hq), g = h / G;
+  int64_t t = c->pos[b];
+  int64_t lo = 0;
+  while (!oracle_visible(c->kind, t, lo, P->window)) ++lo;
+  int64_t n = t - lo + 1;
+  double *scores = (double *)malloc(sizeof(double) * n);
+  double *q = (double *)malloc(sizeof(double) * d);
+  double *kv_new = (double *)malloc(sizeof(double) * 2 * d);
+  size_t kv_off = ((size_t)b * Hkv + g) * d;
+  prepare_key(c->kind, P, c->k + kv_off, c->kw, t, kv_new);
+  for (int i = 0; i < d; ++i) {
+    kv_new[i] = oracle_e4m3_decode(oracle_e4m3_encode(kv_new[i] / c8->k_scale)) * c8->k_scale;
+    double v = oracle_bf16_to_double(c->v[kv_off + i]);
+    kv_new[d + i] = oracle_e4m3_decode(oracle_e4m3_encode(v / c8->v_scale)) * c8->v_scale;
+  }
+  decode8_view view = {c8, b, g, lo, t, kv_new, kv_new + d};
+  size_t q_off = ((size_t)b * Hq + h) * d;
+  prepare_query(c->kind, P, c->q + q_off, c->qw, t, q);
+  attend_one(P, q, n, decode8_row, &view, c->gate + q_off, (double)c->bias[h], scores,
+             c->out + q_off);
+  free(scores); free(q); free(kv_new);
+}
+
+int oracle_decode_fp8(int kind, const oracle_params *P, int B, const uint16_t *q,
+                      const uint16_t *k, const uint16_t *v, const uint16_t *gate,
+                      const float *q_norm_w, const float *k_norm_w, const float *gate_bias,
+                      const int64_t *pos, const uint8_t *k_codes, const uint8_t *v_codes,
+                      int64_t slots, double k_scale, double v_scale, double *out, int n_threads) {
+  if (!P || P->n_kv_heads <= 0 || P->n_q_heads % P->n_kv_heads) return -1;
+  if (!(k_scale > 0.0) || !(v_scale > 0.0)) return -1;
+  for (int b = 0; b < B; ++b) {
+    if (pos[b] < 0) return -1;
+    if (kind == ORACLE_GLOBAL && pos[b] >= slots) return -1;
+    if (kind == ORACLE_LOCAL && slots < P->window) return -1;
+  }
+  int d = P->head_dim;
+  double *qw = (double *)malloc(sizeof(double) * d), *kw = (double *)malloc(sizeof(double) * d);
+  for (int i = 0; i < d; ++i) { qw[i] = q_norm_w[i]; kw[i] = k_norm_w[i]; }
+  decode8_ctx c = {{kind, P, B, q, k, v, gate, qw, kw, gate_bias, pos, NULL, NULL, slots, out},
+                   k_codes, v_codes, k_scale, v_scale};
+  run_parallel(decode8_job, &c, (int64_t)B * P->n_q_heads, n_threads);
+  free(qw); free(kw);
+  return 0;
+}
+
+/* Expected FP8 cache rows for one token at position j: codes of the exact
+ * prepared key and of the raw value, each divided by its scale. */
+void oracle_kv_row_fp8(int kind, const oracle_params *P, const uint16_t *k_raw_token,
+                       const uint16_t *v_raw_token, const float *k_norm_w, int64_t j,
+                       double k_scale, double v_scale, uint8_t *k_row, uint8_t *v_row) {
+  int d = P->head_dim;
+  double *tmp = (double *)malloc(sizeof(double) * d);
+  for (int g = 0; g < P->n_kv_heads; ++g) {
+    oracle_prepare_key(kind, P, k_raw_token + (size_t)g * d, k_norm_w, j, tmp);
+    for (int i = 0; i < d; ++i) {
+      k_row[(size_t)g * d + i] = oracle_e4m3_encode(tmp[i] / k_scale);
+      v_row[(size_t)g * d + i] =
+          oracle_e4m3_encode(oracle_bf16_to_double(v_raw_token[(size_t)g * d + i]) / v_scale);
+    }
+  }
+  free(tmp);
+}
+
 /* Expected cache rows written for one token at position j: the prepared key
  * rounded to the nearest bf16 and the raw value bits, one row per KV head
  * ([Hkv][d] each).  Tests compare these with what the device wrote at slot

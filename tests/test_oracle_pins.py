@@ -415,6 +415,128 @@ def test_chunk_after_cache_fill_matches_prefill(orc, kind):
     assert np.max(np.abs(shifted - want)) > 0.05
 
 
+# ---------------------------------------------------------------- FP8 E4M3 cache
+def _torch_e4m3(codes):
+    import torch
+    t = torch.tensor(np.asarray(codes, np.uint8)).view(torch.float8_e4m3fn)
+    return t.to(torch.float64).numpy()
+
+
+def test_e4m3_decode_matches_library_and_format_facts(orc):
+    """All 256 codes against PyTorch's float8_e4m3fn, and the format's fixed points:
+    largest 448, smallest normal 2^-6, smallest subnormal 2^-9, 1.0 = 0x38, NaN only at
+    S.1111.111, strictly increasing over 0x00 .. 0x7E, sign symmetric."""
+    got = np.array([orc.e4m3_decode(c) for c in range(256)])
+    ref = _torch_e4m3(np.arange(256))
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan) and set(np.flatnonzero(nan)) == {0x7F, 0xFF}
+    np.testing.assert_array_equal(got[~nan], ref[~nan])
+    assert got[0x7E] == 448.0 and got[0x08] == 2.0 ** -6 and got[0x01] == 2.0 ** -9
+    assert got[0x38] == 1.0 and got[0xB8] == -1.0
+    assert np.all(np.diff(got[:0x7F]) > 0)
+    np.testing.assert_array_equal(got[0x80:0xFF], -got[0x00:0x7F])
+
+
+def test_e4m3_encode_rounds_to_nearest_even_and_saturates(orc):
+    vals = np.array([orc.e4m3_decode(c) for c in range(0x7F)])
+    for c in range(0x7F):
+        assert orc.e4m3_encode(vals[c]) == c
+        assert orc.e4m3_encode(-vals[c]) == (c | 0x80)
+    for c in range(0x7E):          # midpoints go to the even code, just off them to the nearer
+        mid = 0.5 * (vals[c] + vals[c + 1])
+        assert orc.e4m3_encode(mid) == (c if c % 2 == 0 else c + 1), hex(c)
+        assert orc.e4m3_encode(np.nextafter(mid, 0)) == c
+        assert orc.e4m3_encode(np.nextafter(mid, 1e9)) == c + 1
+    for x, code in ((448.0, 0x7E), (460.0, 0x7E), (1000.0, 0x7E), (-1e9, 0xFE), (1e-30, 0x00)):
+        assert orc.e4m3_encode(x) == code
+    # agrees with PyTorch's float -> float8_e4m3fn conversion inside the finite range
+    import torch
+    r = np.random.default_rng(5).standard_normal(4000) * np.exp(np.random.default_rng(6)
+                                                                 .uniform(-8, 5, 4000))
+    r = r[np.abs(r) < 440]
+    lib = torch.tensor(r).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    mine = np.array([orc.e4m3_encode(x) for x in r], np.uint8)
+    np.testing.assert_array_equal(mine, lib)
+
+
+def _fp8_problem(B, seed, d=16, Hq=6, Hkv=2):
+    q, gate = _rand((B, Hq * d), seed, "q"), _rand((B, Hq * d), seed, "g")
+    k, v = _rand((B, Hkv * d), seed, "k"), _rand((B, Hkv * d), seed, "v")
+    qw, kw = wl.norm_weight(seed, "qw")[:d], wl.norm_weight(seed, "kw")[:d]
+    bias = np.linspace(-0.5, 0.5, Hq).astype(np.float32)
+    return q, k, v, gate, qw, kw, bias
+
+
+def _grid_bf16(orc, codes, scale):
+    """bf16 bits of E4M3^-1(code) * scale (exact for a power-of-two scale)."""
+    vals = np.vectorize(orc.e4m3_decode)(codes) * scale
+    return _bf16(vals.astype(np.float32))
+
+
+@pytest.mark.parametrize("kind", [0, 1])
+def test_decode_fp8_equals_bf16_decode_of_the_dequantised_cache(orc, kind):
+    """With the new token's key zero (RMSNorm keeps it zero, an exact code) and its
+    value on the E4M3 grid, the FP8 decode is the BF16 decode of a cache holding the
+    dequantised codes: same slots, same scales (k_scale 2, v_scale 1/2)."""
+    d, Hq, Hkv, W = 16, 6, 2, 8
+    P = orc.params(n_q_heads=Hq, n_kv_heads=Hkv, head_dim=d, window=W)
+    pos = np.array([0, 3, 8, 29], np.int64)
+    B, slots = pos.size, (W if kind == orc.LOCAL else 40)
+    q, k, v, gate, qw, kw, bias = _fp8_problem(B, 31)
+    k[:] = 0
+    rng = np.random.default_rng(7)
+    vcodes_new = rng.integers(0, 0x7F, size=v.shape).astype(np.uint8) | \
+        (rng.integers(0, 2, size=v.shape).astype(np.uint8) << 7)
+    v = _grid_bf16(orc, vcodes_new, 0.5)      # exactly representable after / 0.5
+    kc = rng.integers(0, 256, size=(B, Hkv, slots, d)).astype(np.uint8)
+    vc = rng.integers(0, 256, size=(B, Hkv, slots, d)).astype(np.uint8)
+    for c in (kc, vc):
+        c[(c & 0x7F) == 0x7F] ^= 0x01        # no NaN codes
+    got = orc.decode_fp8(kind, P, q, k, v, gate, qw, kw, bias, pos, kc, vc, 2.0, 0.5)
+    ref = orc.decode(kind, P, q, k, v, gate, qw, kw, bias, pos, _grid_bf16(orc, kc, 2.0),
+                     _grid_bf16(orc, vc, 0.5))
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-13)
+
+
+def test_decode_fp8_window_of_one_is_the_quantised_new_value(orc):
+    """W = 1: the output is the new token's value read back from its code, gated."""
+    d, Hq, Hkv = 16, 6, 2
+    P = orc.params(n_q_heads=Hq, n_kv_heads=Hkv, head_dim=d, window=1)
+    q, k, v, gate, qw, kw, bias = _fp8_problem(2, 32)
+    kc = np.zeros((2, Hkv, 1, d), np.uint8)
+    pos = np.array([0, 77], np.int64)
+    vs = 0.75
+    got = orc.decode_fp8(orc.LOCAL, P, q, k, v, gate, qw, kw, bias, pos, kc, kc, 1.0, vs)
+    vf = wl.bf16_bits_to_f32(v).astype(np.float64).reshape(2, Hkv, d)
+    deq = np.vectorize(lambda x: orc.e4m3_decode(orc.e4m3_encode(x / vs)) * vs)(vf)
+    assert np.max(np.abs(deq - vf)) > 0            # the quantisation is visible
+    g = wl.bf16_bits_to_f32(gate).astype(np.float64).reshape(2, Hq, d)
+    sig = 1.0 / (1.0 + np.exp(-(g + bias[None, :, None])))
+    ref = deq[:, np.arange(Hq) // (Hq // Hkv)] * sig
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-14)
+
+
+def test_kv_row_fp8_codes_are_nearest_to_the_exact_rows(orc):
+    """Each code's value is within half an E4M3 step of the exact prepared key / raw
+    value (relative 2^-4 in the normal range); a value on the grid is exact."""
+    d, Hkv = 16, 2
+    P = orc.params(n_q_heads=6, n_kv_heads=Hkv, head_dim=d, window=8)
+    k, v = _rand((Hkv * d,), 33, "k"), _rand((Hkv * d,), 33, "v")
+    kw = wl.norm_weight(33, "kw")[:d]
+    for kind in (0, 1):
+        kr, vr = orc.kv_row_fp8(kind, P, k, v, kw, 5, 0.5, 2.0)
+        exact_k = np.stack([orc.prepare_key(kind, P, k[g * d:(g + 1) * d], kw, 5)
+                            for g in range(Hkv)])
+        exact_v = wl.bf16_bits_to_f32(v).astype(np.float64).reshape(Hkv, d)
+        for codes, exact, sc in ((kr, exact_k, 0.5), (vr, exact_v, 2.0)):
+            deq = np.vectorize(orc.e4m3_decode)(codes) * sc
+            assert np.all(np.abs(deq - exact) <= np.maximum(np.abs(exact) * 2.0 ** -4,
+                                                             2.0 ** -10 * sc) * 1.0000001)
+    grid = _grid_bf16(orc, np.arange(0x30, 0x50, dtype=np.uint8)[:Hkv * d], 1.0)
+    _, vr = orc.kv_row_fp8(1, P, k, grid, kw, 0, 1.0, 1.0)
+    np.testing.assert_array_equal(vr.ravel(), np.arange(0x30, 0x50, dtype=np.uint8)[:Hkv * d])
+
+
 # ---------------------------------------------------------------- bf16
 def test_bf16_rounding_ties_to_even(orc):
     cases = {1.0 + 2.0 ** -8: 0x3F80, 1.0 + 3 * 2.0 ** -8: 0x3F82, -2.5: 0xC020,
