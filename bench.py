@@ -41,11 +41,11 @@ def prefill_flops(B: int, T: int, kind: int, window: int = wl.WINDOW) -> int:
     return B * pairs * HEAD_FLOPS_PER_PAIR
 
 
-def decode_kv_bytes(ctx, kind: int, window: int = wl.WINDOW) -> int:
+def decode_kv_bytes(ctx, kind: int, window: int = wl.WINDOW, elem_bytes: int = 2) -> int:
     """Algorithmic bytes of one decode layer: the visible K and V rows (4 KiB per
-    token per layer) plus the new token's q, k, v, gate and output."""
+    token per layer in bf16, 2 KiB in FP8) plus the new token's q, k, v, gate and output."""
     vis = sum(min(c, window) if kind == wl.LOCAL else c for c in ctx)
-    per_token = 2 * wl.N_KV_HEADS * wl.HEAD_DIM * 2
+    per_token = 2 * wl.N_KV_HEADS * wl.HEAD_DIM * elem_bytes
     io = len(ctx) * 2 * (3 * wl.N_Q_HEADS * wl.HEAD_DIM + 2 * wl.N_KV_HEADS * wl.HEAD_DIM)
     return vis * per_token + io
 
@@ -218,8 +218,9 @@ class PrefillLayer:
 
 
 class DecodeLayer:
-    def __init__(self, torch, beam, kind, ctx, slots, seed, tag, cache=None):
-        self.torch, self.beam, self.kind = torch, beam, kind
+    def __init__(self, torch, beam, kind, ctx, slots, seed, tag, cache=None, fp8=False):
+        self.torch, self.beam, self.kind, self.fp8 = torch, beam, kind, fp8
+        self.k_scale, self.v_scale = 0.5, 1.0
         self.params = beam.default_params()
         dev = "cuda"
         ctx = np.asarray(ctx, np.int64)
@@ -233,8 +234,16 @@ class DecodeLayer:
         self.kw = torch.from_numpy(di.k_norm_w).to(dev)
         self.bias = torch.from_numpy(di.gate_bias).to(dev)
         self.pos = torch.from_numpy(di.pos).to(dev)
-        self.layout = beam.beam_kv_layout(kind, self.params, self.B, slots)
-        if cache is None:
+        if fp8:
+            self.layout = beam.beam_kv_layout_fp8(kind, self.params, self.B, slots)
+        else:
+            self.layout = beam.beam_kv_layout(kind, self.params, self.B, slots)
+        if cache is None and fp8:
+            self.kc = torch.empty(self.layout.bytes_k, dtype=torch.uint8, device=dev)
+            self.vc = torch.empty_like(self.kc)
+            wl.device_normal_e4m3_(self.kc, seed, f"{tag}/kc", self.k_scale)
+            wl.device_normal_e4m3_(self.vc, seed, f"{tag}/vc", self.v_scale)
+        elif cache is None:
             self.kc = torch.empty(self.layout.bytes_k // 2, dtype=torch.bfloat16, device=dev)
             self.vc = torch.empty_like(self.kc)
             wl.device_normal_bf16_(self.kc, seed, f"{tag}/kc")
@@ -246,11 +255,18 @@ class DecodeLayer:
                                                                       self.layout)),
                               dtype=torch.uint8, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
-        self.bytes = decode_kv_bytes(ctx, kind)
+        self.bytes = decode_kv_bytes(ctx, kind, elem_bytes=1 if fp8 else 2)
         # a ring layer is one launch; a global layer is split-K + combine
         self.launches_per_call = 1 if kind == wl.LOCAL else 2
 
     def run(self):
+        if self.fp8:
+            self.beam.beam_attn_decode_fp8(self.kind, self.params, self.q, self.k, self.v,
+                                           self.gate, self.qw, self.kw, self.bias, self.pos,
+                                           self.kc, self.vc, self.layout, self.k_scale,
+                                           self.v_scale, self.out, workspace=self.ws,
+                                           dev_status=self.status)
+            return
         self.beam.beam_attn_decode(self.kind, self.params, self.q, self.k, self.v, self.gate,
                                    self.qw, self.kw, self.bias, self.pos, self.kc, self.vc,
                                    self.layout, self.out, workspace=self.ws, dev_status=self.status)
@@ -270,20 +286,15 @@ def time_loop(torch, fn, steps, warmup):
     return ev[0].elapsed_time(ev[1]) / 1e3 / steps
 
 
-def bench_decode_1m(torch, beam, steps, warmup, seed):
-    """52-layer decode step at context 1,048,576: 9 global layers with 4 GiB caches,
-    43 local rings; the whole step is one CUDA graph replay."""
+def bench_decode_1m(torch, beam, steps, warmup, seed, fp8=False):
+    """52-layer decode step at context 1,048,576: 9 global layers with 4 GiB caches
+    (2 GiB in FP8), 43 local rings; the whole step is one CUDA graph replay."""
     layers = []
-    ring_cache = None
     for i in range(1, wl.N_LAYERS + 1):
         kind = wl.layer_kind(i)
-        if kind == wl.GLOBAL:
-            layers.append(DecodeLayer(torch, beam, kind, [wl.MAX_CONTEXT], wl.MAX_CONTEXT, seed,
-                                      f"d1m/L{i}"))
-        else:
-            layers.append(DecodeLayer(torch, beam, kind, [wl.MAX_CONTEXT], wl.WINDOW, seed,
-                                      f"d1m/L{i}"))
-    del ring_cache
+        slots = wl.MAX_CONTEXT if kind == wl.GLOBAL else wl.WINDOW
+        layers.append(DecodeLayer(torch, beam, kind, [wl.MAX_CONTEXT], slots, seed,
+                                  f"d1m/L{i}", fp8=fp8))
     total_bytes = sum(L.bytes for L in layers)
     glob_bytes = sum(L.bytes for L in layers if L.kind == wl.GLOBAL)
 
@@ -307,7 +318,9 @@ def bench_decode_1m(torch, beam, steps, warmup, seed):
     status = [int(L.status.item()) for L in layers]
     assert all(s == 0 for s in status), status
     res = {
-        "workload": "decode_1m: B=1, context 1048576, 52 layers (9 global 4 GiB caches, 43 x 512-slot rings)",
+        "workload": ("decode_1m_fp8: B=1, context 1048576, 52 layers, FP8 E4M3 caches (9 global "
+                     "2 GiB caches, 43 x 512-slot rings)") if fp8 else
+                    "decode_1m: B=1, context 1048576, 52 layers (9 global 4 GiB caches, 43 x 512-slot rings)",
         "ms_per_token": sec * 1e3,
         "tokens_per_s": 1.0 / sec,
         "kv_read_GBps": total_bytes / sec / 1e9,
@@ -565,6 +578,9 @@ def run_gpu(args):
         db = bench_decode_batched(torch, beam, args.steps, args.warmup, args.seed)
         db["pct_of_hbm"] = round(100 * db["kv_read_GBps"] / pk["hbm_gbs"], 2)
         result["decode_batched"] = db
+        d8, _ = bench_decode_1m(torch, beam, args.steps, args.warmup, args.seed, fp8=True)
+        d8["pct_of_hbm"] = round(100 * d8["kv_read_GBps"] / pk["hbm_gbs"], 2)
+        result["decode_1m_fp8"] = d8
         pc = bench_prefill_chunk(torch, beam, args.steps, args.warmup, args.seed)
         pc["pct_of_bf16_peak"] = round(100 * pc["tflops"] / pk["bf16_tflops"], 2)
         result["prefill_chunk"] = pc

@@ -28,6 +28,7 @@ EXPORTS = (
     "beam_default_params", "beam_kv_layout", "beam_prefill_workspace_bytes", "beam_attn_prefill",
     "beam_kv_append", "beam_decode_workspace_bytes", "beam_attn_decode", "beam_status_string",
     "beam_attn_decode_noalloc", "beam_prefill_chunk_workspace_bytes", "beam_attn_prefill_chunk",
+    "beam_kv_layout_fp8", "beam_kv_append_fp8", "beam_attn_decode_fp8",
 )
 
 
@@ -92,6 +93,15 @@ def lib() -> ctypes.CDLL:
         L.beam_attn_decode_noalloc.restype = ctypes.c_int
         L.beam_attn_decode_noalloc.argtypes = [ctypes.c_int, pp, i32, vp, vp, vp, vp, vp, vp, vp,
                                                vp, vp, vp, lp, vp, vp, vp]
+        f32 = ctypes.c_float
+        L.beam_kv_layout_fp8.restype = ctypes.c_int
+        L.beam_kv_layout_fp8.argtypes = [ctypes.c_int, pp, i32, i64, lp]
+        L.beam_kv_append_fp8.restype = ctypes.c_int
+        L.beam_kv_append_fp8.argtypes = [ctypes.c_int, pp, i32, i32, vp, vp, vp, vp, vp, vp, lp,
+                                         f32, f32, vp, vp]
+        L.beam_attn_decode_fp8.restype = ctypes.c_int
+        L.beam_attn_decode_fp8.argtypes = [ctypes.c_int, pp, i32, vp, vp, vp, vp, vp, vp, vp, vp,
+                                           vp, vp, lp, f32, f32, vp, vp, sz, vp, vp]
         L.beam_status_string.restype = ctypes.c_char_p
         L.beam_status_string.argtypes = [ctypes.c_int]
         _lib = L
@@ -228,6 +238,43 @@ def beam_attn_decode_noalloc(kind, params, q, k, v, gate, q_norm_w, k_norm_w, ga
         _ptr(k_norm_w), _ptr(gate_bias), _ptr(pos), _ptr(k_cache), _ptr(v_cache),
         ctypes.byref(layout), _ptr(out), _ptr(dev_status), _stream(stream))
     _check("beam_attn_decode_noalloc", rc)
+    return out
+
+
+def beam_kv_layout_fp8(kind: int, params: Params, batch: int, capacity_tokens: int) -> KVLayout:
+    """Layout of an FP8 E4M3 cache (one byte per element; same element strides)."""
+    out = KVLayout()
+    _check("beam_kv_layout_fp8", lib().beam_kv_layout_fp8(kind, ctypes.byref(params), batch,
+                                                          capacity_tokens, ctypes.byref(out)))
+    return out
+
+
+def beam_kv_append_fp8(kind, params, k, v, k_norm_w, pos0, k_cache, v_cache, layout: KVLayout,
+                       k_scale: float, v_scale: float, dev_status=None, stream=None):
+    """k, v: [B, T, 1024] bf16; caches: uint8 code arrays of the FP8 layout."""
+    B, T = k.shape[0], k.shape[1]
+    rc = lib().beam_kv_append_fp8(kind, ctypes.byref(params), B, T, _ptr(k), _ptr(v),
+                                  _ptr(k_norm_w), _ptr(pos0), _ptr(k_cache), _ptr(v_cache),
+                                  ctypes.byref(layout), float(k_scale), float(v_scale),
+                                  _ptr(dev_status), _stream(stream))
+    _check("beam_kv_append_fp8", rc)
+
+
+def beam_attn_decode_fp8(kind, params, q, k, v, gate, q_norm_w, k_norm_w, gate_bias, pos, k_cache,
+                         v_cache, layout: KVLayout, k_scale: float, v_scale: float, out,
+                         workspace=None, dev_status=None, stream=None):
+    """Decode over FP8 E4M3 caches (uint8 code arrays); otherwise as beam_attn_decode."""
+    B = q.shape[0]
+    need = beam_decode_workspace_bytes(kind, params, B, layout)
+    if workspace is None:
+        workspace = _workspace(need, q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    rc = lib().beam_attn_decode_fp8(
+        kind, ctypes.byref(params), B, _ptr(q), _ptr(k), _ptr(v), _ptr(gate), _ptr(q_norm_w),
+        _ptr(k_norm_w), _ptr(gate_bias), _ptr(pos), _ptr(k_cache), _ptr(v_cache),
+        ctypes.byref(layout), float(k_scale), float(v_scale), _ptr(out), _ptr(workspace),
+        ws_bytes, _ptr(dev_status), _stream(stream))
+    _check("beam_attn_decode_fp8", rc)
     return out
 
 

@@ -18,6 +18,7 @@
 #include "beam_attn.h"
 #include "common.cuh"
 #include "decode.cuh"
+#include "decode8.cuh"
 #include "prefill_tc.cuh"
 #include "prologue.cuh"
 
@@ -64,6 +65,14 @@ int device_info(DeviceInfo **out) {
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem),
                           "decode shared-memory opt-in")))
       return st;
+    if ((st = cuda_status(cudaFuncSetAttribute(decode8_attn_kernel<false>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, kDec8Smem),
+                          "FP8 decode shared-memory opt-in")))
+      return st;
+    if ((st = cuda_status(cudaFuncSetAttribute(decode8_attn_kernel<true>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, kDec8Smem),
+                          "FP8 decode shared-memory opt-in")))
+      return st;
     if ((st = cuda_status(cudaFuncSetAttribute(prefill_tc_kernel,
                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                kTcSmemBytes),
@@ -100,6 +109,16 @@ int check_layout(int kind, const beam_attn_params *p, const beam_kv_layout_t *L)
   if (kind == BEAM_LOCAL && L->slots_per_seq != p->window) return BEAM_ERR_INVALID_ARG;
   return BEAM_OK;
 }
+
+// An FP8 cache holds one-byte codes: its rows must start on 16 bytes as well.
+int check_layout_fp8(int kind, const beam_attn_params *p, const beam_kv_layout_t *L) {
+  int st = check_layout(kind, p, L);
+  if (st) return st;
+  if ((L->stride_head % 16) || (L->stride_seq % 16)) return BEAM_ERR_ALIGNMENT;
+  return BEAM_OK;
+}
+
+bool valid_scale(float s) { return std::isfinite(s) && s > 0.f && std::isfinite(1.0f / s); }
 
 void fill_inv_freq(double (&f)[64], double theta) {
   for (int i = 0; i < 64; ++i) f[i] = std::pow(theta, -2.0 * i / (double)kD);
@@ -513,12 +532,18 @@ size_t beam_decode_workspace_bytes(int kind, const beam_attn_params *p, int32_t 
   return decode_workspace(nullptr, B, n_split_max).bytes;
 }
 
-int beam_attn_decode(int kind, const beam_attn_params *p, int32_t B, const void *q, const void *k,
-                     const void *v, const void *gate, const float *q_norm_w,
-                     const float *k_norm_w, const float *gate_bias, const int64_t *pos,
-                     void *k_cache, void *v_cache, const beam_kv_layout_t *layout, void *out,
-                     void *workspace, size_t workspace_bytes, int32_t *dev_status,
-                     beam_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// One decode step over a BF16 cache (fp8 == false) or an FP8 E4M3 cache with the given
+// scales: validation, then one cluster launch (local ring) or split-K + combine (global).
+int decode_call(int kind, const beam_attn_params *p, int32_t B, const void *q, const void *k,
+                const void *v, const void *gate, const float *q_norm_w, const float *k_norm_w,
+                const float *gate_bias, const int64_t *pos, void *k_cache, void *v_cache,
+                const beam_kv_layout_t *layout, void *out, void *workspace,
+                size_t workspace_bytes, int32_t *dev_status, beam_stream_t stream, bool fp8,
+                float k_scale, float v_scale) {
   int st = check_params(kind, p);
   if (st) return st;
   if (B < 0) return BEAM_ERR_INVALID_ARG;
@@ -530,7 +555,8 @@ int beam_attn_decode(int kind, const beam_attn_params *p, int32_t B, const void 
       !aligned16(q_norm_w) || !aligned16(k_norm_w) || !aligned16(k_cache) || !aligned16(v_cache) ||
       !aligned16(workspace) || (reinterpret_cast<uintptr_t>(pos) & 7u))
     return BEAM_ERR_ALIGNMENT;
-  if ((st = check_layout(kind, p, layout))) return st;
+  if ((st = fp8 ? check_layout_fp8(kind, p, layout) : check_layout(kind, p, layout))) return st;
+  if (fp8 && (!valid_scale(k_scale) || !valid_scale(v_scale))) return BEAM_ERR_INVALID_ARG;
   DeviceInfo *dev = nullptr;
   if ((st = device_info(&dev))) return st;
   const int split = decode_split(kind, p, B, layout->slots_per_seq, dev->sm_count);
@@ -572,6 +598,12 @@ int beam_attn_decode(int kind, const beam_attn_params *p, int32_t B, const void 
   da.status = dev_status;
   da.eps = p->rms_eps;
   fill_inv_freq(da.inv_freq, p->rope_theta);
+  Decode8Args d8;
+  d8.base = da;
+  d8.k_scale = k_scale;
+  d8.v_scale = v_scale;
+  d8.inv_k_scale = 1.0f / k_scale;
+  d8.inv_v_scale = 1.0f / v_scale;
 
   if (kind == BEAM_LOCAL) {
     // one launch: the ring's splits form a cluster that also merges through distributed
@@ -580,7 +612,7 @@ int beam_attn_decode(int kind, const beam_attn_params *p, int32_t B, const void 
     memset(&cfg, 0, sizeof cfg);
     cfg.gridDim = grid;
     cfg.blockDim = dim3(kDecThreads);
-    cfg.dynamicSmemBytes = kDecSmem;
+    cfg.dynamicSmemBytes = fp8 ? kDec8Smem : kDecSmem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -589,10 +621,15 @@ int beam_attn_decode(int kind, const beam_attn_params *p, int32_t B, const void 
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cuda_status(cudaLaunchKernelEx(&cfg, decode_attn_kernel<true>, da), "ring decode launch");
+    return cuda_status(fp8 ? cudaLaunchKernelEx(&cfg, decode8_attn_kernel<true>, d8)
+                           : cudaLaunchKernelEx(&cfg, decode_attn_kernel<true>, da),
+                       "ring decode launch");
   }
 
-  decode_attn_kernel<false><<<grid, kDecThreads, kDecSmem, s>>>(da);
+  if (fp8)
+    decode8_attn_kernel<false><<<grid, kDecThreads, kDec8Smem, s>>>(d8);
+  else
+    decode_attn_kernel<false><<<grid, kDecThreads, kDecSmem, s>>>(da);
   if ((st = launch_status())) return st;
 
   CombineArgs ca;
@@ -608,6 +645,83 @@ int beam_attn_decode(int kind, const beam_attn_params *p, int32_t B, const void 
   ca.n_split_max = n_split_max;
   ca.slots = layout->slots_per_seq;
   decode_combine_kernel<<<dim3(kHq, B), 256, 0, s>>>(ca);
+  return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+int beam_attn_decode(int kind, const beam_attn_params *p, int32_t B, const void *q, const void *k,
+                     const void *v, const void *gate, const float *q_norm_w,
+                     const float *k_norm_w, const float *gate_bias, const int64_t *pos,
+                     void *k_cache, void *v_cache, const beam_kv_layout_t *layout, void *out,
+                     void *workspace, size_t workspace_bytes, int32_t *dev_status,
+                     beam_stream_t stream) {
+  return decode_call(kind, p, B, q, k, v, gate, q_norm_w, k_norm_w, gate_bias, pos, k_cache,
+                     v_cache, layout, out, workspace, workspace_bytes, dev_status, stream, false,
+                     1.0f, 1.0f);
+}
+
+int beam_attn_decode_fp8(int kind, const beam_attn_params *p, int32_t B, const void *q,
+                         const void *k, const void *v, const void *gate, const float *q_norm_w,
+                         const float *k_norm_w, const float *gate_bias, const int64_t *pos,
+                         void *k_cache, void *v_cache, const beam_kv_layout_t *layout,
+                         float k_scale, float v_scale, void *out, void *workspace,
+                         size_t workspace_bytes, int32_t *dev_status, beam_stream_t stream) {
+  return decode_call(kind, p, B, q, k, v, gate, q_norm_w, k_norm_w, gate_bias, pos, k_cache,
+                     v_cache, layout, out, workspace, workspace_bytes, dev_status, stream, true,
+                     k_scale, v_scale);
+}
+
+int beam_kv_layout_fp8(int kind, const beam_attn_params *p, int32_t batch,
+                       int64_t capacity_tokens, beam_kv_layout_t *out) {
+  int st = beam_kv_layout(kind, p, batch, capacity_tokens, out);
+  if (st) return st;
+  out->bytes_k = (int64_t)batch * out->stride_seq;   // one byte per element
+  out->bytes_v = out->bytes_k;
+  return BEAM_OK;
+}
+
+int beam_kv_append_fp8(int kind, const beam_attn_params *p, int32_t B, int32_t T, const void *k,
+                       const void *v, const float *k_norm_w, const int64_t *pos0, void *k_cache,
+                       void *v_cache, const beam_kv_layout_t *layout, float k_scale,
+                       float v_scale, int32_t *dev_status, beam_stream_t stream) {
+  int st = check_params(kind, p);
+  if (st) return st;
+  if (B < 0 || T < 0) return BEAM_ERR_INVALID_ARG;
+  if (B == 0 || T == 0) return BEAM_OK;
+  if (!k || !v || !k_norm_w || !pos0 || !k_cache || !v_cache) return BEAM_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_norm_w) || !aligned16(k_cache) ||
+      !aligned16(v_cache) || (reinterpret_cast<uintptr_t>(pos0) & 7u))
+    return BEAM_ERR_ALIGNMENT;
+  if ((st = check_layout_fp8(kind, p, layout))) return st;
+  if (!valid_scale(k_scale) || !valid_scale(v_scale)) return BEAM_ERR_INVALID_ARG;
+  if ((int64_t)B * T > INT32_MAX) return BEAM_ERR_UNSUPPORTED;
+  DeviceInfo *dev = nullptr;
+  if ((st = device_info(&dev))) return st;
+  PrologueArgs pa;
+  memset(&pa, 0, sizeof pa);
+  pa.k = static_cast<const uint16_t *>(k);
+  pa.v = static_cast<const uint16_t *>(v);
+  pa.qw = k_norm_w;  // unused: no query rows
+  pa.kw = k_norm_w;
+  pa.k_cache = static_cast<uint16_t *>(k_cache);
+  pa.v_cache = static_cast<uint16_t *>(v_cache);
+  pa.stride_seq = layout->stride_seq;
+  pa.stride_head = layout->stride_head;
+  pa.slots = layout->slots_per_seq;
+  pa.pos0 = pos0;
+  pa.cache_fp8 = 1;
+  pa.inv_k_scale = 1.0f / k_scale;
+  pa.inv_v_scale = 1.0f / v_scale;
+  pa.status = dev_status;
+  pa.T = T;
+  pa.kind = kind;
+  pa.window = p->window;
+  pa.eps = p->rms_eps;
+  fill_inv_freq(pa.inv_freq, p->rope_theta);
+  prologue_kernel<<<(unsigned)((size_t)B * T), 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(pa);
   return launch_status();
 }
 

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -74,6 +75,22 @@ __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t add
 // XOR-swizzled so that eight consecutive rows at one chunk hit distinct banks.
 __device__ __forceinline__ uint32_t swz256(int r, int c) {
   return (uint32_t)(r * 256 + ((c ^ (r & 7)) << 4));
+}
+
+// Two E4M3 codes (low byte first) -> fp16x2 (low half first); exact.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two & 0xFFFFu), __NV_E4M3);
+  return (uint32_t)h.x | ((uint32_t)h.y << 16);
+}
+
+// Eight fp32 values -> eight E4M3 codes (value * inv_scale, nearest, saturating), in order.
+__device__ __forceinline__ uint2 f32x8_to_e4m3(const float (&x)[8], float inv_scale) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    w[i] = __nv_cvt_float2_to_fp8x2(make_float2(x[2 * i] * inv_scale, x[2 * i + 1] * inv_scale),
+                                    __NV_SATFINITE, __NV_E4M3);
+  return make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
 }
 
 }  // namespace beam

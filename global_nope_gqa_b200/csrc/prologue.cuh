@@ -38,6 +38,8 @@ struct PrologueArgs {
   float *rope_tab;       // local layers, or null: cos (64) then sin (64) of each token's angles
   int rope_per_seq;      // rope_tab is [B][T][128] (own positions) rather than [T][128] (0 .. T-1)
   int whole_seq;         // a sequence whose tokens do not all fit is not written at all
+  int cache_fp8;         // the caches hold E4M3 codes of value * inv scale (one byte each)
+  float inv_k_scale, inv_v_scale;
   int32_t *status;
   int T;                 // tokens per sequence in this call
   int kind;
@@ -64,11 +66,11 @@ __device__ __forceinline__ void rope_angles(const double *inv_freq, int64_t t, i
 // RMSNorm of one 128-wide row held by a half-warp (lane l16 holds coordinates
 // 8 l16 .. 8 l16 + 7 as eight bf16 in `raw`), times the weights w, then -- for a local
 // layer -- rotate-half RoPE with the angles' cos / sin (the partner of coordinate c < 64 is
-// c + 64, held by lane l16 ^ 8).  Returns the eight results as bf16.
-__device__ __forceinline__ uint4 norm_rope_row(uint4 raw, const float (&w)[8], bool rope,
-                                               const float (&cs)[8], const float (&sn)[8],
-                                               int l16, unsigned half_mask, float eps) {
-  float x[8];
+// c + 64, held by lane l16 ^ 8).  The eight results in fp32.
+__device__ __forceinline__ void norm_rope_f32(uint4 raw, const float (&w)[8], bool rope,
+                                              const float (&cs)[8], const float (&sn)[8],
+                                              int l16, unsigned half_mask, float eps,
+                                              float (&x)[8]) {
   x[0] = bf16_lo(raw.x); x[1] = bf16_hi(raw.x); x[2] = bf16_lo(raw.y); x[3] = bf16_hi(raw.y);
   x[4] = bf16_lo(raw.z); x[5] = bf16_hi(raw.z); x[6] = bf16_lo(raw.w); x[7] = bf16_hi(raw.w);
   float ss = 0.f;
@@ -89,6 +91,14 @@ __device__ __forceinline__ uint4 norm_rope_row(uint4 raw, const float (&w)[8], b
 #pragma unroll
     for (int e = 0; e < 8; ++e) x[e] = y[e];
   }
+}
+
+// The same row rounded to bf16.
+__device__ __forceinline__ uint4 norm_rope_row(uint4 raw, const float (&w)[8], bool rope,
+                                               const float (&cs)[8], const float (&sn)[8],
+                                               int l16, unsigned half_mask, float eps) {
+  float x[8];
+  norm_rope_f32(raw, w, rope, cs, sn, l16, half_mask, eps, x);
   uint4 res;
   res.x = pack_bf16(x[0], x[1]); res.y = pack_bf16(x[2], x[3]);
   res.z = pack_bf16(x[4], x[5]); res.w = pack_bf16(x[6], x[7]);
@@ -167,8 +177,18 @@ __global__ void __launch_bounds__(128) prologue_kernel(const PrologueArgs a) {
     const uint16_t *src = is_q ? a.q + (size_t)tok * (kHq * kD) + head * kD
                                : (is_k ? a.k : a.v) + (size_t)tok * (kHkv * kD) + head * kD;
     uint4 raw = *reinterpret_cast<const uint4 *>(src + l16 * 8);
-    const uint4 res = is_v ? raw : norm_rope_row(raw, is_q ? wq : wk, local, cs, sn, l16,
-                                                 half_mask, a.eps);
+    float x[8];
+    if (is_v) {
+      x[0] = bf16_lo(raw.x); x[1] = bf16_hi(raw.x); x[2] = bf16_lo(raw.y); x[3] = bf16_hi(raw.y);
+      x[4] = bf16_lo(raw.z); x[5] = bf16_hi(raw.z); x[6] = bf16_lo(raw.w); x[7] = bf16_hi(raw.w);
+    } else {
+      norm_rope_f32(raw, is_q ? wq : wk, local, cs, sn, l16, half_mask, a.eps, x);
+    }
+    uint4 res = raw;
+    if (!is_v) {
+      res.x = pack_bf16(x[0], x[1]); res.y = pack_bf16(x[2], x[3]);
+      res.z = pack_bf16(x[4], x[5]); res.w = pack_bf16(x[6], x[7]);
+    }
     if (is_q) {
       *reinterpret_cast<uint4 *>(a.q_out + (size_t)tok * (kHq * kD) + head * kD + l16 * 8) = res;
     } else {
@@ -178,9 +198,16 @@ __global__ void __launch_bounds__(128) prologue_kernel(const PrologueArgs a) {
         *reinterpret_cast<uint4 *>(dst + orow * (kHkv * kD) + head * kD + l16 * 8) = res;
       }
       if (write_cache) {
-        uint16_t *cache = is_k ? a.k_cache : a.v_cache;
-        size_t off = (size_t)b * a.stride_seq + (size_t)head * a.stride_head + (size_t)slot * kD;
-        *reinterpret_cast<uint4 *>(cache + off + l16 * 8) = res;
+        const size_t off = (size_t)b * a.stride_seq + (size_t)head * a.stride_head +
+                           (size_t)slot * kD + l16 * 8;
+        if (a.cache_fp8) {   // codes of the fp32 rows, not of their bf16 rounding
+          uint8_t *cache = reinterpret_cast<uint8_t *>(is_k ? a.k_cache : a.v_cache);
+          *reinterpret_cast<uint2 *>(cache + off) =
+              f32x8_to_e4m3(x, is_k ? a.inv_k_scale : a.inv_v_scale);
+        } else {
+          uint16_t *cache = is_k ? a.k_cache : a.v_cache;
+          *reinterpret_cast<uint4 *>(cache + off) = res;
+        }
       }
     }
   }

@@ -204,6 +204,42 @@ BEAM_API int beam_attn_decode(int kind, const beam_attn_params *p, int32_t B, co
                      void *workspace, size_t workspace_bytes, int32_t *dev_status,
                      beam_stream_t stream);
 
+/* ---- FP8 E4M3 KV cache (section "KV memory": 18 KiB per token over the nine
+ * global layers instead of 36 KiB in BF16).  Each element of an FP8 cache is one
+ * E4M3 code (OCP FP8 E4M3: bias 7, no infinities, largest finite 448) of
+ * value / scale, with one float scale per cache tensor of a layer (k_scale for
+ * the keys, v_scale for the values; finite and > 0, else BEAM_ERR_INVALID_ARG).
+ * Codes are the nearest, ties to even, saturating at +-448; keys are quantised
+ * from their fp32 normalised (local: rotated) values, values from their raw
+ * bf16 values.  A code reads back as E4M3^-1(code) * scale. */
+
+/* Layout of an FP8 cache: the same head-major [B][8][slots][128] element order
+ * and strides as beam_kv_layout, one byte per element (bytes_k, bytes_v
+ * halved).  Rows must start on 16 bytes: strides multiples of 16 elements. */
+BEAM_API int beam_kv_layout_fp8(int kind, const beam_attn_params *p, int32_t batch,
+                                int64_t capacity_tokens, beam_kv_layout_t *out);
+
+/* beam_kv_append into an FP8 cache (same positions, slots and capacity
+ * behaviour). */
+BEAM_API int beam_kv_append_fp8(int kind, const beam_attn_params *p, int32_t B, int32_t T,
+                                const void *k, const void *v, const float *k_norm_w,
+                                const int64_t *pos0, void *k_cache, void *v_cache,
+                                const beam_kv_layout_t *layout, float k_scale, float v_scale,
+                                int32_t *dev_status, beam_stream_t stream);
+
+/* beam_attn_decode over an FP8 cache: the new key and value are written as
+ * codes, then the query attends over the cached codes read back as values (the
+ * new token's too).  Workspace as for beam_attn_decode
+ * (beam_decode_workspace_bytes with the FP8 layout). */
+BEAM_API int beam_attn_decode_fp8(int kind, const beam_attn_params *p, int32_t B, const void *q,
+                                  const void *k, const void *v, const void *gate,
+                                  const float *q_norm_w, const float *k_norm_w,
+                                  const float *gate_bias, const int64_t *pos, void *k_cache,
+                                  void *v_cache, const beam_kv_layout_t *layout, float k_scale,
+                                  float v_scale, void *out, void *workspace,
+                                  size_t workspace_bytes, int32_t *dev_status,
+                                  beam_stream_t stream);
+
 /* Decode without any allocation, for callers that cannot call cudaMalloc.
  *
  * There is no counterpart in the paper: this is a deployment convenience.  Some

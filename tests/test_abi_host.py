@@ -185,5 +185,22 @@ def test_host_validation_rejects_before_launch(beam):
                                             ws_bytes=0)) == -5          # T = 16 > 15 slots
     assert L.beam_attn_prefill_chunk(*cargs(kind=0, layout=ctypes.byref(small))) == -1
 
+    # FP8 cache: one byte per element, rows on 16 bytes, positive finite scales
+    f8 = beam.beam_kv_layout_fp8(beam.GLOBAL, p, 2, 4096)
+    assert f8.bytes_k == 2 * 8 * 4096 * 128 and f8.stride_slot == 128
+    assert L.beam_kv_append_fp8(1, P, 1, 4, A, A, A, A, A, A, ctypes.byref(f8), 0.0, 1.0, None,
+                                None) == -1
+    assert L.beam_kv_append_fp8(1, P, 1, 4, A, A, A, A, A, A, ctypes.byref(f8), 1.0,
+                                float("inf"), None, None) == -1
+    odd = beam.beam_kv_layout_fp8(beam.GLOBAL, p, 1, 4096)
+    odd.stride_head = 4096 * 128 + 8         # a bf16-aligned but not FP8-aligned row stride
+    odd.stride_seq = 8 * odd.stride_head
+    assert L.beam_kv_append_fp8(1, P, 1, 4, A, A, A, A, A, A, ctypes.byref(odd), 1.0, 1.0, None,
+                                None) == -7
+    f8args = lambda **kw: [1, P, 2, A, A, A, A, A, A, A, A, A, A, ctypes.byref(f8),
+                           kw.get("ks", 1.0), kw.get("vs", 1.0), A, A, dws, None, None]
+    assert L.beam_attn_decode_fp8(*f8args(ks=-1.0)) == -1
+    assert L.beam_attn_decode_fp8(*f8args(vs=float("nan"))) == -1
+
     for s in (0, -1, -2, -3, -4, -5, -6, -7, -8, 99):
         assert isinstance(beam.beam_status_string(s), str)

@@ -84,6 +84,29 @@ def gate_bias(seed: int, tag: str = "gate_bias") -> np.ndarray:
     return (0.5 * g.standard_normal(N_Q_HEADS)).astype(np.float32)
 
 
+def normal_e4m3(shape, seed: int, tag: str, scale: float = 1.0) -> np.ndarray:
+    """FP8 E4M3 codes (uint8) of seeded N(0,1) draws divided by `scale` -- synthetic
+    cache contents; the draw is rounded to the nearest code by PyTorch's float8_e4m3fn
+    cast (values stay far inside the finite range)."""
+    import torch
+    x = rng(seed, tag).standard_normal(size=shape, dtype=np.float32) / np.float32(scale)
+    return torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def device_normal_e4m3_(tensor_u8, seed: int, tag: str, scale: float = 1.0):
+    """Fill a CUDA uint8 tensor in place with E4M3 codes of seeded N(0,1) / scale draws."""
+    import torch
+    g = torch.Generator(device=tensor_u8.device)
+    g.manual_seed((int(seed) << 32) ^ zlib.crc32(tag.encode()))
+    flat = tensor_u8.view(-1)
+    chunk = 1 << 28
+    for s in range(0, flat.numel(), chunk):
+        part = flat[s:s + chunk]
+        x = torch.randn(part.numel(), device=tensor_u8.device, dtype=torch.float32, generator=g)
+        part.copy_((x / scale).to(torch.float8_e4m3fn).view(torch.uint8))
+    return tensor_u8
+
+
 @dataclass
 class PrefillInputs:
     """bf16 bit patterns (uint16) of one prefill call, token-major as projected."""
