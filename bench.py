@@ -592,6 +592,23 @@ def run_gpu(args):
         torch.distributed.destroy_process_group()
 
 
+def run_decode_case(args):
+    """Profiling case: one global-layer decode call (B=1) at --context, BF16 or FP8 cache,
+    timed alone; prints one JSON line (not the headline)."""
+    import torch
+    torch.cuda.set_device(0)
+    import global_nope_gqa_b200 as beam
+    beam.lib()
+    fp8 = args.decode_case == "fp8"
+    L = DecodeLayer(torch, beam, wl.GLOBAL, [args.context], args.context, args.seed, "case",
+                    fp8=fp8)
+    sec = time_loop(torch, L.run, args.steps, args.warmup)
+    assert int(L.status.item()) == 0
+    print(json.dumps({"case": f"global decode, B=1, context {args.context}, "
+                              f"{'FP8 E4M3' if fp8 else 'BF16'} cache",
+                      "ms": sec * 1e3, "GBps": L.bytes / sec / 1e9}), flush=True)
+
+
 def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
@@ -631,10 +648,15 @@ def main(argv=None):
     ap.add_argument("--layers", default="both", choices=["both", "global", "local"],
                     help="prefill layers per step (profiling cases; the headline step is both)")
     ap.add_argument("--batch", type=int, default=0, help="override B (profiling cases)")
+    ap.add_argument("--decode-case", choices=["bf16", "fp8"], default=None,
+                    help="profiling case: time one global decode call at --context only")
+    ap.add_argument("--context", type=int, default=wl.MAX_CONTEXT)
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
+    if args.decode_case:
+        run_decode_case(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_gpu(args)

@@ -204,17 +204,18 @@ int launch_prefill_attention(int kind, const beam_attn_params *p, int32_t B, int
 }
 
 // Decode split size: cache slots per CTA.  A local ring is cut into at most four
-// splits (one thread-block cluster); a global
-// cache is cut so that the grid holds several waves of the SMs at its largest
-// context, in runs of at least 512 slots (the partial results are then well
-// under 1% of the bytes streamed).
-int decode_split(int kind, const beam_attn_params *p, int32_t B, int64_t slots, int sm_count) {
+// splits (one thread-block cluster); a global cache is cut so that the grid holds about
+// three waves of resident CTAs at its largest context (2 per SM for a BF16 cache, 3 for
+// FP8), in runs of at least 512 slots.  Longer runs measured faster than more waves of
+// shorter ones: each CTA pays a fixed start (queries, first tiles) and end (merge).
+int decode_split(int kind, const beam_attn_params *p, int32_t B, int64_t slots, int sm_count,
+                 bool fp8) {
   if (kind == BEAM_LOCAL) {  // the ring: one split, or up to 4 (a cluster) for small batches
     const size_t ring = round_up((size_t)p->window, kDecTile);
     if ((int64_t)B * kHkv >= 2 * sm_count) return (int)ring;
     return (int)std::max<size_t>(kDecTile, round_up(((size_t)p->window + 3) / 4, kDecTile));
   }
-  const int64_t target_ctas = (int64_t)sm_count * 2 * 8;  // ~8 waves at 2 CTAs per SM
+  const int64_t target_ctas = (int64_t)sm_count * (fp8 ? 3 : 2) * 3;
   int64_t split = 512;
   while (split < 16384 && (int64_t)B * kHkv * ((slots + split - 1) / split) > target_ctas)
     split *= 2;
@@ -526,7 +527,9 @@ size_t beam_decode_workspace_bytes(int kind, const beam_attn_params *p, int32_t 
   DeviceInfo *dev = nullptr;
   int sm = 148;
   if (device_info(&dev) == BEAM_OK) sm = dev->sm_count;
-  const int split = decode_split(kind, p, B, layout->slots_per_seq, sm);
+  // one workspace size serves a BF16 and an FP8 cache: the smaller of their splits
+  const int split = std::min(decode_split(kind, p, B, layout->slots_per_seq, sm, false),
+                             decode_split(kind, p, B, layout->slots_per_seq, sm, true));
   const int64_t vis_max = kind == BEAM_LOCAL ? p->window : layout->slots_per_seq;
   const int n_split_max = (int)((vis_max + split - 1) / split);
   return decode_workspace(nullptr, B, n_split_max).bytes;
@@ -559,7 +562,7 @@ int decode_call(int kind, const beam_attn_params *p, int32_t B, const void *q, c
   if (fp8 && (!valid_scale(k_scale) || !valid_scale(v_scale))) return BEAM_ERR_INVALID_ARG;
   DeviceInfo *dev = nullptr;
   if ((st = device_info(&dev))) return st;
-  const int split = decode_split(kind, p, B, layout->slots_per_seq, dev->sm_count);
+  const int split = decode_split(kind, p, B, layout->slots_per_seq, dev->sm_count, fp8);
   const int64_t vis_max = kind == BEAM_LOCAL ? p->window : layout->slots_per_seq;
   const int n_split_max = (int)((vis_max + split - 1) / split);
   DecodeWorkspace w = decode_workspace(workspace, B, n_split_max);

@@ -93,4 +93,11 @@ __device__ __forceinline__ uint2 f32x8_to_e4m3(const float (&x)[8], float inv_sc
   return make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
 }
 
+// 2^x on the special-function unit (flushes subnormal results to zero; 2^-inf = 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+
 }  // namespace beam

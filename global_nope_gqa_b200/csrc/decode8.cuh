@@ -10,19 +10,28 @@
 // CTA prepares its group's six queries, the owner of the new token's slot writes the new
 // key and value as codes, and the CTA streams its run of slots through a 4-stage cp.async
 // ring of 64-slot tiles (64 x 128 bytes for K and for V; 16-byte chunks XOR-swizzled by
-// row).  Every E4M3 value is exact in fp16, so the codes are widened to fp16 in registers
-// and the m16n8k16 MMAs run on fp16 operands with fp32 accumulation; the queries and the
-// probabilities are fp16 too.  k_scale joins the score scale, v_scale the partial output.
+// row).  S = Q K^T runs on E4M3 MMAs (m16n8k32, fp32 accumulation) straight on the key
+// codes, the six heads as M rows: each query row is split into two E4M3 terms,
+// 16 q = hi + lo with lo = E4M3(16 q - hi), which keeps about 8 significant bits (bf16
+// keeps 8), and both terms go into the same accumulator.  The output is formed transposed,
+// O^T = V^T P^T, on fp16 m16n8k16 MMAs with d as M (eight 16-row tiles) and the heads as
+// N (8 columns, 6 used), so no MMA row is padding: every E4M3 value is exact in fp16, so
+// the value codes are widened to fp16 in registers, and P is fp16 (two E4M3 terms would
+// not hold the small probabilities of a long context).  The score accumulator of a lane
+// (head lane / 4, keys 2c + {0, 1} of an 8-key block, c = lane % 4) is exactly the P^T
+// operand fragment the second MMA wants, so P never leaves registers.  k_scale / 16 joins
+// the score scale, v_scale the partial output.
 //
 // Operand layout.  A dot product over d may visit d in any order as long as both
-// operands use the same one, and so may the sum over keys in P V, so the fragments are
-// laid out for wide shared-memory loads instead of the MMA's natural order:
-//   S = Q K^T: in k-step ks, MMA k-slot 2c + {0, 1} (+ 8) of lane c = lane % 4 is
-//     d = 32 c + 4 ks + {0, 1} ({2, 3}), so a lane reads its 32 bytes of a key row with
-//     two 16-byte loads and takes four bytes per k-step;
-//   O = P V: MMA n-index n of n-block nb is d = 16 n + nb, so a lane holding n = lane / 4
-//     reads 16 contiguous bytes of each of its four key rows and pairs bytes of two keys
-//     with a byte permute; the accumulator column n of n-block nb is then d = 16 n + nb.
+// operands use the same one, and a result row may sit anywhere as long as it is written
+// back to its own d, so the fragments are laid out for wide shared-memory loads:
+//   S = Q K^T: in k-step ks (of 4), MMA k-slot 4c + j (16 + 4c + j) of lane c = lane % 4 is
+//     d = 32 c + 8 ks + j (+ 4), j < 4, so a lane reads its 32 bytes of a key row with two
+//     16-byte loads and takes two words per k-step;
+//   O^T = V^T P^T: row r of tile mt is d = 16 r + mt (r < 8) or 16 (r - 8) + 8 + mt, so a
+//     lane holding rows g = lane / 4 and g + 8 reads 16 contiguous bytes (d = 16 g ..
+//     16 g + 15) of each of its four key rows and pairs bytes of two keys with a byte
+//     permute.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -63,6 +72,26 @@ __device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+__device__ __forceinline__ void mma_e4m3_16832(float (&d)[4], uint32_t a0, uint32_t a2,
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+
+constexpr float kDec8QScale = 16.0f;  // queries are split as E4M3 terms of 16 q
+
+// Four E4M3 codes (bytes 0..3 of w) -> two fp16x2: (byte 0, byte 1) and (byte 2, byte 3),
+// the lower byte in the lower half; exact.
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t w, uint32_t &lo, uint32_t &hi) {
+  asm("{\n .reg .b16 a, b;\n mov.b32 {a, b}, %2;\n cvt.rn.f16x2.e4m3x2 %0, a;\n"
+      " cvt.rn.f16x2.e4m3x2 %1, b;\n}\n"
+      : "=r"(lo), "=r"(hi)
+      : "r"(w));
+}
+
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t r;
   asm("prmt.b32 %0, %1, %2, %3;\n" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
@@ -76,7 +105,8 @@ template <bool kCluster>
 __global__ void __launch_bounds__(kDecThreads) decode8_attn_kernel(const Decode8Args A) {
   const DecodeArgs &a = A.base;
   extern __shared__ __align__(1024) uint8_t smem[];
-  __shared__ __align__(16) __half q_prep[kGroup * kD];
+  __shared__ __align__(16) uint8_t q_hi[kGroup * kD];   // E4M3 codes of 16 q
+  __shared__ __align__(16) uint8_t q_lo[kGroup * kD];   // E4M3 codes of 16 q - hi
   const int s_idx = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int64_t t = a.pos[b];
   const int64_t n_vis = decode_visible(a, t);
@@ -95,19 +125,34 @@ __global__ void __launch_bounds__(kDecThreads) decode8_attn_kernel(const Decode8
   uint8_t *kbase = reinterpret_cast<uint8_t *>(a.k_cache) + head_off;
   uint8_t *vbase = reinterpret_cast<uint8_t *>(a.v_cache) + head_off;
 
+  // Thread tid moves chunk tid % 8 of rows tid / 8 + 16 it, it < 4: its swizzle is the same
+  // in every row it moves, so the four copies differ by constant offsets.
+  const int ld_r = tid >> 3;
+  const uint32_t ld_soff = swz128(ld_r, tid & 7);
+  const uint8_t *ld_k = kbase + (size_t)(key_lo + ld_r) * kD + (tid & 7) * 16;
+  const uint8_t *ld_v = vbase + (size_t)(key_lo + ld_r) * kD + (tid & 7) * 16;
   auto load_tile = [&](int tile, int stage) {
-    uint8_t *ks = smem + stage * 2 * kDec8TileBytes;
-    uint8_t *vs = ks + kDec8TileBytes;
-    const int64_t row0 = key_lo + (int64_t)tile * kDec8Tile;
+    const uint32_t ks = smem_u32(smem + stage * 2 * kDec8TileBytes) + ld_soff;
+    const uint32_t vs = ks + kDec8TileBytes;
+    const size_t goff = (size_t)tile * kDec8TileBytes;
+    const int rows_left = n_keys - tile * kDec8Tile - ld_r;   // this thread's rows: 0, 16, 32, 48
+    if (rows_left > 48) {
 #pragma unroll
-    for (int it = 0; it < (kDec8Tile * 8) / kDecThreads; ++it) {
-      const int id = tid + it * kDecThreads;
-      const int r = id >> 3, c = id & 7;
-      const bool valid = row0 + r < key_hi;
-      const int64_t row = valid ? row0 + r : key_lo;
-      const uint32_t off = swz128(r, c);
-      cp_async16(smem_u32(ks + off), kbase + row * kD + c * 16, valid);
-      cp_async16(smem_u32(vs + off), vbase + row * kD + c * 16, valid);
+      for (int it = 0; it < 4; ++it) {
+        cp_async16(ks + it * 2048, ld_k + goff + it * 2048, true);
+        cp_async16(vs + it * 2048, ld_v + goff + it * 2048, true);
+      }
+    } else {
+      // rows past the run read as zeros (source size 0) and point at the run's first row,
+      // which exists (the run is never empty)
+      const uint8_t *k_first = kbase + (size_t)key_lo * kD + (tid & 7) * 16;
+      const uint8_t *v_first = vbase + (size_t)key_lo * kD + (tid & 7) * 16;
+#pragma unroll
+      for (int it = 0; it < 4; ++it) {
+        const bool valid = 16 * it < rows_left;
+        cp_async16(ks + it * 2048, valid ? ld_k + goff + it * 2048 : k_first, valid);
+        cp_async16(vs + it * 2048, valid ? ld_v + goff + it * 2048 : v_first, valid);
+      }
     }
   };
 #pragma unroll
@@ -149,10 +194,17 @@ __global__ void __launch_bounds__(kDecThreads) decode8_attn_kernel(const Decode8
     }
     const int64_t slot = a.kind == BEAM_LOCAL ? t % a.window : t;
     if (row < kGroup) {
-      uint4 hv;
-      hv.x = pack_f16(x[0], x[1]); hv.y = pack_f16(x[2], x[3]);
-      hv.z = pack_f16(x[4], x[5]); hv.w = pack_f16(x[6], x[7]);
-      *reinterpret_cast<uint4 *>(q_prep + row * kD + l16 * 8) = hv;
+      const uint2 hi = f32x8_to_e4m3(x, kDec8QScale);
+      const uint32_t hw[4] = {hi.x & 0xFFFFu, hi.x >> 16, hi.y & 0xFFFFu, hi.y >> 16};
+      float r[8];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {   // residual 16 q - hi, exact in fp32
+        const uint32_t h2 = e4m3x2_to_f16x2(hw[e]);
+        r[2 * e] = fmaf(x[2 * e], kDec8QScale, -__half2float(__ushort_as_half(h2 & 0xFFFFu)));
+        r[2 * e + 1] = fmaf(x[2 * e + 1], kDec8QScale, -__half2float(__ushort_as_half(h2 >> 16)));
+      }
+      *reinterpret_cast<uint2 *>(q_hi + row * kD + l16 * 8) = hi;
+      *reinterpret_cast<uint2 *>(q_lo + row * kD + l16 * 8) = f32x8_to_e4m3(r, 1.0f);
     } else if (slot / a.split == s_idx) {
       const uint2 codes = f32x8_to_e4m3(x, row == kGroup ? A.inv_k_scale : A.inv_v_scale);
       uint8_t *cache = row == kGroup ? kbase : vbase;
@@ -168,27 +220,29 @@ __global__ void __launch_bounds__(kDecThreads) decode8_attn_kernel(const Decode8
     __syncthreads();  // the queries are in shared memory
   }
 
-  float factor = a.scale_log2 * A.k_scale;
+  float factor = a.scale_log2 * A.k_scale * (1.0f / kDec8QScale);
   if (a.kind == BEAM_GLOBAL) factor *= ssmax_factor(t + 1, a.ssmax_base, a.ssmax_exp);
 
-  // Query fragments (fp16): row h = lane/4 (< 6 valid); k-step ks holds d = 32c + 4ks + 0..3.
+  // Query fragments (E4M3 hi and lo terms): row h = lane/4 (< 6 valid); k-step ks holds
+  // d = 32c + 8ks + 0..3 (register a0) and + 4..7 (a2).
   const int c4 = lane & 3, h = lane >> 2;
-  uint32_t qa[8][2];
+  uint4 qh[2], ql[2];   // 32 bytes of the row at d = 32c: words 2ks, 2ks + 1 of k-step ks
   {
-    const __half *qrow = q_prep + (h < kGroup ? h : 0) * kD + c4 * 32;
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      const uint2 v = *reinterpret_cast<const uint2 *>(qrow + ks * 4);
-      qa[ks][0] = h < kGroup ? v.x : 0u;
-      qa[ks][1] = h < kGroup ? v.y : 0u;
-    }
+    const int hr = h < kGroup ? h : 0;
+    qh[0] = *reinterpret_cast<const uint4 *>(q_hi + hr * kD + c4 * 32);
+    qh[1] = *reinterpret_cast<const uint4 *>(q_hi + hr * kD + c4 * 32 + 16);
+    ql[0] = *reinterpret_cast<const uint4 *>(q_lo + hr * kD + c4 * 32);
+    ql[1] = *reinterpret_cast<const uint4 *>(q_lo + hr * kD + c4 * 32 + 16);
+    if (h >= kGroup) qh[0] = qh[1] = ql[0] = ql[1] = make_uint4(0u, 0u, 0u, 0u);
   }
+  const uint32_t qhw[8] = {qh[0].x, qh[0].y, qh[0].z, qh[0].w, qh[1].x, qh[1].y, qh[1].z, qh[1].w};
+  const uint32_t qlw[8] = {ql[0].x, ql[0].y, ql[0].z, ql[0].w, ql[1].x, ql[1].y, ql[1].z, ql[1].w};
 
   float m_run = -INFINITY;
   float l_run = 0.f;
-  float o[16][4];
+  float o[8][4];   // O^T tiles: rows d = 16 g + mt (c0, c1) and 16 g + 8 + mt (c2, c3)
 #pragma unroll
-  for (int nb = 0; nb < 16; ++nb) o[nb][0] = o[nb][1] = o[nb][2] = o[nb][3] = 0.f;
+  for (int mt = 0; mt < 8; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
 
   const bool any_patch = __syncthreads_or(patch_tile >= 0);
   for (int tile = 0; tile < n_tiles; ++tile) {
@@ -220,31 +274,40 @@ __global__ void __launch_bounds__(kDecThreads) decode8_attn_kernel(const Decode8
       const int r = wrow + nb * 8 + h;
       const uint4 k0 = *reinterpret_cast<const uint4 *>(ks + swz128(r, 2 * c4));
       const uint4 k1 = *reinterpret_cast<const uint4 *>(ks + swz128(r, 2 * c4 + 1));
-      const uint32_t kw8[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+      const uint32_t kw8[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};  // as codes
 #pragma unroll
-      for (int kstep = 0; kstep < 8; ++kstep) {
-        const uint32_t afr[4] = {qa[kstep][0], 0u, qa[kstep][1], 0u};
-        mma_f16_16816(s[nb], afr, e4m3x2_to_f16x2(kw8[kstep]), e4m3x2_to_f16x2(kw8[kstep] >> 16));
+      for (int ks = 0; ks < 4; ++ks) {
+        mma_e4m3_16832(s[nb], qhw[2 * ks], qhw[2 * ks + 1], kw8[2 * ks], kw8[2 * ks + 1]);
+        mma_e4m3_16832(s[nb], qlw[2 * ks], qlw[2 * ks + 1], kw8[2 * ks], kw8[2 * ks + 1]);
       }
     }
-    // scale, mask the ragged end, online softmax for head lane/4 (as in the BF16 kernel)
-    const int key0 = tile * kDec8Tile + wrow + c4 * 2;
+    // scale, mask the ragged end (last tile only), online softmax for head lane/4
     float mx = -INFINITY;
+    if ((tile + 1) * kDec8Tile > n_keys) {
+      const int key0 = tile * kDec8Tile + wrow + c4 * 2;
 #pragma unroll
-    for (int nb = 0; nb < 2; ++nb)
+      for (int nb = 0; nb < 2; ++nb)
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int kk = key0 + nb * 8 + e;
-        float v = s[nb][e] * factor;
-        v = kk < n_keys ? v : -INFINITY;
-        s[nb][e] = v;
-        mx = fmaxf(mx, v);
-      }
+        for (int e = 0; e < 2; ++e) {
+          const int kk = key0 + nb * 8 + e;
+          s[nb][e] = kk < n_keys ? s[nb][e] * factor : -INFINITY;
+          mx = fmaxf(mx, s[nb][e]);
+        }
+    } else {
+#pragma unroll
+      for (int nb = 0; nb < 2; ++nb)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          s[nb][e] *= factor;
+          mx = fmaxf(mx, s[nb][e]);
+        }
+    }
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
     const float m_new = fmaxf(m_run, mx);
     const float m_use = m_new == -INFINITY ? 0.f : m_new;
-    const float corr = exp2f(m_run - m_use);
+    const bool grew = m_new > m_run;
+    const float corr = ex2_approx(m_run - m_use);
     m_run = m_new;
     float p[2][2];
     float psum = 0.f;
@@ -252,15 +315,22 @@ __global__ void __launch_bounds__(kDecThreads) decode8_attn_kernel(const Decode8
     for (int nb = 0; nb < 2; ++nb)
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        p[nb][e] = exp2f(s[nb][e] - m_use);
+        p[nb][e] = ex2_approx(s[nb][e] - m_use);
         psum += p[nb][e];
       }
     l_run = l_run * corr + psum;
+    if (__any_sync(0xffffffffu, grew)) {  // O^T columns of heads 2c, 2c + 1: their corrections
+      const float corr0 = __shfl_sync(0xffffffffu, corr, (2 * c4) * 4);
+      const float corr1 = __shfl_sync(0xffffffffu, corr, (2 * c4 + 1) * 4);
 #pragma unroll
-    for (int nb = 0; nb < 16; ++nb) { o[nb][0] *= corr; o[nb][1] *= corr; }
+      for (int mt = 0; mt < 8; ++mt) {
+        o[mt][0] *= corr0; o[mt][1] *= corr1; o[mt][2] *= corr0; o[mt][3] *= corr1;
+      }
+    }
 
-    // O[head][d] += P[head][key] V[key][d]: keys wrow + 2c + {0,1} (+ 8), d = 16 (lane/4) + nb
-    const uint32_t pa[4] = {pack_f16(p[0][0], p[0][1]), 0u, pack_f16(p[1][0], p[1][1]), 0u};
+    // O^T[d][head] += V^T[d][key] P^T[key][head]: keys wrow + 2c + {0,1} (+ 8); the lane's
+    // rows are d = 16 g + mt and 16 g + 8 + mt (g = lane / 4)
+    const uint32_t pb0 = pack_f16(p[0][0], p[0][1]), pb1 = pack_f16(p[1][0], p[1][1]);
     const int r0 = wrow + c4 * 2;
     const uint4 va = *reinterpret_cast<const uint4 *>(vs + swz128(r0, h));
     const uint4 vb = *reinterpret_cast<const uint4 *>(vs + swz128(r0 + 1, h));
@@ -269,31 +339,46 @@ __global__ void __launch_bounds__(kDecThreads) decode8_attn_kernel(const Decode8
     const uint32_t wa[4] = {va.x, va.y, va.z, va.w}, wb[4] = {vb.x, vb.y, vb.z, vb.w};
     const uint32_t wc[4] = {vc.x, vc.y, vc.z, vc.w}, wd[4] = {vd.x, vd.y, vd.z, vd.w};
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      // byte j of each word is d = 16 (lane/4) + 4q + j: pair the two keys' bytes
-      const uint32_t lo01 = prmt(wa[q], wb[q], 0x5140u), lo23 = prmt(wa[q], wb[q], 0x7362u);
-      const uint32_t hi01 = prmt(wc[q], wd[q], 0x5140u), hi23 = prmt(wc[q], wd[q], 0x7362u);
-      mma_f16_16816(o[4 * q + 0], pa, e4m3x2_to_f16x2(lo01), e4m3x2_to_f16x2(hi01));
-      mma_f16_16816(o[4 * q + 1], pa, e4m3x2_to_f16x2(lo01 >> 16), e4m3x2_to_f16x2(hi01 >> 16));
-      mma_f16_16816(o[4 * q + 2], pa, e4m3x2_to_f16x2(lo23), e4m3x2_to_f16x2(hi23));
-      mma_f16_16816(o[4 * q + 3], pa, e4m3x2_to_f16x2(lo23 >> 16), e4m3x2_to_f16x2(hi23 >> 16));
+    for (int q = 0; q < 2; ++q) {
+      // byte j of word q is d = 16 g + 4q + j, of word q + 2 is d = 16 g + 8 + 4q + j:
+      // pair the bytes of keys (r0, r0 + 1) and (r0 + 8, r0 + 9), widen the pairs
+      uint32_t x01[4], y01[4], x23[4], y23[4];   // [j]: the pair at byte j
+      e4m3x4_to_f16x2x2(prmt(wa[q], wb[q], 0x5140u), x01[0], x01[1]);
+      e4m3x4_to_f16x2x2(prmt(wa[q], wb[q], 0x7362u), x01[2], x01[3]);
+      e4m3x4_to_f16x2x2(prmt(wa[q + 2], wb[q + 2], 0x5140u), y01[0], y01[1]);
+      e4m3x4_to_f16x2x2(prmt(wa[q + 2], wb[q + 2], 0x7362u), y01[2], y01[3]);
+      e4m3x4_to_f16x2x2(prmt(wc[q], wd[q], 0x5140u), x23[0], x23[1]);
+      e4m3x4_to_f16x2x2(prmt(wc[q], wd[q], 0x7362u), x23[2], x23[3]);
+      e4m3x4_to_f16x2x2(prmt(wc[q + 2], wd[q + 2], 0x5140u), y23[0], y23[1]);
+      e4m3x4_to_f16x2x2(prmt(wc[q + 2], wd[q + 2], 0x7362u), y23[2], y23[3]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t afr[4] = {x01[j], y01[j], x23[j], y23[j]};
+        mma_f16_16816(o[4 * q + j], afr, pb0, pb1);
+      }
     }
   }
   cp_async_wait<0>();
   __syncthreads();
 
-  // Merge the four warps (accumulator column n of n-block nb is d = 16 n + nb).
+  // Merge the four warps.
   float *sm_o = reinterpret_cast<float *>(smem);                 // [4 warps][6][128]
   float *sm_m = sm_o + 4 * kGroup * kD;                          // [4][6]
   float *sm_l = sm_m + 4 * kGroup;                               // [4][6]
   l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
   l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
-  if (h < kGroup) {
+  if (2 * c4 < kGroup) {   // heads 2c, 2c + 1 (lanes with c = 3 hold the padding columns)
+    float *o0 = sm_o + (warp * kGroup + 2 * c4) * kD + 16 * h;
+    float *o1 = o0 + kD;
 #pragma unroll
-    for (int nb = 0; nb < 16; ++nb) {
-      sm_o[(warp * kGroup + h) * kD + (c4 * 2) * 16 + nb] = o[nb][0];
-      sm_o[(warp * kGroup + h) * kD + (c4 * 2 + 1) * 16 + nb] = o[nb][1];
+    for (int mt = 0; mt < 8; ++mt) {
+      o0[mt] = o[mt][0];
+      o1[mt] = o[mt][1];
+      o0[8 + mt] = o[mt][2];
+      o1[8 + mt] = o[mt][3];
     }
+  }
+  if (h < kGroup) {
     if (c4 == 0) {
       sm_m[warp * kGroup + h] = m_run;
       sm_l[warp * kGroup + h] = l_run;

@@ -93,11 +93,6 @@ constexpr uint32_t kTmemHolder = kNumBars * 8;      // u32: tensor-memory base a
 constexpr uint32_t kAbortFlag = kTmemHolder + 4;    // u32: set when a wait ran out
 }  // namespace tcd
 
-__device__ __forceinline__ float ex2_approx(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
-  return y;
-}
 __device__ __forceinline__ float tanh_approx(float x) {
   float y;
   asm("tanh.approx.f32 %0, %1;\n" : "=f"(y) : "f"(x));
