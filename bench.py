@@ -382,7 +382,8 @@ def bench_prefill_chunk(torch, beam, steps, warmup, seed):
         vc = torch.empty_like(kc)
         wl.device_normal_bf16_(kc, seed, f"chunk/kc{kind}")
         wl.device_normal_bf16_(vc, seed, f"chunk/vc{kind}")
-        ws = torch.empty(max(16, beam.beam_prefill_chunk_workspace_bytes(kind, params, w.B, w.T)),
+        ws = torch.empty(max(16, beam.beam_prefill_chunk_workspace_bytes(kind, params, w.B, w.T,
+                                                                         layout)),
                          dtype=torch.uint8, device=dev)
 
         def call(kind=kind, layout=layout, kc=kc, vc=vc, ws=ws):

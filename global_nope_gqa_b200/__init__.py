@@ -79,7 +79,7 @@ def lib() -> ctypes.CDLL:
         L.beam_attn_prefill.argtypes = [ctypes.c_int, pp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp,
                                         vp, vp, lp, vp, sz, vp, vp]
         L.beam_prefill_chunk_workspace_bytes.restype = sz
-        L.beam_prefill_chunk_workspace_bytes.argtypes = [ctypes.c_int, pp, i32, i32]
+        L.beam_prefill_chunk_workspace_bytes.argtypes = [ctypes.c_int, pp, i32, i32, lp]
         L.beam_attn_prefill_chunk.restype = ctypes.c_int
         L.beam_attn_prefill_chunk.argtypes = [ctypes.c_int, pp, i32, i32, vp, vp, vp, vp, vp, vp, vp,
                                               vp, vp, vp, vp, lp, vp, sz, vp, vp]
@@ -179,8 +179,10 @@ def beam_attn_prefill(kind, params, q, k, v, gate, q_norm_w, k_norm_w, gate_bias
     return out
 
 
-def beam_prefill_chunk_workspace_bytes(kind: int, params: Params, B: int, T: int) -> int:
-    return lib().beam_prefill_chunk_workspace_bytes(kind, ctypes.byref(params), B, T)
+def beam_prefill_chunk_workspace_bytes(kind: int, params: Params, B: int, T: int,
+                                       layout: KVLayout | None = None) -> int:
+    return lib().beam_prefill_chunk_workspace_bytes(
+        kind, ctypes.byref(params), B, T, ctypes.byref(layout) if layout is not None else None)
 
 
 def beam_attn_prefill_chunk(kind, params, q, k, v, gate, q_norm_w, k_norm_w, gate_bias, pos0, out,
@@ -189,7 +191,7 @@ def beam_attn_prefill_chunk(kind, params, q, k, v, gate, q_norm_w, k_norm_w, gat
     """Chunked prefill: q, gate [B, T, 6144]; k, v [B, T, 1024] bf16; pos0 [B] int64 on the
     device (position of each sequence's first new token); caches as for decode."""
     B, T = q.shape[0], q.shape[1]
-    need = beam_prefill_chunk_workspace_bytes(kind, params, B, T)
+    need = beam_prefill_chunk_workspace_bytes(kind, params, B, T, layout)
     if workspace is None and need:
         workspace = _workspace(need, q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()

@@ -19,6 +19,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "decode8.cuh"
+#include "decode_multi.cuh"
 #include "prefill_tc.cuh"
 #include "prologue.cuh"
 
@@ -64,6 +65,10 @@ int device_info(DeviceInfo **out) {
     if ((st = cuda_status(cudaFuncSetAttribute(decode_attn_kernel<true>,
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem),
                           "decode shared-memory opt-in")))
+      return st;
+    if ((st = cuda_status(cudaFuncSetAttribute(decode_multi_kernel,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem),
+                          "multi-token decode shared-memory opt-in")))
       return st;
     if ((st = cuda_status(cudaFuncSetAttribute(decode8_attn_kernel<false>,
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, kDec8Smem),
@@ -357,13 +362,62 @@ int beam_attn_prefill(int kind, const beam_attn_params *p, int32_t B, int32_t T,
   return launch_prefill_attention(kind, p, B, T, tm_q, tm_k, tm_v, fa, dev, s);
 }
 
+}  // extern "C"
+
+namespace {
+
+// Split-K plan of a chunk of T <= 16 new tokens (decode_multi_kernel): key coordinates
+// covered per sequence (at most), run length per CTA and runs per sequence.
+struct MultiPlan {
+  int n_mt;            // m-tiles of two new tokens
+  int64_t range;       // largest number of key coordinates one sequence spans
+  int split;           // coordinates per CTA (multiple of the 64-row tile)
+  int n_split_max;
+};
+
+MultiPlan multi_plan(int kind, const beam_attn_params *p, int32_t B, int32_t T, int64_t slots,
+                     int sm_count) {
+  MultiPlan m;
+  m.n_mt = (T + kMultiTokPerTile - 1) / kMultiTokPerTile;
+  m.range = kind == BEAM_LOCAL ? (int64_t)p->window - 1 + T : slots;
+  // about three waves of two CTAs per SM, runs of at least 256 coordinates
+  const int64_t target = (int64_t)sm_count * 2 * 3;
+  int64_t split = 256;
+  while (split < (int64_t)1 << 20 &&
+         (int64_t)B * kHkv * m.n_mt * ((m.range + split - 1) / split) > target)
+    split *= 2;
+  m.split = (int)split;
+  m.n_split_max = (int)((m.range + split - 1) / split);
+  return m;
+}
+
+size_t multi_partial_bytes(int32_t B, const MultiPlan &m) {
+  const size_t parts = (size_t)B * kHkv * m.n_mt * m.n_split_max * 16;
+  return round_up(parts * kD * 4, 256) + round_up(parts * 2 * 4, 256);
+}
+
+}  // namespace
+
+extern "C" {
+
 size_t beam_prefill_chunk_workspace_bytes(int kind, const beam_attn_params *p, int32_t B,
-                                          int32_t T) {
+                                          int32_t T, const beam_kv_layout_t *layout) {
   if (!p || B <= 0 || T <= 0 || p->window < 1) return 0;
-  if (kind != BEAM_LOCAL) return 0;  // a global chunk reads and writes the cache itself
-  const size_t rows = (size_t)B * ((size_t)p->window - 1 + T);
-  // keys and values [B][window - 1 + T][8][128] bf16, then the RoPE table [B][T][128] fp32
-  return 2 * round_up(rows * kHkv * kD * 2, 256) + round_up((size_t)B * T * 128 * 4, 256);
+  size_t bytes = 0;
+  if (kind == BEAM_LOCAL) {
+    // keys and values [B][window - 1 + T][8][128] bf16 (the ring rows the chunk still sees,
+    // then the new rows), then the RoPE table [B][T][128] fp32
+    const size_t rows = (size_t)B * ((size_t)p->window - 1 + T);
+    bytes = 2 * round_up(rows * kHkv * kD * 2, 256) + round_up((size_t)B * T * 128 * 4, 256);
+  }
+  if (T <= kMultiMaxT) {  // split-K partials of the few-token path
+    DeviceInfo *dev = nullptr;
+    int sm = 148;
+    if (device_info(&dev) == BEAM_OK) sm = dev->sm_count;
+    const int64_t slots = layout ? layout->slots_per_seq : (int64_t)p->window;
+    bytes += multi_partial_bytes(B, multi_plan(kind, p, B, T, slots, sm));
+  }
+  return bytes;
 }
 
 int beam_attn_prefill_chunk(int kind, const beam_attn_params *p, int32_t B, int32_t T,
@@ -387,7 +441,7 @@ int beam_attn_prefill_chunk(int kind, const beam_attn_params *p, int32_t B, int3
   const bool local = kind == BEAM_LOCAL;
   if (!local && layout->slots_per_seq < T) return BEAM_ERR_CAPACITY;
   if (!local && layout->slots_per_seq > INT32_MAX - kTcBN) return BEAM_ERR_UNSUPPORTED;
-  const size_t need = beam_prefill_chunk_workspace_bytes(kind, p, B, T);
+  const size_t need = beam_prefill_chunk_workspace_bytes(kind, p, B, T, layout);
   if (need && (!workspace || workspace_bytes < need)) return BEAM_ERR_WORKSPACE;
   const int64_t ext_rows = local ? (int64_t)p->window - 1 + T : T;
   if ((int64_t)B * ext_rows > INT32_MAX) return BEAM_ERR_UNSUPPORTED;
@@ -420,7 +474,8 @@ int beam_attn_prefill_chunk(int kind, const beam_attn_params *p, int32_t B, int3
   ca.T = T;
   ca.window = p->window;
   ca.kind = kind;
-  const int64_t prep_ctas = (int64_t)B * (local ? prefix : kChunkPadRows);
+  // (the few-token path reads a global cache only up to pos0 + T: no padding needed)
+  const int64_t prep_ctas = local ? (int64_t)B * prefix : T <= kMultiMaxT ? 0 : (int64_t)B * kChunkPadRows;
   if (prep_ctas > 0) {
     chunk_prep_kernel<<<(unsigned)prep_ctas, 128, 0, s>>>(ca);
     if ((st = launch_status())) return st;
@@ -457,6 +512,67 @@ int beam_attn_prefill_chunk(int kind, const beam_attn_params *p, int32_t B, int3
   if ((st = launch_status())) return st;
 
   // 3. attention of the new rows over the earlier and the new keys
+  if (T <= kMultiMaxT) {
+    // a few new tokens (multi-token decode): split the keys across CTAs, then merge
+    const MultiPlan mp = multi_plan(kind, p, B, T, layout->slots_per_seq, dev->sm_count);
+    uint8_t *pw = static_cast<uint8_t *>(workspace) + (local ? 2 * ext_bytes +
+                                                       round_up((size_t)B * T * 128 * 4, 256)
+                                                             : 0);
+    const size_t parts = (size_t)B * kHkv * mp.n_mt * mp.n_split_max * 16;
+    MultiArgs ma;
+    memset(&ma, 0, sizeof ma);
+    ma.q_raw = static_cast<const uint16_t *>(q);
+    if (local) {
+      ma.key = k_ext;
+      ma.val = v_ext;
+      ma.stride_seq = ext_rows * kHkv * kD;
+      ma.stride_head = kD;
+      ma.stride_row = kHkv * kD;
+    } else {
+      ma.key = static_cast<const uint16_t *>(k_cache);
+      ma.val = static_cast<const uint16_t *>(v_cache);
+      ma.stride_seq = layout->stride_seq;
+      ma.stride_head = layout->stride_head;
+      ma.stride_row = layout->stride_slot;
+    }
+    ma.pos0 = pos0;
+    ma.qw = q_norm_w;
+    ma.eps = p->rms_eps;
+    ma.kind = kind;
+    ma.window = p->window;
+    ma.T = T;
+    ma.n_mt = mp.n_mt;
+    ma.prefix = prefix;
+    ma.slots = layout->slots_per_seq;
+    ma.split = mp.split;
+    ma.n_split_max = mp.n_split_max;
+    ma.scale_log2 = p->softmax_scale * kLog2e;
+    ma.ssmax_base = p->ssmax_base;
+    ma.ssmax_exp = p->ssmax_exp;
+    ma.part_o = reinterpret_cast<float *>(pw);
+    ma.part_ml = reinterpret_cast<float *>(pw + round_up(parts * kD * 4, 256));
+    fill_inv_freq(ma.inv_freq, p->rope_theta);
+    if (mp.n_split_max > 65535 || (int64_t)kHkv * mp.n_mt > 65535) return BEAM_ERR_UNSUPPORTED;
+    decode_multi_kernel<<<dim3(mp.n_split_max, kHkv * mp.n_mt, B), kDecThreads, kDecSmem, s>>>(ma);
+    if ((st = launch_status())) return st;
+    MultiCombineArgs mc;
+    mc.part_o = ma.part_o;
+    mc.part_ml = ma.part_ml;
+    mc.pos0 = pos0;
+    mc.gate = static_cast<const uint16_t *>(gate);
+    mc.gate_bias = gate_bias;
+    mc.out = static_cast<uint16_t *>(out);
+    mc.kind = kind;
+    mc.window = p->window;
+    mc.T = T;
+    mc.n_mt = mp.n_mt;
+    mc.prefix = prefix;
+    mc.split = mp.split;
+    mc.n_split_max = mp.n_split_max;
+    mc.slots = layout->slots_per_seq;
+    decode_multi_combine_kernel<<<dim3(kHq, T, B), kD, 0, s>>>(mc);
+    return launch_status();
+  }
   if ((st = encode_fn())) return st;
   CUtensorMap tm_q, tm_k, tm_v;
   if ((st = make_head_map(&tm_q, q, kHq, T, B))) return st;

@@ -166,10 +166,17 @@ def test_host_validation_rejects_before_launch(beam):
     assert L.beam_kv_append(1, P, 1, 0, A, A, A, A, A, A, ctypes.byref(glob), None, None) == 0
     # chunked prefill: the cache is required, pos0 is a device int64 array
     ring = beam.beam_kv_layout(beam.LOCAL, p, 1, 0)
-    cws = beam.beam_prefill_chunk_workspace_bytes(beam.LOCAL, p, 1, 16)
-    assert cws == 2 * (511 + 16) * 8 * 128 * 2 + 16 * 128 * 4   # earlier + new K/V rows, RoPE table
-    assert beam.beam_prefill_chunk_workspace_bytes(beam.GLOBAL, p, 1, 16) == 0
-    cargs = lambda **kw: [kw.get("kind", 0), P, kw.get("B", 1), kw.get("T", 16), A, A, A, A, A, A,
+    cws = beam.beam_prefill_chunk_workspace_bytes(beam.LOCAL, p, 1, 17, ring)
+    assert cws == 2 * (511 + 17) * 8 * 128 * 2 + 17 * 128 * 4   # earlier + new K/V rows, RoPE table
+    assert beam.beam_prefill_chunk_workspace_bytes(beam.GLOBAL, p, 1, 17, glob) == 0
+    # up to 16 new tokens: also the split-K partials, growing with the cache capacity
+    few = beam.beam_prefill_chunk_workspace_bytes(beam.LOCAL, p, 1, 16, ring)
+    assert few > 2 * (511 + 16) * 8 * 128 * 2 + 16 * 128 * 4
+    g1 = beam.beam_prefill_chunk_workspace_bytes(beam.GLOBAL, p, 1, 8, glob)
+    g2 = beam.beam_prefill_chunk_workspace_bytes(beam.GLOBAL, p, 1, 8,
+                                                 beam.beam_kv_layout(beam.GLOBAL, p, 1, 1 << 20))
+    assert 0 < g1 <= g2
+    cargs = lambda **kw: [kw.get("kind", 0), P, kw.get("B", 1), kw.get("T", 17), A, A, A, A, A, A,
                           A, kw.get("pos0", A), A, kw.get("kc", A), A,
                           kw.get("layout", ctypes.byref(ring)), kw.get("ws", A),
                           kw.get("ws_bytes", cws), None, None]
@@ -182,7 +189,7 @@ def test_host_validation_rejects_before_launch(beam):
     assert L.beam_attn_prefill_chunk(*cargs(ws=None)) == -6
     small = beam.beam_kv_layout(beam.GLOBAL, p, 1, 15)
     assert L.beam_attn_prefill_chunk(*cargs(kind=1, layout=ctypes.byref(small), ws=None,
-                                            ws_bytes=0)) == -5          # T = 16 > 15 slots
+                                            ws_bytes=0)) == -5          # T = 17 > 15 slots
     assert L.beam_attn_prefill_chunk(*cargs(kind=0, layout=ctypes.byref(small))) == -1
 
     # FP8 cache: one byte per element, rows on 16 bytes, positive finite scales

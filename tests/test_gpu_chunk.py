@@ -68,7 +68,7 @@ def check_cache(orc, ci, params, kc, vc, skip=()):
             d = np.abs(as_f64(kh[b, :, s]) - as_f64(kr))
             assert np.all(d <= np.abs(as_f64(kr)) * 2.0 ** -7 + K_ABS), (b, t)
             written[b, s] = True
-        if ci.kind == wl.GLOBAL:
+        if ci.kind == wl.GLOBAL and ci.T > 16:   # the tcgen05 path reads whole 128-key blocks
             end = p0 + ci.T
             padded[b, end:min(S, (end + 127) // 128 * 128)] = True
     keep = ~written
@@ -88,6 +88,14 @@ def check_cache(orc, ci, params, kc, vc, skip=()):
     (wl.GLOBAL, [5], 1, 512, 64),
     (wl.GLOBAL, [4000], 130, 512, 4200),          # padding stops at the capacity
     (wl.GLOBAL, [1, 128, 255], 128, 512, 640),
+    # up to 16 new tokens: the split-K multi-token decode path
+    (wl.LOCAL, [0, 100, 2000], 8, 512, 512),
+    (wl.LOCAL, [37, 5], 3, 100, 100),
+    (wl.LOCAL, [3], 16, 1, 1),
+    (wl.LOCAL, [510, 511, 520], 16, 512, 512),
+    (wl.GLOBAL, [0, 1000, 127], 16, 512, 2048),
+    (wl.GLOBAL, [0, 4090], 5, 512, 4096),
+    (wl.GLOBAL, [70000], 2, 512, 70002),
 ])
 def test_chunk_matches_oracle_and_appends(env, kind, pos0, T, window, slots):
     torch, beam, orc = env
@@ -137,6 +145,30 @@ def test_chunked_prefill_workload_sampled_rows(env, kind):
     assert_close(got, ref, f"chunked_prefill kind={kind}")
 
 
+def test_multi_token_decode_1m_context_sampled(env):
+    """Eight new tokens after 1,048,568 cached ones in a global layer (the
+    verification of an 8-token drafted block at 1M context): every output of the
+    first, fourth and last new token against the oracle; cache drawn on the device."""
+    torch, beam, orc = env
+    params = beam.default_params()
+    P = oracle_params(orc, params)
+    T, slots = 8, wl.MAX_CONTEXT
+    ci = wl.chunk_inputs(wl.GLOBAL, T, [slots - T], slots, 53, layer="m1m", with_cache=False)
+    layout = beam.beam_kv_layout(wl.GLOBAL, params, 1, slots)
+    kc = torch.empty(layout.bytes_k // 2, dtype=torch.bfloat16, device="cuda")
+    vc = torch.empty_like(kc)
+    wl.device_normal_bf16_(kc, 53, "m1m/kc")
+    wl.device_normal_bf16_(vc, 53, "m1m/vc")
+    ci.k_cache = host_bits(kc).reshape(1, 8, slots, 128)
+    ci.v_cache = host_bits(vc).reshape(1, 8, slots, 128)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, *_ = run_chunk(torch, beam, ci, params, status, kc=kc, vc=vc)
+    assert int(status.item()) == 0
+    ri = np.array([0, 3, T - 1])
+    ref = oracle_chunk(orc, beam, ci, params, (np.zeros_like(ri), ri))
+    assert_close(host_bits(out).reshape(1, T, 48, 128)[0, ri], ref, "multi-token decode 1M")
+
+
 @pytest.mark.parametrize("kind", [wl.GLOBAL, wl.LOCAL])
 def test_prefill_then_chunk_equals_one_shot(env, kind):
     """The GPU's own prefill fills the cache with the first T1 tokens, then one chunk
@@ -146,6 +178,11 @@ def test_prefill_then_chunk_equals_one_shot(env, kind):
     torch, beam, orc = env
     params = beam.default_params()
     T1, T2 = 700, 333
+    _prefill_then_chunk(torch, beam, orc, kind, params, T1, T2)
+    _prefill_then_chunk(torch, beam, orc, kind, params, 1000, 9)   # the few-token path
+
+
+def _prefill_then_chunk(torch, beam, orc, kind, params, T1, T2):
     full = wl.prefill_inputs(1, T1 + T2, 51, layer=f"two{kind}")
     layout = beam.beam_kv_layout(kind, params, 1, T1 + T2)
     kc = torch.zeros(layout.bytes_k // 2, dtype=torch.bfloat16, device="cuda")
