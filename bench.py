@@ -4,10 +4,11 @@ One step = the prefill of one local and one global attention layer of the
 batched-prefill workload (4 sequences x 8192 tokens, 48 query / 8 KV heads,
 head_dim 128), including the fused KV-cache append, through the C ABI.  The
 headline value is algorithmic TFLOP/s (visible (query, key) pairs x 4 x 128 x 48).
-Three more measurements ride along on the same line: the 1M-context decode step
-across the 52-layer schedule (KV-read GB/s, tokens/s), the batched decode step
-(64 sequences, contexts in [1024, 32768]) and the chunked prefill (8192 new tokens
-after 57,344 cached ones, one local and one global layer; TFLOP/s).
+More measurements ride along on the same line: the 1M-context decode step across the
+52-layer schedule over BF16 and over FP8 caches (KV-read GB/s, tokens/s), the
+52-layer step verifying 8 new tokens at 1M context, the batched decode step (64
+sequences, contexts in [1024, 32768]) and the chunked prefill (8192 new tokens after
+57,344 cached ones, one local and one global layer; TFLOP/s).
 
 Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl beam|reference]
 N > 1 runs under torch.distributed.run, one process per GPU; every rank processes
@@ -334,6 +335,83 @@ def bench_decode_1m(torch, beam, steps, warmup, seed, fp8=False):
     return res, glob_bytes
 
 
+class ChunkLayer:
+    """One chunk call (T new tokens after pos0 cached ones, B = 1) with its own caches."""
+
+    def __init__(self, torch, beam, kind, T, pos0, slots, seed, tag):
+        self.beam, self.kind = beam, kind
+        self.params = beam.default_params()
+        dev = "cuda"
+        ci = wl.chunk_inputs(kind, T, [pos0], slots, seed, layer=tag, with_cache=False)
+
+        def d(bits):
+            return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+        self.q, self.k, self.v, self.gate = d(ci.q), d(ci.k), d(ci.v), d(ci.gate)
+        self.qw = torch.from_numpy(ci.q_norm_w).to(dev)
+        self.kw = torch.from_numpy(ci.k_norm_w).to(dev)
+        self.bias = torch.from_numpy(ci.gate_bias).to(dev)
+        self.pos0 = torch.from_numpy(ci.pos0).to(dev)
+        self.layout = beam.beam_kv_layout(kind, self.params, 1, slots)
+        self.kc = torch.empty(self.layout.bytes_k // 2, dtype=torch.bfloat16, device=dev)
+        self.vc = torch.empty_like(self.kc)
+        wl.device_normal_bf16_(self.kc, seed, f"{tag}/kc")
+        wl.device_normal_bf16_(self.vc, seed, f"{tag}/vc")
+        self.out = torch.empty_like(self.q)
+        self.ws = torch.empty(max(16, beam.beam_prefill_chunk_workspace_bytes(
+            kind, self.params, 1, T, self.layout)), dtype=torch.uint8, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        vis = wl.chunk_visible_pairs(T, pos0, wl.WINDOW if kind == wl.LOCAL else None)
+        self.flops = vis * HEAD_FLOPS_PER_PAIR
+        ctx = [pos0 + T]
+        self.bytes = decode_kv_bytes(ctx, kind) + (T - 1) * 2 * 2 * (3 * 6144 + 2 * 1024)
+        # local: ring copy + prologue + split-K + combine; global: prologue + split-K + combine
+        self.launches_per_call = 4 if kind == wl.LOCAL else 3
+
+    def run(self):
+        self.beam.beam_attn_prefill_chunk(self.kind, self.params, self.q, self.k, self.v, self.gate,
+                                          self.qw, self.kw, self.bias, self.pos0, self.out,
+                                          self.kc, self.vc, self.layout, workspace=self.ws,
+                                          dev_status=self.status)
+
+
+def bench_decode_multi_1m(torch, beam, steps, warmup, seed, T=8):
+    """52-layer step verifying T = 8 drafted tokens at context 1,048,576 (the last T positions
+    of the 1M window): every layer is one chunk call of T new tokens; one CUDA graph."""
+    pos0 = wl.MAX_CONTEXT - T
+    layers = []
+    for i in range(1, wl.N_LAYERS + 1):
+        kind = wl.layer_kind(i)
+        slots = wl.MAX_CONTEXT if kind == wl.GLOBAL else wl.WINDOW
+        layers.append(ChunkLayer(torch, beam, kind, T, pos0, slots, seed, f"dm/L{i}"))
+
+    def step():
+        for L in layers:
+            L.run()
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        step()
+    torch.cuda.current_stream().wait_stream(stream)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    sec = time_loop(torch, graph.replay, steps, warmup)
+    assert all(int(L.status.item()) == 0 for L in layers)
+    total_bytes = sum(L.bytes for L in layers)
+    res = {
+        "workload": f"decode_multi_1m: B=1, {T} new tokens per step after {pos0} cached, 52 layers "
+                    "(9 global 4 GiB caches, 43 x 512-slot rings)",
+        "ms_per_step": sec * 1e3,
+        "tokens_per_s": T / sec,
+        "kv_read_GBps": total_bytes / sec / 1e9,
+        "gpu_launches_per_step": sum(L.launches_per_call for L in layers),
+    }
+    del graph, layers
+    torch.cuda.empty_cache()
+    return res
+
+
 def bench_decode_batched(torch, beam, steps, warmup, seed):
     w = wl.workload("batched_decode", seed)
     g = DecodeLayer(torch, beam, wl.GLOBAL, w.ctx, w.extra["global_slots"], seed, "bdec/g")
@@ -582,6 +660,9 @@ def run_gpu(args):
         d8, _ = bench_decode_1m(torch, beam, args.steps, args.warmup, args.seed, fp8=True)
         d8["pct_of_hbm"] = round(100 * d8["kv_read_GBps"] / pk["hbm_gbs"], 2)
         result["decode_1m_fp8"] = d8
+        dm = bench_decode_multi_1m(torch, beam, args.steps, args.warmup, args.seed)
+        dm["pct_of_hbm"] = round(100 * dm["kv_read_GBps"] / pk["hbm_gbs"], 2)
+        result["decode_multi_1m"] = dm
         pc = bench_prefill_chunk(torch, beam, args.steps, args.warmup, args.seed)
         pc["pct_of_bf16_peak"] = round(100 * pc["tflops"] / pk["bf16_tflops"], 2)
         result["prefill_chunk"] = pc

@@ -380,14 +380,15 @@ MultiPlan multi_plan(int kind, const beam_attn_params *p, int32_t B, int32_t T, 
   MultiPlan m;
   m.n_mt = (T + kMultiTokPerTile - 1) / kMultiTokPerTile;
   m.range = kind == BEAM_LOCAL ? (int64_t)p->window - 1 + T : slots;
-  // about three waves of two CTAs per SM, runs of at least 256 coordinates
+  // about three waves of two CTAs per SM: runs of a multiple of the 64-row tile, at least
+  // 256 coordinates
   const int64_t target = (int64_t)sm_count * 2 * 3;
-  int64_t split = 256;
-  while (split < (int64_t)1 << 20 &&
-         (int64_t)B * kHkv * m.n_mt * ((m.range + split - 1) / split) > target)
-    split *= 2;
-  m.split = (int)split;
-  m.n_split_max = (int)((m.range + split - 1) / split);
+  const int64_t per_run = (int64_t)B * kHkv * m.n_mt;
+  const int64_t runs = std::max<int64_t>(1, target / per_run);
+  const int64_t split = std::max<int64_t>(256, round_up((size_t)((m.range + runs - 1) / runs),
+                                                        kDecTile));
+  m.split = (int)std::min<int64_t>(split, INT32_MAX / 2);
+  m.n_split_max = (int)((m.range + m.split - 1) / m.split);
   return m;
 }
 
@@ -552,8 +553,8 @@ int beam_attn_prefill_chunk(int kind, const beam_attn_params *p, int32_t B, int3
     ma.part_o = reinterpret_cast<float *>(pw);
     ma.part_ml = reinterpret_cast<float *>(pw + round_up(parts * kD * 4, 256));
     fill_inv_freq(ma.inv_freq, p->rope_theta);
-    if (mp.n_split_max > 65535 || (int64_t)kHkv * mp.n_mt > 65535) return BEAM_ERR_UNSUPPORTED;
-    decode_multi_kernel<<<dim3(mp.n_split_max, kHkv * mp.n_mt, B), kDecThreads, kDecSmem, s>>>(ma);
+    if ((int64_t)mp.n_split_max * mp.n_mt > INT32_MAX || B > 65535) return BEAM_ERR_UNSUPPORTED;
+    decode_multi_kernel<<<dim3(mp.n_split_max * mp.n_mt, kHkv, B), kDecThreads, kDecSmem, s>>>(ma);
     if ((st = launch_status())) return st;
     MultiCombineArgs mc;
     mc.part_o = ma.part_o;

@@ -15,7 +15,9 @@
 // key is at kq + i and it sees c in [max(kq + i - window + 1, kmin), kq + i] (local) or
 // [0, kq + i] (global), as in the chunk kernel.
 //
-// Grid (split, KV head * m-tile, sequence), 128 threads.  M-tile mt holds new tokens 2 mt and
+// Grid (m-tile + n_mt * split, KV head, sequence), 128 threads: the m-tiles of one run of keys
+// are neighbours in launch order, so they stream the same tiles at the same time and all but
+// the first read them from L2.  M-tile mt holds new tokens 2 mt and
 // 2 mt + 1: MMA rows 6 j + h for token 2 mt + j and head h of the group (rows 12..15 are
 // padding).  The CTA prepares those rows (RMSNorm, RoPE at the token's position for a local
 // layer; a(t+1) joins the row's score scale), streams its run of key coordinates through a
@@ -74,7 +76,7 @@ __device__ __forceinline__ bool multi_range(const MultiArgs &a, int b, int64_t &
 __global__ void __launch_bounds__(kDecThreads) decode_multi_kernel(const MultiArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ __align__(16) uint16_t q_prep[16 * kD];
-  const int s_idx = blockIdx.x, g = blockIdx.y / a.n_mt, mt = blockIdx.y - g * a.n_mt;
+  const int s_idx = blockIdx.x / a.n_mt, mt = blockIdx.x - s_idx * a.n_mt, g = blockIdx.y;
   const int b = blockIdx.z;
   int64_t kq, lo_all, hi_all;
   if (!multi_range(a, b, kq, lo_all, hi_all)) return;
