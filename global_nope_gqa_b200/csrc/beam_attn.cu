@@ -224,6 +224,7 @@ int decode_split(int kind, const beam_attn_params *p, int32_t B, int64_t slots, 
   int64_t split = 512;
   while (split < 16384 && (int64_t)B * kHkv * ((slots + split - 1) / split) > target_ctas)
     split *= 2;
+  while ((slots + split - 1) / split > kCombineMaxSplits) split *= 2;  // the combine's limit
   return (int)split;
 }
 
@@ -764,7 +765,7 @@ int decode_call(int kind, const beam_attn_params *p, int32_t B, const void *q, c
   ca.split = split;
   ca.n_split_max = n_split_max;
   ca.slots = layout->slots_per_seq;
-  decode_combine_kernel<<<dim3(kHq, B), 256, 0, s>>>(ca);
+  decode_combine_kernel<<<dim3(kHq, B), kD, 0, s>>>(ca);
   return launch_status();
 }
 

@@ -69,8 +69,8 @@ __device__ __forceinline__ int64_t decode_visible(const DecodeArgs &a, int64_t t
 // kCluster = false (global cache): one split of the keys, partials to the workspace,
 // merged by decode_combine_kernel.  kCluster = true (local ring): the whole step in one
 // launch -- the splits of a (sequence, KV head) form one thread-block cluster (gridDim.x
-// CTAs, at most 4 of 128+ ring slots each), and rank 0 merges the CTAs' partials through
-// distributed shared memory and writes Y = O/l * sigmoid(G + b).
+// CTAs, at most 4 of 128+ ring slots each), and each rank merges its quarter of the outputs
+// across the CTAs' partials through distributed shared memory and writes Y = O/l * sigmoid(G + b).
 template <bool kCluster>
 __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const DecodeArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -118,15 +118,21 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const DecodeAr
 
   int patch_tile = -1, patch_row = 0;  // prefetched tile and row of the new slot
   uint4 patch_val = make_uint4(0u, 0u, 0u, 0u);
-  float gate6[kGroup];                 // cluster rank 0: gate logits + bias of its outputs
+  // cluster: rank r gates outputs [r, r + 1) * 768 / n of the group (idx = 128 hh + d):
+  // this thread's are idx0 + 128 k.  The first two gate values are fetched now (all a rank
+  // of a 3- or 4-CTA cluster needs), any others at the merge.
+  const int merge_n = kGroup * kD / gridDim.x, idx0 = s_idx * merge_n + tid;
+  auto gate_at = [&](int idx) {
+    const int h = g * kGroup + idx / kD;
+    return __uint_as_float((uint32_t)a.gate[((size_t)b * kHq + h) * kD + idx % kD] << 16) +
+           a.gate_bias[h];
+  };
+  float gate_k[2] = {0.f, 0.f};
   {
-    if (kCluster && s_idx == 0) {
+    if (kCluster) {
 #pragma unroll
-      for (int i = 0; i < kGroup; ++i) {
-        const int h = g * kGroup + i;
-        gate6[i] = __uint_as_float((uint32_t)a.gate[((size_t)b * kHq + h) * kD + tid] << 16) +
-                   a.gate_bias[h];
-      }
+      for (int k = 0; k < 2; ++k)
+        if (k * kDecThreads + tid < merge_n) gate_k[k] = gate_at(idx0 + k * kDecThreads);
     }
     // rows: 6 queries, the new key, the new value; a half-warp per row
     const int half = lane >> 4, l16 = lane & 15, row = warp * 2 + half;
@@ -153,9 +159,10 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const DecodeAr
         patch_tile = rel / kDecTile;
         patch_row = rel % kDecTile;
         patch_val = res;
+      } else {
+        __threadfence();  // a later tile streams this row (cp.async.cg reads L2)
       }
     }
-    __threadfence();  // the new row reaches L2 before the later tiles stream it (cp.async.cg)
     __syncthreads();  // the queries are in shared memory
   }
 
@@ -321,31 +328,37 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const DecodeAr
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
     cluster.sync();
-    if (cluster.block_rank() == 0) {
+    {  // rank r merges its share of the outputs across the ranks and gates them
       float *cl = reinterpret_cast<float *>(smem + 16384);
       const int n_rank = (int)cluster.num_blocks();
-      for (int idx = tid; idx < kGroup * kD; idx += kDecThreads) {
-        const int hh = idx / kD;
-        float M = -INFINITY;
-        for (int r = 0; r < n_rank; ++r)
-          M = fmaxf(M, cluster.map_shared_rank(cl, r)[kGroup * kD + hh]);
+      const float *rc[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) rc[r] = cluster.map_shared_rank(cl, r < n_rank ? r : 0);
+      for (int k = 0; k < kGroup; ++k) {
+        if (k * kDecThreads + tid >= merge_n) break;
+        const int idx = idx0 + k * kDecThreads, hh = idx / kD;
+        float m[4], M = -INFINITY;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          m[r] = r < n_rank ? rc[r][kGroup * kD + hh] : -INFINITY;
+          M = fmaxf(M, m[r]);
+        }
         const float Mu = M == -INFINITY ? 0.f : M;
         float acc = 0.f, L = 0.f;
-        for (int r = 0; r < n_rank; ++r) {
-          const float *rc = cluster.map_shared_rank(cl, r);
-          const float sc = exp2f(rc[kGroup * kD + hh] - Mu);
-          acc += sc * rc[idx];
-          L += sc * rc[kGroup * kD + kGroup + hh];
-        }
-        const int h = g * kGroup + hh;
-        const size_t o = ((size_t)b * kHq + h) * kD + (idx - hh * kD);
-        float gl = gate6[0];  // idx = tid + 128 * hh: this thread's d is tid for every head
 #pragma unroll
-        for (int i = 1; i < kGroup; ++i) gl = hh == i ? gate6[i] : gl;
+        for (int r = 0; r < 4; ++r) {
+          if (r < n_rank) {
+            const float sc = ex2_approx(m[r] - Mu);
+            acc += sc * rc[r][idx];
+            L += sc * rc[r][kGroup * kD + kGroup + hh];
+          }
+        }
+        const float gl = k == 0 ? gate_k[0] : k == 1 ? gate_k[1] : gate_at(idx);
+        const size_t o = ((size_t)b * kHq + g * kGroup + hh) * kD + (idx - hh * kD);
         a.out[o] = (uint16_t)(pack_bf16(acc / L / (1.0f + expf(-gl)), 0.f) & 0xFFFFu);
       }
     }
-    cluster.sync();  // the other CTAs' shared memory stays alive until rank 0 is done
+    cluster.sync();  // every CTA's shared memory stays alive until all ranks have read it
   }
 }
 
@@ -360,8 +373,12 @@ struct CombineArgs {
   int64_t slots;
 };
 
-// 256 threads: warp w merges splits w, w+8, ...; lane l owns d = 4l .. 4l+3.
-__global__ void __launch_bounds__(256) decode_combine_kernel(const CombineArgs a) {
+// One CTA of 128 threads per (query head, sequence).  The split weights are formed once in
+// shared memory (2^(m_s - M), with every split's m read in parallel), then thread d sums
+// w_s o_s[d] over the splits: independent, coalesced loads, so the merge costs a few memory
+// latencies rather than one per split.  Y = O / l * sigmoid(G + b_h).
+constexpr int kCombineMaxSplits = 1024;
+__global__ void __launch_bounds__(kD) decode_combine_kernel(const CombineArgs a) {
   const int h = blockIdx.x, b = blockIdx.y;
   const int g = h / kGroup, hh = h - g * kGroup;
   const int64_t t = a.pos[b];
@@ -370,54 +387,48 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const CombineArgs a
   else if (a.kind == BEAM_LOCAL) n_vis = t + 1 < a.window ? t + 1 : a.window;
   else n_vis = t < a.slots ? t + 1 : 0;
   if (n_vis == 0) return;  // invalid position: output untouched, status set upstream
-  const int n_split = (int)((n_vis + a.split - 1) / a.split);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  __shared__ float sm_o[8][kD];
-  __shared__ float sm_m[8], sm_l[8];
-  float M = -INFINITY, L = 0.f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  const int n_split = (int)min((n_vis + a.split - 1) / a.split, (int64_t)kCombineMaxSplits);
+  __shared__ float sm_w[kCombineMaxSplits];
+  __shared__ float sm_red[kD / 32];
+  const int d = threadIdx.x, lane = d & 31, warp = d >> 5;
   const size_t base = ((size_t)b * kHkv + g) * a.n_split_max;
-  for (int s = warp; s < n_split; s += 8) {
-    const size_t part = base + s;
-    const float m = a.part_ml[(part * kGroup + hh) * 2 + 0];
-    const float l = a.part_ml[(part * kGroup + hh) * 2 + 1];
-    const float4 v = reinterpret_cast<const float4 *>(a.part_o + (part * kGroup + hh) * kD)[lane];
-    const float Mn = fmaxf(M, m);
-    const float Mu = Mn == -INFINITY ? 0.f : Mn;
-    const float c0 = exp2f(M - Mu), c1 = exp2f(m - Mu);
-    acc.x = acc.x * c0 + v.x * c1; acc.y = acc.y * c0 + v.y * c1;
-    acc.z = acc.z * c0 + v.z * c1; acc.w = acc.w * c0 + v.w * c1;
-    L = L * c0 + l * c1;
-    M = Mn;
+  // M = max_s m_s
+  float mx = -INFINITY;
+  for (int s = d; s < n_split; s += kD) {
+    const float m = a.part_ml[((base + s) * kGroup + hh) * 2];
+    sm_w[s] = m;
+    mx = fmaxf(mx, m);
   }
-  reinterpret_cast<float4 *>(sm_o[warp])[lane] = acc;
-  if (lane == 0) { sm_m[warp] = M; sm_l[warp] = L; }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  if (lane == 0) sm_red[warp] = mx;
   __syncthreads();
-  if (warp == 0) {
-    float Mt = -INFINITY;
+  float M = sm_red[0];
 #pragma unroll
-    for (int w = 0; w < 8; ++w) Mt = fmaxf(Mt, sm_m[w]);
-    const float Mu = Mt == -INFINITY ? 0.f : Mt;
-    float Lt = 0.f, r[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int w = 0; w < 8; ++w) {
-      const float c = exp2f(sm_m[w] - Mu);
-      Lt += c * sm_l[w];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) r[e] += c * sm_o[w][lane * 4 + e];
-    }
-    const float inv = 1.0f / Lt;
-    const float bias = a.gate_bias[h];
-    const uint2 graw = reinterpret_cast<const uint2 *>(a.gate + ((size_t)b * kHq + h) * kD)[lane];
-    const float gl[4] = {bf16_lo(graw.x), bf16_hi(graw.x), bf16_lo(graw.y), bf16_hi(graw.y)};
-    float y[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) y[e] = r[e] * inv * (1.0f / (1.0f + expf(-(gl[e] + bias))));
-    uint2 packed;
-    packed.x = pack_bf16(y[0], y[1]);
-    packed.y = pack_bf16(y[2], y[3]);
-    reinterpret_cast<uint2 *>(a.out + ((size_t)b * kHq + h) * kD)[lane] = packed;
+  for (int w = 1; w < kD / 32; ++w) M = fmaxf(M, sm_red[w]);
+  const float Mu = M == -INFINITY ? 0.f : M;
+  __syncthreads();
+  // weights and L = sum_s w_s l_s
+  float lsum = 0.f;
+  for (int s = d; s < n_split; s += kD) {
+    const float w = ex2_approx(sm_w[s] - Mu);
+    sm_w[s] = w;
+    lsum += w * a.part_ml[((base + s) * kGroup + hh) * 2 + 1];
   }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
+  if (lane == 0) sm_red[warp] = lsum;
+  __syncthreads();
+  float L = 0.f;
+#pragma unroll
+  for (int w = 0; w < kD / 32; ++w) L += sm_red[w];
+  float acc = 0.f;
+  const float *po = a.part_o + (base * kGroup + hh) * kD + d;
+#pragma unroll 4
+  for (int s = 0; s < n_split; ++s) acc += sm_w[s] * po[(size_t)s * kGroup * kD];
+  const size_t oi = ((size_t)b * kHq + h) * kD + d;
+  const float gl = bf16_lo(a.gate[oi]) + a.gate_bias[h];
+  a.out[oi] = (uint16_t)(pack_bf16(acc / L / (1.0f + expf(-gl)), 0.f) & 0xFFFFu);
 }
 
 }  // namespace beam

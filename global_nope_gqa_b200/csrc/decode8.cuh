@@ -100,7 +100,8 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
 
 // kCluster = false (global cache): partials to the workspace, merged by
 // decode_combine_kernel.  kCluster = true (local ring): the splits of a (sequence, KV
-// head) form one cluster; rank 0 merges through distributed shared memory and gates.
+// head) form one cluster; the ranks merge their shares of the outputs through
+// distributed shared memory and gate them.
 template <bool kCluster>
 __global__ void __launch_bounds__(kDecThreads) decode8_attn_kernel(const Decode8Args A) {
   const DecodeArgs &a = A.base;
@@ -163,15 +164,21 @@ __global__ void __launch_bounds__(kDecThreads) decode8_attn_kernel(const Decode8
 
   int patch_tile = -1, patch_row = 0;  // prefetched tile and row of the new slot
   uint2 patch_val = make_uint2(0u, 0u);
-  float gate6[kGroup];
+  // cluster: rank r gates outputs [r, r + 1) * 768 / n of the group (idx = 128 hh + d):
+  // this thread's are idx0 + 128 k.  The first two gate values are fetched now (all a rank
+  // of a 3- or 4-CTA cluster needs), any others at the merge.
+  const int merge_n = kGroup * kD / gridDim.x, idx0 = s_idx * merge_n + tid;
+  auto gate_at = [&](int idx) {
+    const int h = g * kGroup + idx / kD;
+    return __uint_as_float((uint32_t)a.gate[((size_t)b * kHq + h) * kD + idx % kD] << 16) +
+           a.gate_bias[h];
+  };
+  float gate_k[2] = {0.f, 0.f};
   {
-    if (kCluster && s_idx == 0) {
+    if (kCluster) {
 #pragma unroll
-      for (int i = 0; i < kGroup; ++i) {
-        const int h = g * kGroup + i;
-        gate6[i] = __uint_as_float((uint32_t)a.gate[((size_t)b * kHq + h) * kD + tid] << 16) +
-                   a.gate_bias[h];
-      }
+      for (int k = 0; k < 2; ++k)
+        if (k * kDecThreads + tid < merge_n) gate_k[k] = gate_at(idx0 + k * kDecThreads);
     }
     // rows: 6 queries, the new key, the new value; a half-warp per row
     const int half = lane >> 4, l16 = lane & 15, row = warp * 2 + half;
@@ -214,9 +221,10 @@ __global__ void __launch_bounds__(kDecThreads) decode8_attn_kernel(const Decode8
         patch_tile = rel / kDec8Tile;
         patch_row = rel % kDec8Tile;
         patch_val = codes;
+      } else {
+        __threadfence();  // a later tile streams this row (cp.async.cg reads L2)
       }
     }
-    __threadfence();  // the new row reaches L2 before the later tiles stream it (cp.async.cg)
     __syncthreads();  // the queries are in shared memory
   }
 
@@ -419,31 +427,37 @@ __global__ void __launch_bounds__(kDecThreads) decode8_attn_kernel(const Decode8
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
     cluster.sync();
-    if (cluster.block_rank() == 0) {
+    {  // rank r merges its share of the outputs across the ranks and gates them
       float *cl = reinterpret_cast<float *>(smem + 16384);
       const int n_rank = (int)cluster.num_blocks();
-      for (int idx = tid; idx < kGroup * kD; idx += kDecThreads) {
-        const int hh = idx / kD;
-        float M = -INFINITY;
-        for (int r = 0; r < n_rank; ++r)
-          M = fmaxf(M, cluster.map_shared_rank(cl, r)[kGroup * kD + hh]);
+      const float *rc[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) rc[r] = cluster.map_shared_rank(cl, r < n_rank ? r : 0);
+      for (int k = 0; k < kGroup; ++k) {
+        if (k * kDecThreads + tid >= merge_n) break;
+        const int idx = idx0 + k * kDecThreads, hh = idx / kD;
+        float m[4], M = -INFINITY;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          m[r] = r < n_rank ? rc[r][kGroup * kD + hh] : -INFINITY;
+          M = fmaxf(M, m[r]);
+        }
         const float Mu = M == -INFINITY ? 0.f : M;
         float acc = 0.f, L = 0.f;
-        for (int r = 0; r < n_rank; ++r) {
-          const float *rc = cluster.map_shared_rank(cl, r);
-          const float sc = exp2f(rc[kGroup * kD + hh] - Mu);
-          acc += sc * rc[idx];
-          L += sc * rc[kGroup * kD + kGroup + hh];
-        }
-        const int hq = g * kGroup + hh;
-        const size_t oi = ((size_t)b * kHq + hq) * kD + (idx - hh * kD);
-        float gl = gate6[0];  // idx = tid + 128 * hh: this thread's d is tid for every head
 #pragma unroll
-        for (int i = 1; i < kGroup; ++i) gl = hh == i ? gate6[i] : gl;
-        a.out[oi] = (uint16_t)(pack_bf16(acc / L / (1.0f + expf(-gl)), 0.f) & 0xFFFFu);
+        for (int r = 0; r < 4; ++r) {
+          if (r < n_rank) {
+            const float sc = ex2_approx(m[r] - Mu);
+            acc += sc * rc[r][idx];
+            L += sc * rc[r][kGroup * kD + kGroup + hh];
+          }
+        }
+        const float gl = k == 0 ? gate_k[0] : k == 1 ? gate_k[1] : gate_at(idx);
+        const size_t o = ((size_t)b * kHq + g * kGroup + hh) * kD + (idx - hh * kD);
+        a.out[o] = (uint16_t)(pack_bf16(acc / L / (1.0f + expf(-gl)), 0.f) & 0xFFFFu);
       }
     }
-    cluster.sync();
+    cluster.sync();  // every CTA's shared memory stays alive until all ranks have read it
   }
 }
 
