@@ -20,6 +20,7 @@
 #include "decode.cuh"
 #include "decode8.cuh"
 #include "decode_multi.cuh"
+#include "decode_tc.cuh"
 #include "prefill_tc.cuh"
 #include "prologue.cuh"
 
@@ -66,8 +67,9 @@ int device_info(DeviceInfo **out) {
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem),
                           "decode shared-memory opt-in")))
       return st;
-    if ((st = cuda_status(cudaFuncSetAttribute(decode_multi_kernel,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem),
+    if ((st = cuda_status(cudaFuncSetAttribute(decode_tc_kernel,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               kDtSmemBytes),
                           "multi-token decode shared-memory opt-in")))
       return st;
     if ((st = cuda_status(cudaFuncSetAttribute(decode8_attn_kernel<false>,
@@ -367,7 +369,7 @@ int beam_attn_prefill(int kind, const beam_attn_params *p, int32_t B, int32_t T,
 
 namespace {
 
-// Split-K plan of a chunk of T <= 16 new tokens (decode_multi_kernel): key coordinates
+// Split-K plan of a chunk of T <= 16 new tokens (decode_tc_kernel): key coordinates
 // covered per sequence (at most), run length per CTA and runs per sequence.
 struct MultiPlan {
   int n_mt;            // m-tiles of two new tokens
@@ -381,13 +383,13 @@ MultiPlan multi_plan(int kind, const beam_attn_params *p, int32_t B, int32_t T, 
   MultiPlan m;
   m.n_mt = (T + kMultiTokPerTile - 1) / kMultiTokPerTile;
   m.range = kind == BEAM_LOCAL ? (int64_t)p->window - 1 + T : slots;
-  // about three waves of two CTAs per SM: runs of a multiple of the 64-row tile, at least
-  // 256 coordinates
-  const int64_t target = (int64_t)sm_count * 2 * 3;
-  const int64_t per_run = (int64_t)B * kHkv * m.n_mt;
+  // one CTA per SM fits (197 KB of shared memory): about two waves, runs of whole
+  // 128-key tiles
+  const int64_t target = (int64_t)sm_count * 2;
+  const int64_t per_run = (int64_t)B * kHkv;
   const int64_t runs = std::max<int64_t>(1, target / per_run);
-  const int64_t split = std::max<int64_t>(256, round_up((size_t)((m.range + runs - 1) / runs),
-                                                        kDecTile));
+  const int64_t split = std::max<int64_t>(kTcBN, round_up((size_t)((m.range + runs - 1) / runs),
+                                                          kTcBN));
   m.split = (int)std::min<int64_t>(split, INT32_MAX / 2);
   m.n_split_max = (int)((m.range + m.split - 1) / m.split);
   return m;
@@ -476,8 +478,7 @@ int beam_attn_prefill_chunk(int kind, const beam_attn_params *p, int32_t B, int3
   ca.T = T;
   ca.window = p->window;
   ca.kind = kind;
-  // (the few-token path reads a global cache only up to pos0 + T: no padding needed)
-  const int64_t prep_ctas = local ? (int64_t)B * prefix : T <= kMultiMaxT ? 0 : (int64_t)B * kChunkPadRows;
+  const int64_t prep_ctas = (int64_t)B * (local ? prefix : kChunkPadRows);
   if (prep_ctas > 0) {
     chunk_prep_kernel<<<(unsigned)prep_ctas, 128, 0, s>>>(ca);
     if ((st = launch_status())) return st;
@@ -521,45 +522,43 @@ int beam_attn_prefill_chunk(int kind, const beam_attn_params *p, int32_t B, int3
                                                        round_up((size_t)B * T * 128 * 4, 256)
                                                              : 0);
     const size_t parts = (size_t)B * kHkv * mp.n_mt * mp.n_split_max * 16;
-    MultiArgs ma;
-    memset(&ma, 0, sizeof ma);
-    ma.q_raw = static_cast<const uint16_t *>(q);
+    if ((st = encode_fn())) return st;
+    CUtensorMap tk, tv;
     if (local) {
-      ma.key = k_ext;
-      ma.val = v_ext;
-      ma.stride_seq = ext_rows * kHkv * kD;
-      ma.stride_head = kD;
-      ma.stride_row = kHkv * kD;
+      if ((st = make_head_map(&tk, k_ext, kHkv, (int)ext_rows, B))) return st;
+      if ((st = make_head_map(&tv, v_ext, kHkv, (int)ext_rows, B))) return st;
     } else {
-      ma.key = static_cast<const uint16_t *>(k_cache);
-      ma.val = static_cast<const uint16_t *>(v_cache);
-      ma.stride_seq = layout->stride_seq;
-      ma.stride_head = layout->stride_head;
-      ma.stride_row = layout->stride_slot;
+      if ((st = make_cache_map(&tk, k_cache, layout, B))) return st;
+      if ((st = make_cache_map(&tv, v_cache, layout, B))) return st;
     }
-    ma.pos0 = pos0;
-    ma.qw = q_norm_w;
-    ma.eps = p->rms_eps;
-    ma.kind = kind;
-    ma.window = p->window;
-    ma.T = T;
-    ma.n_mt = mp.n_mt;
-    ma.prefix = prefix;
-    ma.slots = layout->slots_per_seq;
-    ma.split = mp.split;
-    ma.n_split_max = mp.n_split_max;
-    ma.scale_log2 = p->softmax_scale * kLog2e;
-    ma.ssmax_base = p->ssmax_base;
-    ma.ssmax_exp = p->ssmax_exp;
-    ma.part_o = reinterpret_cast<float *>(pw);
-    ma.part_ml = reinterpret_cast<float *>(pw + round_up(parts * kD * 4, 256));
-    fill_inv_freq(ma.inv_freq, p->rope_theta);
-    if ((int64_t)mp.n_split_max * mp.n_mt > INT32_MAX || B > 65535) return BEAM_ERR_UNSUPPORTED;
-    decode_multi_kernel<<<dim3(mp.n_split_max * mp.n_mt, kHkv, B), kDecThreads, kDecSmem, s>>>(ma);
+    DecodeTcArgs da;
+    memset(&da, 0, sizeof da);
+    da.q_raw = static_cast<const uint16_t *>(q);
+    da.qw = q_norm_w;
+    da.eps = p->rms_eps;
+    da.rope_tab = rope_tab;
+    da.pos0 = pos0;
+    da.kind = kind;
+    da.window = p->window;
+    da.T = T;
+    da.prefix = prefix;
+    da.slots = layout->slots_per_seq;
+    da.split = mp.split;
+    da.n_split_max = mp.n_split_max;
+    da.n_mt = mp.n_mt;
+    da.scale_log2 = p->softmax_scale * kLog2e;
+    da.ssmax_base = p->ssmax_base;
+    da.ssmax_exp = p->ssmax_exp;
+    da.part_o = reinterpret_cast<float *>(pw);
+    da.part_ml = reinterpret_cast<float *>(pw + round_up(parts * kD * 4, 256));
+    da.status = dev_status;
+    da.kv_slot_major = local ? 0 : 1;
+    if (mp.n_split_max > 65535 || B > 65535) return BEAM_ERR_UNSUPPORTED;
+    decode_tc_kernel<<<dim3(mp.n_split_max, kHkv, B), kDtThreads, kDtSmemBytes, s>>>(tk, tv, da);
     if ((st = launch_status())) return st;
     MultiCombineArgs mc;
-    mc.part_o = ma.part_o;
-    mc.part_ml = ma.part_ml;
+    mc.part_o = da.part_o;
+    mc.part_ml = da.part_ml;
     mc.pos0 = pos0;
     mc.gate = static_cast<const uint16_t *>(gate);
     mc.gate_bias = gate_bias;

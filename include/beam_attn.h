@@ -159,15 +159,15 @@ BEAM_API size_t beam_prefill_chunk_workspace_bytes(int kind, const beam_attn_par
  * the chunk's own keys up to t.  Tensors as in beam_attn_prefill; the new keys
  * and values are appended as there, at their own positions (a local ring keeps
  * the last min(T, window) of them).  pos0 = 0 everywhere is a plain prefill.
- * A global call of more than 16 new tokens also zeroes the value slots from
- * pos0[b]+T up to the next multiple of 128 below the capacity: they hold no
- * token yet.  A sequence with
+ * A global call also zeroes the value slots from pos0[b]+T up to the next
+ * multiple of 128 below the capacity: they hold no token yet.  A sequence with
  * pos0[b] < 0, or (global) pos0[b] + T > slots_per_seq, sets BEAM_ERR_CAPACITY
  * in dev_status and is neither appended nor written to `out`; the others are
  * unaffected.  T > slots_per_seq (global) is BEAM_ERR_CAPACITY before any launch.
  * Up to 16 new tokens (multi-token decode, e.g. verifying a drafted block) run on
- * a split-K kernel that spreads the history over many CTAs; longer chunks on the
- * tcgen05 prefill kernel, whose bounded waits behave as in beam_attn_prefill. */
+ * a split-K tcgen05 kernel that spreads the history over many CTAs; longer chunks
+ * on the tcgen05 prefill kernel.  The bounded waits of both behave as in
+ * beam_attn_prefill. */
 BEAM_API int beam_attn_prefill_chunk(int kind, const beam_attn_params *p, int32_t B, int32_t T,
                                      const void *q, const void *k, const void *v, const void *gate,
                                      const float *q_norm_w, const float *k_norm_w,

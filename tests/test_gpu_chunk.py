@@ -68,7 +68,7 @@ def check_cache(orc, ci, params, kc, vc, skip=()):
             d = np.abs(as_f64(kh[b, :, s]) - as_f64(kr))
             assert np.all(d <= np.abs(as_f64(kr)) * 2.0 ** -7 + K_ABS), (b, t)
             written[b, s] = True
-        if ci.kind == wl.GLOBAL and ci.T > 16:   # the tcgen05 path reads whole 128-key blocks
+        if ci.kind == wl.GLOBAL:   # the attention kernels read whole 128-key blocks
             end = p0 + ci.T
             padded[b, end:min(S, (end + 127) // 128 * 128)] = True
     keep = ~written
