@@ -553,6 +553,10 @@ int beam_attn_prefill_chunk(int kind, const beam_attn_params *p, int32_t B, int3
     da.part_ml = reinterpret_cast<float *>(pw + round_up(parts * kD * 4, 256));
     da.status = dev_status;
     da.kv_slot_major = local ? 0 : 1;
+    {  // the same test-only fault injection as the prefill kernel's
+      const char *f = std::getenv("BEAM_FAULT_INJECT");
+      da.fault_stall = f != nullptr && std::strcmp(f, "prefill_wait_stall") == 0;
+    }
     if (mp.n_split_max > 65535 || B > 65535) return BEAM_ERR_UNSUPPORTED;
     decode_tc_kernel<<<dim3(mp.n_split_max, kHkv, B), kDtThreads, kDtSmemBytes, s>>>(tk, tv, da);
     if ((st = launch_status())) return st;

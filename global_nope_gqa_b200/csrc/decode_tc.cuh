@@ -23,7 +23,9 @@
 //               the swizzled Q tile, then the online softmax per block (mask to the row's
 //               coordinates, stale max, O rescaled only when the max grows by more than 2^8,
 //               after the previous block's P V is done), then one partial (m, l, o[128]).
-// decode_multi_combine_kernel merges the runs and gates.  Every wait is bounded (tc_wait).
+// decode_multi_combine_kernel merges the runs and gates.  Every wait is bounded (tc_wait: 1 s
+// of device time, then BEAM_ERR_DEVICE_TIMEOUT, an abort flag for the other roles, and the
+// in-flight copies and MMAs drained before the tensor memory is freed).
 #pragma once
 
 #include "common.cuh"
@@ -43,7 +45,7 @@ constexpr uint32_t kDtSmemBytes = kDtSmemBar + 256 + 1024;          // 197,888 B
 
 namespace dtd {
 constexpr int kKFull = 0, kKEmpty = 3, kVFull = 6, kVEmpty = 8, kSFull = 10, kPFull = 12,
-              kPVDone = 14, kOFull = 15, kQReady = 16, kDrain = 17, kNumBars = 18;
+              kPVDone = 14, kOFull = 15, kQReady = 16, kDrain = 17, kStall = 18, kNumBars = 19;
 constexpr uint32_t kTmemHolder = kNumBars * 8;
 constexpr uint32_t kAbortFlag = kTmemHolder + 4;
 }  // namespace dtd
@@ -61,6 +63,7 @@ struct DecodeTcArgs {
   float *part_o, *part_ml;    // the layout decode_multi_combine_kernel reads
   int32_t *status;
   int kv_slot_major;          // K/V maps take (d, slot, head, b) rather than (d, head, t, b)
+  int fault_stall;            // tests only: the MMA issuer first waits on a barrier never arrived at
 };
 
 __global__ void __launch_bounds__(kDtThreads, 1)
@@ -77,8 +80,8 @@ __global__ void __launch_bounds__(kDtThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool local = a.kind == BEAM_LOCAL;
 
-  // key coordinates of the sequence (as decode_multi_kernel); an out-of-range pos0 has set
-  // the status in the prologue and does nothing here (the whole CTA returns together)
+  // key coordinates of the sequence (see above); an out-of-range pos0 has set the status in
+  // the prologue and does nothing here (the whole CTA returns together)
   const int64_t p0 = a.pos0[b];
   if (p0 < 0 || (!local && p0 + a.T > a.slots)) return;
   int64_t kq, lo_all;
@@ -184,7 +187,8 @@ __global__ void __launch_bounds__(kDtThreads, 1)
         tc::umma_commit(bar(dtd::kVEmpty + j % kDtVSlots));
         if (j == nb - 1) tc::umma_commit(bar(dtd::kOFull));
       };
-      bool ok = tc_wait(bar(dtd::kQReady), 0u, abort, a.status);
+      bool ok = (!a.fault_stall || tc_wait(bar(dtd::kStall), 0u, abort, a.status)) &&
+                tc_wait(bar(dtd::kQReady), 0u, abort, a.status);
       for (int jj = 0; ok && jj < 2 && jj < nb; ++jj) {
         if (!(ok = tc_wait(bar(dtd::kKFull + jj % kDtKSlots), (jj / kDtKSlots) & 1u, abort,
                            a.status)))
@@ -374,10 +378,15 @@ __global__ void __launch_bounds__(kDtThreads, 1)
       tc::tc_fence_before();
       tc::mbar_arrive(bar(dtd::kPFull + (j & 1)));
     }
-    if (ok && (ok = tc_wait(bar(dtd::kOFull), 0u, abort, a.status))) {
+    const int mt = tok / kMultiTokPerTile, row16 = (tok % kMultiTokPerTile) * kGroup + hh;
+    const size_t part = ((((size_t)b * kHkv + g) * a.n_mt + mt) * a.n_split_max + s_idx) * 16 + row16;
+    if (ok) ok = tc_wait(bar(dtd::kOFull), 0u, abort, a.status);
+    if (!ok && row_ok) {   // a wait ran out: the merge turns these rows into NaN
+      a.part_ml[part * 2] = __int_as_float(0x7fc00000);
+      a.part_ml[part * 2 + 1] = __int_as_float(0x7fc00000);
+    }
+    if (ok) {
       tc::tc_fence_after();
-      const int mt = tok / kMultiTokPerTile, row16 = (tok % kMultiTokPerTile) * kGroup + hh;
-      const size_t part = ((((size_t)b * kHkv + g) * a.n_mt + mt) * a.n_split_max + s_idx) * 16 + row16;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t o[32];

@@ -42,3 +42,28 @@ def test_prefill_wait_timeout_sets_status_and_context_survives(env, monkeypatch,
     ref = orc.prefill(kind, oracle_params(orc, beam.default_params()), inp.q, inp.k, inp.v,
                       inp.gate, inp.q_norm_w, inp.k_norm_w, inp.gate_bias)
     assert_close(host_bits(out).reshape(ref.shape), ref, f"after timeout kind={kind}")
+
+
+@pytest.mark.parametrize("kind", [wl.GLOBAL, wl.LOCAL])
+def test_multi_token_decode_wait_timeout(env, monkeypatch, kind):
+    """The same injected stall in the tcgen05 multi-token decode kernel (a chunk of 8
+    new tokens): status -4, no output row written, then a clean call passes parity."""
+    torch, beam, orc = env
+    from test_gpu_chunk import oracle_chunk, run_chunk
+    params = beam.default_params()
+    slots = 4096 if kind == wl.GLOBAL else 512
+    ci = wl.chunk_inputs(kind, 8, [3000], slots, 93, layer=f"mto{kind}")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    monkeypatch.setenv("BEAM_FAULT_INJECT", "prefill_wait_stall")
+    t0 = time.perf_counter()
+    out, *_ = run_chunk(torch, beam, ci, params, status)
+    elapsed = time.perf_counter() - t0
+    monkeypatch.delenv("BEAM_FAULT_INJECT")
+    assert int(status.item()) == -4
+    assert torch.isnan(out).all()
+    assert elapsed < 30.0
+    status.zero_()
+    out, *_ = run_chunk(torch, beam, ci, params, status)
+    assert int(status.item()) == 0
+    ref = oracle_chunk(orc, beam, ci, params)
+    assert_close(host_bits(out).reshape(ref.shape), ref, f"after timeout kind={kind}")
