@@ -675,12 +675,19 @@ def run_gpu(args):
 
 
 def run_decode_case(args):
-    """Profiling case: one global-layer decode call (B=1) at --context, BF16 or FP8 cache,
-    timed alone; prints one JSON line (not the headline)."""
+    """Profiling case: one global-layer decode call (B=1) at --context, BF16 or FP8 cache, or
+    one 8-new-token chunk call (multi8), timed alone; prints one JSON line (not the headline)."""
     import torch
     torch.cuda.set_device(0)
     import global_nope_gqa_b200 as beam
     beam.lib()
+    if args.decode_case == "multi8":
+        L = ChunkLayer(torch, beam, wl.GLOBAL, 8, args.context - 8, args.context, args.seed, "case")
+        sec = time_loop(torch, L.run, args.steps, args.warmup)
+        assert int(L.status.item()) == 0
+        print(json.dumps({"case": f"global chunk of 8 new tokens, B=1, context {args.context}",
+                          "ms": sec * 1e3, "GBps": L.bytes / sec / 1e9}), flush=True)
+        return
     fp8 = args.decode_case == "fp8"
     L = DecodeLayer(torch, beam, wl.GLOBAL, [args.context], args.context, args.seed, "case",
                     fp8=fp8)
@@ -730,7 +737,7 @@ def main(argv=None):
     ap.add_argument("--layers", default="both", choices=["both", "global", "local"],
                     help="prefill layers per step (profiling cases; the headline step is both)")
     ap.add_argument("--batch", type=int, default=0, help="override B (profiling cases)")
-    ap.add_argument("--decode-case", choices=["bf16", "fp8"], default=None,
+    ap.add_argument("--decode-case", choices=["bf16", "fp8", "multi8"], default=None,
                     help="profiling case: time one global decode call at --context only")
     ap.add_argument("--context", type=int, default=wl.MAX_CONTEXT)
     args = ap.parse_args(argv)

@@ -575,7 +575,7 @@ int beam_attn_prefill_chunk(int kind, const beam_attn_params *p, int32_t B, int3
     mc.split = mp.split;
     mc.n_split_max = mp.n_split_max;
     mc.slots = layout->slots_per_seq;
-    decode_multi_combine_kernel<<<dim3(kHq, T, B), kD, 0, s>>>(mc);
+    decode_multi_combine_kernel<<<dim3(kHq, T, B), kCombineThreads, 0, s>>>(mc);
     return launch_status();
   }
   if ((st = encode_fn())) return st;
@@ -768,7 +768,7 @@ int decode_call(int kind, const beam_attn_params *p, int32_t B, const void *q, c
   ca.split = split;
   ca.n_split_max = n_split_max;
   ca.slots = layout->slots_per_seq;
-  decode_combine_kernel<<<dim3(kHq, B), kD, 0, s>>>(ca);
+  decode_combine_kernel<<<dim3(kHq, B), kCombineThreads, 0, s>>>(ca);
   return launch_status();
 }
 

@@ -373,12 +373,14 @@ struct CombineArgs {
   int64_t slots;
 };
 
-// One CTA of 128 threads per (query head, sequence).  The split weights are formed once in
-// shared memory (2^(m_s - M), with every split's m read in parallel), then thread d sums
-// w_s o_s[d] over the splits: independent, coalesced loads, so the merge costs a few memory
-// latencies rather than one per split.  Y = O / l * sigmoid(G + b_h).
+// One CTA of 256 threads per (query head, sequence).  The split weights 2^(m_s - M) are formed
+// once in shared memory (every split's m read in parallel); then warp w sums the splits
+// w, w + 8, ... for d = 4 lane .. 4 lane + 3 with independent float4 loads, and the eight
+// warp sums are added in shared memory: a few memory latencies in all, not one per split.
+// Y = O / l * sigmoid(G + b_h).
 constexpr int kCombineMaxSplits = 1024;
-__global__ void __launch_bounds__(kD) decode_combine_kernel(const CombineArgs a) {
+constexpr int kCombineThreads = 256;
+__global__ void __launch_bounds__(kCombineThreads) decode_combine_kernel(const CombineArgs a) {
   const int h = blockIdx.x, b = blockIdx.y;
   const int g = h / kGroup, hh = h - g * kGroup;
   const int64_t t = a.pos[b];
@@ -389,12 +391,13 @@ __global__ void __launch_bounds__(kD) decode_combine_kernel(const CombineArgs a)
   if (n_vis == 0) return;  // invalid position: output untouched, status set upstream
   const int n_split = (int)min((n_vis + a.split - 1) / a.split, (int64_t)kCombineMaxSplits);
   __shared__ float sm_w[kCombineMaxSplits];
-  __shared__ float sm_red[kD / 32];
-  const int d = threadIdx.x, lane = d & 31, warp = d >> 5;
+  __shared__ float sm_red[kCombineThreads / 32];
+  __shared__ float4 sm_acc[kCombineThreads / 32][32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const size_t base = ((size_t)b * kHkv + g) * a.n_split_max;
   // M = max_s m_s
   float mx = -INFINITY;
-  for (int s = d; s < n_split; s += kD) {
+  for (int s = tid; s < n_split; s += kCombineThreads) {
     const float m = a.part_ml[((base + s) * kGroup + hh) * 2];
     sm_w[s] = m;
     mx = fmaxf(mx, m);
@@ -405,30 +408,51 @@ __global__ void __launch_bounds__(kD) decode_combine_kernel(const CombineArgs a)
   __syncthreads();
   float M = sm_red[0];
 #pragma unroll
-  for (int w = 1; w < kD / 32; ++w) M = fmaxf(M, sm_red[w]);
+  for (int w = 1; w < kCombineThreads / 32; ++w) M = fmaxf(M, sm_red[w]);
   const float Mu = M == -INFINITY ? 0.f : M;
   __syncthreads();
   // weights and L = sum_s w_s l_s
   float lsum = 0.f;
-  for (int s = d; s < n_split; s += kD) {
+  for (int s = tid; s < n_split; s += kCombineThreads) {
     const float w = ex2_approx(sm_w[s] - Mu);
     sm_w[s] = w;
     lsum += w * a.part_ml[((base + s) * kGroup + hh) * 2 + 1];
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
-  if (lane == 0) sm_red[warp] = lsum;
   __syncthreads();
-  float L = 0.f;
-#pragma unroll
-  for (int w = 0; w < kD / 32; ++w) L += sm_red[w];
-  float acc = 0.f;
-  const float *po = a.part_o + (base * kGroup + hh) * kD + d;
+  if (lane == 0) sm_red[warp] = lsum;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  const float4 *po = reinterpret_cast<const float4 *>(a.part_o + (base * kGroup + hh) * kD) + lane;
 #pragma unroll 4
-  for (int s = 0; s < n_split; ++s) acc += sm_w[s] * po[(size_t)s * kGroup * kD];
-  const size_t oi = ((size_t)b * kHq + h) * kD + d;
-  const float gl = bf16_lo(a.gate[oi]) + a.gate_bias[h];
-  a.out[oi] = (uint16_t)(pack_bf16(acc / L / (1.0f + expf(-gl)), 0.f) & 0xFFFFu);
+  for (int s = warp; s < n_split; s += kCombineThreads / 32) {
+    const float w = sm_w[s];
+    const float4 v = po[(size_t)s * kGroup * kD / 4];
+    acc.x = fmaf(w, v.x, acc.x); acc.y = fmaf(w, v.y, acc.y);
+    acc.z = fmaf(w, v.z, acc.z); acc.w = fmaf(w, v.w, acc.w);
+  }
+  sm_acc[warp][lane] = acc;
+  __syncthreads();
+  if (warp == 0) {
+    float L = 0.f;
+#pragma unroll
+    for (int w = 0; w < kCombineThreads / 32; ++w) L += sm_red[w];
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int w = 0; w < kCombineThreads / 32; ++w) {
+      o.x += sm_acc[w][lane].x; o.y += sm_acc[w][lane].y;
+      o.z += sm_acc[w][lane].z; o.w += sm_acc[w][lane].w;
+    }
+    const size_t oi = ((size_t)b * kHq + h) * kD + 4 * lane;
+    const uint2 graw = *reinterpret_cast<const uint2 *>(a.gate + oi);
+    const float bias = a.gate_bias[h], inv = 1.0f / L;
+    const float gl[4] = {bf16_lo(graw.x), bf16_hi(graw.x), bf16_lo(graw.y), bf16_hi(graw.y)};
+    const float ov[4] = {o.x, o.y, o.z, o.w};
+    float y[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) y[e] = ov[e] * inv / (1.0f + expf(-(gl[e] + bias)));
+    *reinterpret_cast<uint2 *>(a.out + oi) = make_uint2(pack_bf16(y[0], y[1]), pack_bf16(y[2], y[3]));
+  }
 }
 
 }  // namespace beam

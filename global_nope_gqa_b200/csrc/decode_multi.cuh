@@ -29,14 +29,15 @@ struct MultiCombineArgs {
   int64_t slots;
 };
 
-// One CTA of 128 threads per (query head, new token, sequence): thread d merges the splits of
-// coordinate d (all loads independent), then applies Y = O / l * sigmoid(G + b_h).
-__global__ void __launch_bounds__(kD) decode_multi_combine_kernel(const MultiCombineArgs c) {
+// One CTA of 256 threads per (query head, new token, sequence), organised as the one-token
+// combine: split weights in shared memory, then warp w sums the splits w, w + 8, ... with
+// float4 loads, the warp sums are added, and Y = O / l * sigmoid(G + b_h).
+__global__ void __launch_bounds__(kCombineThreads) decode_multi_combine_kernel(const MultiCombineArgs c) {
   const int h = blockIdx.x, tok = blockIdx.y, b = blockIdx.z;
   const int g = h / kGroup, hh = h - g * kGroup;
   const int64_t p0 = c.pos0[b];
   if (p0 < 0 || (c.kind == BEAM_GLOBAL && p0 + c.T > c.slots)) return;  // status set upstream
-  int64_t lo, hi = 0;
+  int64_t lo, hi;
   if (c.kind == BEAM_LOCAL) {
     const int64_t kmin = c.prefix - min(p0, (int64_t)c.prefix);
     lo = max(kmin, (int64_t)c.prefix - c.window + 1);
@@ -45,23 +46,69 @@ __global__ void __launch_bounds__(kD) decode_multi_combine_kernel(const MultiCom
     lo = 0;
     hi = p0 + c.T - 1;
   }
-  const int n_split = (int)((hi - lo) / c.split + 1);
+  const int n_split = (int)min((hi - lo) / c.split + 1, (int64_t)kCombineMaxSplits);
   const int mt = tok / kMultiTokPerTile, row = (tok % kMultiTokPerTile) * kGroup + hh;
   const size_t base = (((size_t)b * kHkv + g) * c.n_mt + mt) * c.n_split_max;
-  const int d = threadIdx.x;
-  float M = -INFINITY;
-  for (int s = 0; s < n_split; ++s) M = fmaxf(M, c.part_ml[((base + s) * 16 + row) * 2]);
-  const float Mu = M == -INFINITY ? 0.f : M;
-  float acc = 0.f, L = 0.f;
-  for (int s = 0; s < n_split; ++s) {
-    const size_t pr = (base + s) * 16 + row;
-    const float w = ex2_approx(c.part_ml[pr * 2] - Mu);
-    acc += w * c.part_o[pr * kD + d];
-    L += w * c.part_ml[pr * 2 + 1];
+  __shared__ float sm_w[kCombineMaxSplits];
+  __shared__ float sm_red[kCombineThreads / 32];
+  __shared__ float4 sm_acc[kCombineThreads / 32][32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  float mx = -INFINITY;
+  for (int s = tid; s < n_split; s += kCombineThreads) {
+    const float m = c.part_ml[((base + s) * 16 + row) * 2];
+    sm_w[s] = m;
+    mx = fmaxf(mx, m);
   }
-  const size_t oi = (((size_t)b * c.T + tok) * kHq + h) * kD + d;
-  const float gl = __uint_as_float((uint32_t)c.gate[oi] << 16) + c.gate_bias[h];
-  c.out[oi] = (uint16_t)(pack_bf16(acc / L / (1.0f + expf(-gl)), 0.f) & 0xFFFFu);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  if (lane == 0) sm_red[warp] = mx;
+  __syncthreads();
+  float M = sm_red[0];
+#pragma unroll
+  for (int w = 1; w < kCombineThreads / 32; ++w) M = fmaxf(M, sm_red[w]);
+  const float Mu = M == -INFINITY ? 0.f : M;
+  __syncthreads();
+  float lsum = 0.f;
+  for (int s = tid; s < n_split; s += kCombineThreads) {
+    const float w = ex2_approx(sm_w[s] - Mu);
+    sm_w[s] = w;
+    lsum += w * c.part_ml[((base + s) * 16 + row) * 2 + 1];
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
+  __syncthreads();
+  if (lane == 0) sm_red[warp] = lsum;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  const float4 *po = reinterpret_cast<const float4 *>(c.part_o + (base * 16 + row) * kD) + lane;
+#pragma unroll 4
+  for (int s = warp; s < n_split; s += kCombineThreads / 32) {
+    const float w = sm_w[s];
+    const float4 v = po[(size_t)s * 16 * kD / 4];
+    acc.x = fmaf(w, v.x, acc.x); acc.y = fmaf(w, v.y, acc.y);
+    acc.z = fmaf(w, v.z, acc.z); acc.w = fmaf(w, v.w, acc.w);
+  }
+  sm_acc[warp][lane] = acc;
+  __syncthreads();
+  if (warp == 0) {
+    float L = 0.f;
+#pragma unroll
+    for (int w = 0; w < kCombineThreads / 32; ++w) L += sm_red[w];
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int w = 0; w < kCombineThreads / 32; ++w) {
+      o.x += sm_acc[w][lane].x; o.y += sm_acc[w][lane].y;
+      o.z += sm_acc[w][lane].z; o.w += sm_acc[w][lane].w;
+    }
+    const size_t oi = (((size_t)b * c.T + tok) * kHq + h) * kD + 4 * lane;
+    const uint2 graw = *reinterpret_cast<const uint2 *>(c.gate + oi);
+    const float bias = c.gate_bias[h], inv = 1.0f / L;
+    const float gl[4] = {bf16_lo(graw.x), bf16_hi(graw.x), bf16_lo(graw.y), bf16_hi(graw.y)};
+    const float ov[4] = {o.x, o.y, o.z, o.w};
+    float y[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) y[e] = ov[e] * inv / (1.0f + expf(-(gl[e] + bias)));
+    *reinterpret_cast<uint2 *>(c.out + oi) = make_uint2(pack_bf16(y[0], y[1]), pack_bf16(y[2], y[3]));
+  }
 }
 
 }  // namespace beam
