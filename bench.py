@@ -519,22 +519,54 @@ def cpu_baseline_prefill(seconds_target=10.0, seconds_cap=30.0, seed=1234):
 
 
 def e2e_prefill(torch, beam, layers, steps, warmup):
-    """Same metric through the public call with pinned host buffers: each step copies
-    the step's inputs host->device and reads the outputs back."""
-    host_in = []
-    for L in layers:
-        host_in.append({k: v.cpu().pin_memory() for k, v in L.x.items()})
+    """Same metric through the public call with pinned host buffers: every step copies the
+    step's inputs host->device and reads the outputs back.  The step is streamed one
+    sequence at a time (the call with B = 1, caches offset to that sequence): uploads on one
+    stream into two alternating device buffers, the attention on the compute stream, the
+    read-back on a third stream, so the upload of sequence b + 1 and the read-back of b - 1
+    overlap the attention of b (PCIe is full duplex)."""
+    h2d_stream, d2h_stream = torch.cuda.Stream(), torch.cuda.Stream()
+    compute = torch.cuda.current_stream()
+    host_in = [{k: v.cpu().pin_memory() for k, v in L.x.items()} for L in layers]
     host_out = [torch.empty(L.out.shape, dtype=L.out.dtype, pin_memory=True) for L in layers]
-    dev_in = [{k: torch.empty_like(v) for k, v in L.x.items()} for L in layers]
+    B, T = layers[0].B, layers[0].T
+    dev_in = [{k: torch.empty_like(v[:1]) for k, v in layers[0].x.items()} for _ in range(2)]
+    params = layers[0].params
+    ws = torch.empty(beam.beam_prefill_workspace_bytes(params, 1, T), dtype=torch.uint8,
+                     device="cuda")
+    one = {L.kind: beam.beam_kv_layout(L.kind, params, 1, T) for L in layers}
     h2d = sum(v.numel() * v.element_size() for d in host_in for v in d.values())
     d2h = sum(o.numel() * o.element_size() for o in host_out)
+    free = [torch.cuda.Event() for _ in range(2)]
+    loaded = [torch.cuda.Event() for _ in range(2)]
+    done = torch.cuda.Event()
+    for e in free:
+        e.record(compute)
 
     def step():
-        for L, hi, di, ho in zip(layers, host_in, dev_in, host_out):
-            for k in hi:
-                di[k].copy_(hi[k], non_blocking=True)
-            L.run(di)
-            ho.copy_(L.out, non_blocking=True)
+        i = 0
+        for L, hi, ho in zip(layers, host_in, host_out):
+            kc = L.kc.view(B, -1)
+            vc = L.vc.view(B, -1)
+            for b in range(B):
+                buf = i % 2
+                with torch.cuda.stream(h2d_stream):
+                    h2d_stream.wait_event(free[buf])
+                    for k in hi:
+                        dev_in[buf][k].copy_(hi[k][b:b + 1], non_blocking=True)
+                    loaded[buf].record(h2d_stream)
+                compute.wait_event(loaded[buf])
+                x = dev_in[buf]
+                beam.beam_attn_prefill(L.kind, params, x["q"], x["k"], x["v"], x["gate"], L.qw,
+                                       L.kw, L.bias, L.out[b:b + 1], kc[b], vc[b], one[L.kind],
+                                       workspace=ws, dev_status=L.status)
+                free[buf].record(compute)
+                done.record(compute)
+                with torch.cuda.stream(d2h_stream):
+                    d2h_stream.wait_event(done)
+                    ho[b:b + 1].copy_(L.out[b:b + 1], non_blocking=True)
+                i += 1
+        compute.wait_stream(d2h_stream)
     sec = time_loop(torch, step, max(1, steps // 2), max(1, warmup // 2))
     return sec, h2d, d2h
 
