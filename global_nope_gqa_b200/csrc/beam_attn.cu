@@ -383,7 +383,7 @@ MultiPlan multi_plan(int kind, const beam_attn_params *p, int32_t B, int32_t T, 
   MultiPlan m;
   m.n_mt = (T + kMultiTokPerTile - 1) / kMultiTokPerTile;
   m.range = kind == BEAM_LOCAL ? (int64_t)p->window - 1 + T : slots;
-  // one CTA per SM fits (197 KB of shared memory): about two waves, runs of whole
+  // one CTA per SM fits (225 KB of shared memory): about two waves, runs of whole
   // 128-key tiles
   const int64_t target = (int64_t)sm_count * 2;
   const int64_t per_run = (int64_t)B * kHkv;

@@ -12,7 +12,7 @@
 // (token, head) rows r = 6 i + h of the group for all T new tokens (6 T <= 96 rows; the rest
 // are zero), so every key tile is multiplied once for all of them, on tcgen05 MMAs:
 //   warp 0      TMA producer: 128-key K tiles into a three-slot ring running two blocks
-//               ahead of the V tiles (two slots), 128-byte swizzled 128 x 64 boxes;
+//               ahead of the V tiles (three slots), 128-byte swizzled 128 x 64 boxes;
 //   warp 1      MMA issuer (one thread) and the tensor memory (512 columns): S in two
 //               buffers [0,128) [128,256), O [256,384) (fp32).  Block j uses S buffer j % 2,
 //               its P (bf16 pairs) overwrites the first 64 columns of that buffer, and
@@ -36,16 +36,19 @@
 namespace beam {
 
 constexpr int kDtThreads = 192;
-constexpr int kDtKSlots = 3, kDtVSlots = 2;
+constexpr int kDtKSlots = 3, kDtVSlots = 3;
 constexpr uint32_t kDtSmemQ = 0;                                    // one 128 x 128 Q tile
 constexpr uint32_t kDtSmemK = kTcTileBytes;                         // K ring
 constexpr uint32_t kDtSmemV = kDtSmemK + kDtKSlots * kTcTileBytes;  // V ring
 constexpr uint32_t kDtSmemBar = kDtSmemV + kDtVSlots * kTcTileBytes;
-constexpr uint32_t kDtSmemBytes = kDtSmemBar + 256 + 1024;          // 197,888 B
+constexpr uint32_t kDtSmemBytes = kDtSmemBar + 256 + 1024;          // 230,656 B
 
-namespace dtd {
-constexpr int kKFull = 0, kKEmpty = 3, kVFull = 6, kVEmpty = 8, kSFull = 10, kPFull = 12,
-              kPVDone = 14, kOFull = 15, kQReady = 16, kDrain = 17, kStall = 18, kNumBars = 19;
+namespace dtd {  // barrier slots (8 bytes each) after kDtSmemBar, laid out from the ring sizes
+constexpr int kKFull = 0, kKEmpty = kKFull + kDtKSlots, kVFull = kKEmpty + kDtKSlots,
+              kVEmpty = kVFull + kDtVSlots, kSFull = kVEmpty + kDtVSlots, kPFull = kSFull + 2,
+              kPVDone = kPFull + 2, kOFull = kPVDone + 1, kQReady = kOFull + 1,
+              kDrain = kQReady + 1, kStall = kDrain + 1, kNumBars = kStall + 1;
+static_assert(kNumBars * 8 + 8 <= 256, "the barrier area holds 256 bytes");
 constexpr uint32_t kTmemHolder = kNumBars * 8;
 constexpr uint32_t kAbortFlag = kTmemHolder + 4;
 }  // namespace dtd
@@ -292,7 +295,15 @@ __global__ void __launch_bounds__(kDtThreads, 1)
     const uint32_t t_o = tmem + lane_off + 256;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < nb; ++j) {
+    // A warp whose 32 rows are all padding (6 T <= 32 wq) only keeps the barrier phases: its
+    // query rows are zero, so its scores are zero and its P rows stay zero in tensor memory,
+    // and P V never mixes rows.  It leaves the special-function units to the real rows.
+    const bool warp_rows = wq * 32 < kGroup * a.T;
+    for (int j = 0; j < nb && !warp_rows; ++j) {
+      if (!(ok = tc_wait(bar(dtd::kSFull + (j & 1)), (j >> 1) & 1u, abort, a.status))) break;
+      tc::mbar_arrive(bar(dtd::kPFull + (j & 1)));
+    }
+    for (int j = 0; j < nb && warp_rows; ++j) {
       if (!(ok = tc_wait(bar(dtd::kSFull + (j & 1)), (j >> 1) & 1u, abort, a.status))) break;
       tc::tc_fence_after();
       const uint32_t t_s = tmem + lane_off + 128 * (j & 1);
