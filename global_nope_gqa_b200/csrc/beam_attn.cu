@@ -80,7 +80,12 @@ int device_info(DeviceInfo **out) {
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, kDec8Smem),
                           "FP8 decode shared-memory opt-in")))
       return st;
-    if ((st = cuda_status(cudaFuncSetAttribute(prefill_tc_kernel,
+    if ((st = cuda_status(cudaFuncSetAttribute(prefill_tc_kernel<true>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               kTcSmemBytes),
+                          "prefill shared-memory opt-in")))
+      return st;
+    if ((st = cuda_status(cudaFuncSetAttribute(prefill_tc_kernel<false>,
                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                kTcSmemBytes),
                           "prefill shared-memory opt-in")))
@@ -204,9 +209,14 @@ int launch_prefill_attention(int kind, const beam_attn_params *p, int32_t B, int
   const int64_t n_units = (int64_t)fa.n_qblocks * (kHq / 2) * B;
   if (n_units > INT32_MAX) return BEAM_ERR_UNSUPPORTED;
   fa.n_units = (int)n_units;
+  CUtensorMap tm_o;   // the output rows, stored tile by tile (rows past T are clipped)
+  if (int st = make_head_map(&tm_o, fa.out, kHq, T, B)) return st;
   // persistent: one CTA per SM (the kernel's shared memory admits one per SM)
   const int grid = (int)std::min<int64_t>(n_units, dev->sm_count);
-  prefill_tc_kernel<<<grid, kTcThreads, kTcSmemBytes, s>>>(tm_q, tm_k, tm_v, fa);
+  if (kind == BEAM_GLOBAL)
+    prefill_tc_kernel<true><<<grid, kTcThreads, kTcSmemBytes, s>>>(tm_q, tm_k, tm_v, tm_o, fa);
+  else
+    prefill_tc_kernel<false><<<grid, kTcThreads, kTcSmemBytes, s>>>(tm_q, tm_k, tm_v, tm_o, fa);
   return launch_status();
 }
 

@@ -22,7 +22,14 @@
 //               written as bf16 pairs over the first 64 columns of S_t;
 //   warp 2      Q producer (TMA): the raw Q tiles of unit n into Q set n % 2, so the next
 //               unit's Q is loaded and prepared while the current unit runs;
-//   warp 3      idle;
+//   warp 3      output store (TMA), global layer: the softmax threads stage a unit's Y
+//               tiles in the unit's own Q set, whose Q is no longer read once O is final;
+//               one thread stores both tiles (rows past T are clipped by the copy) and
+//               hands the set back to the Q producer once the copies have read it.  A
+//               local layer's units are short (at most five key blocks), too short to hide
+//               that later release (the set's next Q must be loaded and prepared while the
+//               following unit runs), so there the softmax threads store their rows
+//               directly and the MMA issuer releases the set after the unit's last Q K^T;
 //   warps 12-15 Q preparation: once a unit's raw Q tiles have landed, RMSNorm (and RoPE
 //               with a per-position cos/sin table for a local layer) each row in place in
 //               shared memory, then release the tiles to the MMA issuer;
@@ -32,7 +39,8 @@
 //               m and sum l in exp2 units, writes P and, only when the row max grew by more
 //               than 2^8, rescales its O row in tensor memory (the stale max keeps every
 //               P <= 256, safe in fp32 and bf16).  After a unit's last block the same
-//               threads run the epilogue O/l * sigmoid(G + b) and release O.
+//               threads run the epilogue O/l * sigmoid(G + b), release O and write Y
+//               as bf16 rows, into the unit's Q tile t for the store warp or to HBM.
 // MMAs issued by one thread run in issue order, so S_t(j+1), which overwrites P_t(j), is
 // issued after O_t += P_t(j) V_j; the commit that publishes S_t(j) also covers the O_t
 // update of block j-1, which lets the softmax rescale O_t without a further wait.  Key
@@ -72,7 +80,7 @@ struct PrefillTcArgs {
   float eps;
   const uint16_t *gate;   // [B][T][48*128]
   const float *gate_bias; // [48]
-  uint16_t *out;          // [B][T][48*128]
+  uint16_t *out;          // [B][T][48*128], written directly or through the map tm_o
   int32_t *status;
   int B, T, kind, window, n_qblocks, n_units;
   float scale_log2, ssmax_base, ssmax_exp;
@@ -88,10 +96,12 @@ struct PrefillTcArgs {
 namespace tcd {
 // barrier slots (8 bytes each) after kTcSmemBar
 constexpr int kQFull = 0, kQEmpty = 2, kQReady = 4, kKVFull = 6, kKVEmpty = 9, kSFull = 12,
-              kPFull = 14, kOFull = 16, kOEmpty = 18, kDrain = 20, kStall = 21, kNumBars = 22;
+              kPFull = 14, kOFull = 16, kOEmpty = 18, kDrain = 20, kStall = 21, kYReady = 22,
+              kNumBars = 24;
 constexpr uint32_t kTmemHolder = kNumBars * 8;      // u32: tensor-memory base address
 constexpr uint32_t kAbortFlag = kTmemHolder + 4;    // u32: set when a wait ran out
 }  // namespace tcd
+static_assert(tcd::kAbortFlag + 4 <= 256, "barrier area of the prefill kernel overflows");
 
 __device__ __forceinline__ float tanh_approx(float x) {
   float y;
@@ -208,10 +218,31 @@ __device__ __forceinline__ TcUnit tc_unit(const PrefillTcArgs &a, int u) {
   return w;
 }
 
+// Y = O * inv * (1 + tanh((G + b) / 2)) (inv = 1 / (2 l), hb = b / 2) for the 8 coordinates
+// of one 16-byte word: o holds the 32 fp32 O values of a chunk, q picks 8 of them.
+__device__ __forceinline__ uint4 gated_y8(const uint4 g4, const uint32_t (&o)[32], int q, float inv,
+                                          float hb) {
+  const uint32_t gw[4] = {g4.x, g4.y, g4.z, g4.w};
+  uint32_t yw[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float s0 = 1.0f + tanh_approx(fmaf(0.5f, bf16_lo(gw[e]), hb));
+    const float s1 = 1.0f + tanh_approx(fmaf(0.5f, bf16_hi(gw[e]), hb));
+    yw[e] = pack_bf16(__uint_as_float(o[q * 8 + 2 * e]) * inv * s0,
+                      __uint_as_float(o[q * 8 + 2 * e + 1]) * inv * s1);
+  }
+  return make_uint4(yw[0], yw[1], yw[2], yw[3]);
+}
+
+// kStage: the output goes through shared memory and the store warp (global layer); the
+// two forms are separate instantiations so that each keeps its own register allocation.
+template <bool kStage>
+
 __global__ void __launch_bounds__(kTcThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
-                      const __grid_constant__ CUtensorMap tm_v, const PrefillTcArgs a) {
+                      const __grid_constant__ CUtensorMap tm_v,
+                      const __grid_constant__ CUtensorMap tm_o, const PrefillTcArgs a) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;  // SW128 tiles need 1024-byte alignment
@@ -227,7 +258,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int i = 0; i < tcd::kNumBars; ++i) {
       uint32_t count = 1;
       if (i == tcd::kPFull || i == tcd::kPFull + 1 || i == tcd::kOEmpty || i == tcd::kOEmpty + 1 ||
-          i == tcd::kQReady || i == tcd::kQReady + 1)
+          i == tcd::kQReady || i == tcd::kQReady + 1 || i == tcd::kYReady || i == tcd::kYReady + 1)
         count = 128;
       tc::mbar_init(bar(i), count);
     }
@@ -388,7 +419,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               tc::umma_commit(bar(tcd::kSFull + t));
               if (t == 1) {
                 tc::umma_commit(bar(tcd::kKVEmpty + ks_slot));
-                if (j == w.n_blk - 1) tc::umma_commit(bar(tcd::kQEmpty + qset));
+                if (j == w.n_blk - 1 && !kStage) tc::umma_commit(bar(tcd::kQEmpty + qset));
               }
             }
           }
@@ -402,7 +433,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncwarp();
   } else if (warp == 2) {
     // ------------------------------------------------------------ Q producer
-    // Raw Q tiles of unit n into set n & 1, as soon as unit n - 2 has released the set.
+    // Raw Q tiles of unit n into set n & 1, as soon as unit n - 2 has released the set (its
+    // last Q K^T is done or, when its Y tiles were staged there, their copies have read them).
     asm volatile("setmaxnreg.dec.sync.aligned.u32 56;\n" ::: "memory");
     if (lane == 0) {
       tc::prefetch_tmap(&tm_q);
@@ -426,7 +458,31 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     __syncwarp();
   } else if (warp == 3) {
+    // ------------------------------------------------------------ output store
     asm volatile("setmaxnreg.dec.sync.aligned.u32 56;\n" ::: "memory");
+    if (lane == 0) {
+      tc::prefetch_tmap(&tm_o);
+      bool ok = true;
+      uint32_t ns = 0;   // staged units so far (phases of the kYReady barriers)
+      for (int u = blockIdx.x, n = 0; ok && u < a.n_units; u += gridDim.x, ++n) {
+        if (!kStage) break;
+        const TcUnit w = tc_unit(a, u);
+        const int qset = n & 1;
+        for (int t = 0; t < 2; ++t) {
+          if (!(ok = tc_wait(bar(tcd::kYReady + t), ns & 1u, abort, a.status))) break;
+          if (!w.bad)   // a sequence whose pos0 is out of range is not written
+            for (int hf = 0; hf < 2; ++hf)
+              tc::tma_store_4d(&tm_o, sbase + kTcSmemQ + (qset * 2 + t) * kTcTileBytes + hf * kTcHalfBytes,
+                               hf * 64, 2 * w.pair + t, w.q0, w.b);
+        }
+        tc::bulk_commit_group();
+        tc::bulk_wait_read_all();   // the set may be overwritten once the copies have read it
+        if (ok) tc::mbar_arrive(bar(tcd::kQEmpty + qset));
+        ++ns;
+      }
+      tc::bulk_wait_all();   // the output rows are written before the CTA ends
+    }
+    __syncwarp();
   } else if (warp >= 12) {
     // ------------------------------------------------------------ Q preparation
     // RMSNorm of each raw Q row in shared memory (in place), then RoPE for a local layer;
@@ -646,7 +702,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tc::mbar_arrive(bar(tcd::kPFull + t));
       }
       if (!ok) break;
-      // ---- epilogue: Y = O / l * sigmoid(G + b_h), sigmoid(x) = (1 + tanh(x/2)) / 2.
+      // ---- epilogue: Y = O / l * sigmoid(G + b_h), sigmoid(x) = (1 + tanh(x/2)) / 2, as
+      // bf16 into row r of the unit's Q tile t (128-byte swizzled, as the copies read it)
+      // or, for a unit that is not staged, straight to its output row.
       // The gate row is fetched before the wait for the last P V, to hide its latency.
       const bool valid = tok < a.T;
       const size_t row = ((size_t)w.b * a.T + (valid ? tok : 0)) * (kHq * kD) + (size_t)h * kD;
@@ -660,31 +718,44 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc::tc_fence_after();
       const float inv = 0.5f / l;
       const float hb = 0.5f * a.gate_bias[h];
+      if constexpr (kStage) {
+        // row r of the tile, with the row's swizzle (r % 8) in the chunk bits: the row starts
+        // on a 128-byte boundary, so chunk k sits at yrow ^ (k << 4)
+        const uint32_t yrow =
+            (sbase + kTcSmemQ + ((n & 1) * 2 + t) * kTcTileBytes + r * 128) | ((r & 7) << 4);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t o[32];
-        tc::tmem_ld32(t_o + 32 * c, o);
-        tc::tmem_ld_wait();
-        if (valid) {
-          uint4 *op = reinterpret_cast<uint4 *>(a.out + row + c * 32);
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tc::tmem_ld32(t_o + 32 * c, o);
+          tc::tmem_ld_wait();
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint4 g4 = gr[4 * c + q];
-            const uint32_t gw[4] = {g4.x, g4.y, g4.z, g4.w};
-            uint32_t yw[4];
+          for (int q = 0; q < 4; ++q) {   // d = 32 c + 8 q: half c / 2, chunk 4 (c % 2) + q
+            const uint4 y = gated_y8(gr[4 * c + q], o, q, inv, hb);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(
+                             (yrow ^ (((c & 1) * 4 + q) << 4)) + (c >> 1) * kTcHalfBytes),
+                         "r"(y.x), "r"(y.y), "r"(y.z), "r"(y.w) : "memory");
+          }
+        }
+      } else {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float s0 = 1.0f + tanh_approx(fmaf(0.5f, bf16_lo(gw[e]), hb));
-              const float s1 = 1.0f + tanh_approx(fmaf(0.5f, bf16_hi(gw[e]), hb));
-              yw[e] = pack_bf16(__uint_as_float(o[q * 8 + 2 * e]) * inv * s0,
-                                __uint_as_float(o[q * 8 + 2 * e + 1]) * inv * s1);
-            }
-            op[q] = make_uint4(yw[0], yw[1], yw[2], yw[3]);
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tc::tmem_ld32(t_o + 32 * c, o);
+          tc::tmem_ld_wait();
+          if (valid) {
+            uint4 *op = reinterpret_cast<uint4 *>(a.out + row + c * 32);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) op[q] = gated_y8(gr[4 * c + q], o, q, inv, hb);
           }
         }
       }
       tc::tc_fence_before();
       tc::mbar_arrive(bar(tcd::kOEmpty + t));
+      if constexpr (kStage) {
+        // generic-proxy writes -> visible to the copies' async proxy, then publish the tile
+        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+        tc::mbar_arrive(bar(tcd::kYReady + t));
+      }
     }
   }
 
