@@ -484,6 +484,26 @@ def bench_prefill_chunk(torch, beam, steps, warmup, seed):
     return res
 
 
+def bench_long_global_prefill(torch, beam, steps, warmup, seed, pk):
+    """The long-context global prefill: one global-layer call over B=1, T=131072 (211 TFLOP,
+    a(p) up to p = 131072).  A call runs for about 0.2 s under the power cap, so it is
+    set against the sustained bf16 figure as well as the burst one."""
+    w = wl.workload("long_global_prefill", seed)
+    L = PrefillLayer(torch, beam, wl.GLOBAL, w.B, w.T, w.seed, "bench/long")
+    sec = time_loop(torch, L.run, steps, warmup)
+    assert int(L.status.item()) == 0, "device status set during the long-prefill bench"
+    flops = prefill_flops(w.B, w.T, wl.GLOBAL)
+    tf = flops / sec / 1e12
+    res = {"workload": f"long_global_prefill: B={w.B}, T={w.T}, global layer only",
+           "ms": sec * 1e3, "tflop": flops / 1e12, "tflops": tf,
+           "pct_of_bf16_peak": round(100 * tf / pk["bf16_tflops"], 2),
+           "pct_of_sustained_bf16": round(100 * tf / pk["bf16_tflops_sustained"], 2),
+           "gpu_launches_per_step": L.launches_per_call}
+    del L
+    torch.cuda.empty_cache()
+    return res
+
+
 _CPU_INPUTS = {}
 
 
@@ -698,6 +718,8 @@ def run_gpu(args):
         pc = bench_prefill_chunk(torch, beam, args.steps, args.warmup, args.seed)
         pc["pct_of_bf16_peak"] = round(100 * pc["tflops"] / pk["bf16_tflops"], 2)
         result["prefill_chunk"] = pc
+        result["prefill_long_global"] = bench_long_global_prefill(
+            torch, beam, min(args.steps, 5), args.warmup, args.seed, pk)
     if rank == 0 and world == 1 and not args.no_cpu:
         result["cpu_baseline"] = cpu_baseline_prefill(seed=args.seed)
     if rank == 0:
