@@ -80,16 +80,12 @@ int device_info(DeviceInfo **out) {
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, kDec8Smem),
                           "FP8 decode shared-memory opt-in")))
       return st;
-    if ((st = cuda_status(cudaFuncSetAttribute(prefill_tc_kernel<true>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               kTcSmemBytes),
-                          "prefill shared-memory opt-in")))
-      return st;
-    if ((st = cuda_status(cudaFuncSetAttribute(prefill_tc_kernel<false>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               kTcSmemBytes),
-                          "prefill shared-memory opt-in")))
-      return st;
+    for (auto kernel : {prefill_tc_kernel<true, true>, prefill_tc_kernel<true, false>,
+                        prefill_tc_kernel<false, true>, prefill_tc_kernel<false, false>})
+      if ((st = cuda_status(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 kTcSmemBytes),
+                            "prefill shared-memory opt-in")))
+        return st;
     d.ready = true;
   }
   *out = &d;
@@ -213,10 +209,10 @@ int launch_prefill_attention(int kind, const beam_attn_params *p, int32_t B, int
   if (int st = make_head_map(&tm_o, fa.out, kHq, T, B)) return st;
   // persistent: one CTA per SM (the kernel's shared memory admits one per SM)
   const int grid = (int)std::min<int64_t>(n_units, dev->sm_count);
-  if (kind == BEAM_GLOBAL)
-    prefill_tc_kernel<true><<<grid, kTcThreads, kTcSmemBytes, s>>>(tm_q, tm_k, tm_v, tm_o, fa);
-  else
-    prefill_tc_kernel<false><<<grid, kTcThreads, kTcSmemBytes, s>>>(tm_q, tm_k, tm_v, tm_o, fa);
+  const bool wide = ((reinterpret_cast<uintptr_t>(fa.gate) | reinterpret_cast<uintptr_t>(fa.out)) & 31u) == 0;
+  auto kernel = kind == BEAM_GLOBAL ? (wide ? prefill_tc_kernel<true, true> : prefill_tc_kernel<true, false>)
+                                    : (wide ? prefill_tc_kernel<false, true> : prefill_tc_kernel<false, false>);
+  kernel<<<grid, kTcThreads, kTcSmemBytes, s>>>(tm_q, tm_k, tm_v, tm_o, fa);
   return launch_status();
 }
 

@@ -234,9 +234,11 @@ __device__ __forceinline__ uint4 gated_y8(const uint4 g4, const uint32_t (&o)[32
   return make_uint4(yw[0], yw[1], yw[2], yw[3]);
 }
 
-// kStage: the output goes through shared memory and the store warp (global layer); the
-// two forms are separate instantiations so that each keeps its own register allocation.
-template <bool kStage>
+// kStage: the output goes through shared memory and the store warp (global layer).
+// kWide: the gate and output rows are 32-byte aligned, so each thread moves its row with
+// 32-byte accesses (half the requests of 16-byte ones).  The forms are separate
+// instantiations so that each keeps its own register allocation.
+template <bool kStage, bool kWide>
 
 __global__ void __launch_bounds__(kTcThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -712,7 +714,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       {
         const uint4 *gp = reinterpret_cast<const uint4 *>(a.gate + row);
 #pragma unroll
-        for (int q = 0; q < 16; ++q) gr[q] = valid ? __ldg(gp + q) : make_uint4(0u, 0u, 0u, 0u);
+        if constexpr (kWide) {
+#pragma unroll
+          for (int q = 0; q < 16; q += 2) {
+            if (valid) tc::ld_nc_v8(gp + q, gr[q], gr[q + 1]);
+            else gr[q] = gr[q + 1] = make_uint4(0u, 0u, 0u, 0u);
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 16; ++q) gr[q] = valid ? __ldg(gp + q) : make_uint4(0u, 0u, 0u, 0u);
+        }
       }
       if (!(ok = tc_wait(bar(tcd::kOFull + t), n & 1, abort, a.status))) break;
       tc::tc_fence_after();
@@ -745,7 +756,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (valid) {
             uint4 *op = reinterpret_cast<uint4 *>(a.out + row + c * 32);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) op[q] = gated_y8(gr[4 * c + q], o, q, inv, hb);
+            for (int q = 0; q < 4; q += 2) {
+              const uint4 y0 = gated_y8(gr[4 * c + q], o, q, inv, hb);
+              const uint4 y1 = gated_y8(gr[4 * c + q + 1], o, q + 1, inv, hb);
+              if constexpr (kWide) {
+                tc::st_v8(op + q, y0, y1);
+              } else {
+                op[q] = y0;
+                op[q + 1] = y1;
+              }
+            }
           }
         }
       }

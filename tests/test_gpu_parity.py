@@ -94,6 +94,40 @@ def test_prefill_tiny_workload_all_rows(env, kind):
     assert_close(host_bits(out).reshape(ref.shape), ref, f"tiny kind={kind}")
 
 
+@pytest.mark.parametrize("kind", [wl.LOCAL, wl.GLOBAL])
+def test_prefill_gate_and_output_only_16_byte_aligned(env, kind):
+    """Gate and output buffers that start 16 bytes past a 32-byte boundary (the API asks
+    for 16): the kernel then moves those rows with 16-byte accesses instead of 32-byte
+    ones.  Every output element against the oracle, and the guard words around the
+    output untouched."""
+    torch, beam, orc = env
+    B, T = 1, 300
+    inp = wl.prefill_inputs(B, T, 97, layer=f"align{kind}")
+    params = beam.default_params()
+    n = B * T * 48 * 128
+    q, k, v = (dev(torch, x) for x in (inp.q, inp.k, inp.v))
+    gbuf = torch.zeros(n + 16, dtype=torch.bfloat16, device="cuda")
+    gbuf[8:8 + n].copy_(dev(torch, inp.gate).reshape(-1))
+    obuf = torch.full((n + 16,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    obuf[:8] = 3.0
+    obuf[8 + n:] = 3.0
+    g, out = gbuf[8:8 + n], obuf[8:8 + n]
+    assert g.data_ptr() % 32 == 16 and out.data_ptr() % 32 == 16
+    qw = torch.from_numpy(inp.q_norm_w).cuda()
+    kw = torch.from_numpy(inp.k_norm_w).cuda()
+    bias = torch.from_numpy(inp.gate_bias).cuda()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    beam.beam_attn_prefill(kind, params, q, k, v, g, qw, kw, bias, out, None, None, None,
+                           dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    guard = host_bits(torch.cat([obuf[:8], obuf[8 + n:]]))
+    assert (guard == host_bits(torch.full((16,), 3.0, dtype=torch.bfloat16))).all()
+    ref = orc.prefill(kind, oracle_params(orc, params), inp.q, inp.k, inp.v, inp.gate,
+                      inp.q_norm_w, inp.k_norm_w, inp.gate_bias)
+    assert_close(host_bits(out).reshape(ref.shape), ref, f"16-byte aligned kind={kind}")
+
+
 @pytest.mark.parametrize("kind,B,T,window", [
     (wl.LOCAL, 2, 333, 512), (wl.GLOBAL, 2, 333, 512), (wl.LOCAL, 1, 1000, 100),
     (wl.LOCAL, 1, 700, 64), (wl.GLOBAL, 3, 1, 512), (wl.LOCAL, 1, 1, 1), (wl.LOCAL, 1, 130, 1),
