@@ -235,8 +235,8 @@ __device__ __forceinline__ uint4 gated_y8(const uint4 g4, const uint32_t (&o)[32
 }
 
 // kStage: the output goes through shared memory and the store warp (global layer).
-// kWide: the gate and output rows are 32-byte aligned, so each thread moves its row with
-// 32-byte accesses (half the requests of 16-byte ones).  The forms are separate
+// kWide: the gate, output and RoPE-table rows are 32-byte aligned, so each thread moves
+// its row with 32-byte accesses (half the requests of 16-byte ones).  The forms are separate
 // instantiations so that each keeps its own register allocation.
 template <bool kStage, bool kWide>
 
@@ -504,10 +504,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 : nullptr;
       float4 tb[8];   // per slot: cos lo, cos hi, sin lo, sin hi of one chunk of 8
       auto tab_load = [&](int c, int slot) {
-        tb[4 * slot + 0] = __ldg(tab + 2 * c);
-        tb[4 * slot + 1] = __ldg(tab + 2 * c + 1);
-        tb[4 * slot + 2] = __ldg(tab + 16 + 2 * c);
-        tb[4 * slot + 3] = __ldg(tab + 16 + 2 * c + 1);
+        if constexpr (kWide) {
+          tc::ld_nc_v8(tab + 2 * c, tb[4 * slot + 0], tb[4 * slot + 1]);
+          tc::ld_nc_v8(tab + 16 + 2 * c, tb[4 * slot + 2], tb[4 * slot + 3]);
+        } else {
+          tb[4 * slot + 0] = __ldg(tab + 2 * c);
+          tb[4 * slot + 1] = __ldg(tab + 2 * c + 1);
+          tb[4 * slot + 2] = __ldg(tab + 16 + 2 * c);
+          tb[4 * slot + 3] = __ldg(tab + 16 + 2 * c + 1);
+        }
       };
       if (local) {
         tab_load(0, 0);
@@ -713,7 +718,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       uint4 gr[16];
       {
         const uint4 *gp = reinterpret_cast<const uint4 *>(a.gate + row);
-#pragma unroll
         if constexpr (kWide) {
 #pragma unroll
           for (int q = 0; q < 16; q += 2) {
