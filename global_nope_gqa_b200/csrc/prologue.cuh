@@ -9,11 +9,12 @@
 //
 // One CTA of 128 threads per token.  Each half-warp owns one 128-wide row:
 // lane l (0..15) holds coordinates 8l .. 8l+7 as one 16-byte load, so the
-// rotate-half partner of lane l is lane l ^ 8.  The 64 RoPE angles of a token
-// are formed once per lane in fp64 (t * frequency, then reduced to [-pi, pi]),
-// because in fp32 t * frequency is off by up to ~0.06 rad at t ~ 1e6; the
-// reduced angle then goes through fp32 sincosf.  Rows: 48 query heads, 8 key
-// heads, and 8 value heads when a cache is written (copied unchanged).
+// rotate-half partner of lane l is lane l ^ 8.  Each of the 64 RoPE angles of a
+// token is formed once, by one thread, in fp64 (t * frequency, then reduced to
+// [-pi, pi]), because in fp32 t * frequency is off by up to ~0.06 rad at t ~ 1e6;
+// the reduced angle then goes through fp32 sincosf, and the cos / sin values reach
+// the other threads through shared memory.  Rows: 48 query heads, 8 key heads, and
+// 8 value heads when a cache is written (copied unchanged).
 #pragma once
 
 #include "common.cuh"
@@ -48,19 +49,22 @@ struct PrologueArgs {
   double inv_freq[64];   // theta^(-2i/128), formed on the host in double
 };
 
-// cos / sin of the angles t * f_i, i = 8 sub .. 8 sub + 7, formed and reduced to [-pi, pi]
-// in fp64, then evaluated in fp32.
-__device__ __forceinline__ void rope_angles(const double *inv_freq, int64_t t, int sub,
-                                            float (&cs)[8], float (&sn)[8]) {
+// cos / sin of the angle t * f, formed and reduced to [-pi, pi] in fp64, then evaluated
+// in fp32.
+__device__ __forceinline__ void rope_angle(double f, int64_t t, float &cs, float &sn) {
   const double two_pi = 6.283185307179586;
   const double inv_two_pi = 0.15915494309189535;
+  const double phi = (double)t * f;
+  const double n = rint(phi * inv_two_pi);
+  const double r = fma(-n, two_pi, phi);  // |r| <= pi (+ rounding)
+  sincosf((float)r, &sn, &cs);
+}
+
+// The angles t * f_i, i = 8 sub .. 8 sub + 7.
+__device__ __forceinline__ void rope_angles(const double *inv_freq, int64_t t, int sub,
+                                            float (&cs)[8], float (&sn)[8]) {
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    double phi = (double)t * inv_freq[sub * 8 + e];
-    double n = rint(phi * inv_two_pi);
-    double r = fma(-n, two_pi, phi);  // |r| <= pi (+ rounding)
-    sincosf((float)r, &sn[e], &cs[e]);
-  }
+  for (int e = 0; e < 8; ++e) rope_angle(inv_freq[sub * 8 + e], t, cs[e], sn[e]);
 }
 
 // RMSNorm of one 128-wide row held by a half-warp (lane l16 holds coordinates
@@ -147,17 +151,32 @@ __global__ void __launch_bounds__(128) prologue_kernel(const PrologueArgs a) {
     }
   }
 
+  // The token's 64 angles, one per thread of warps 0-1, shared through shared memory: every
+  // row of the token uses the same angles (and, for the table at positions 0 .. T-1,
+  // every sequence).
+  __shared__ float4 s_cs[16], s_sn[16];
   float cs[8], sn[8];
-  if (local) rope_angles(a.inv_freq, t < 0 ? 0 : t, l16 & 7, cs, sn);
-  if (local && a.rope_tab && (a.rope_per_seq || b == 0) && warp == 0 && lane < 8) {
-    // the angles serve every head (and, at positions 0 .. T-1, every sequence)
-    const size_t trow = (size_t)(a.rope_per_seq ? tok : i) * 128;
-    float4 *c4 = reinterpret_cast<float4 *>(a.rope_tab + trow + lane * 8);
-    float4 *s4 = reinterpret_cast<float4 *>(a.rope_tab + trow + 64 + lane * 8);
-    c4[0] = make_float4(cs[0], cs[1], cs[2], cs[3]);
-    c4[1] = make_float4(cs[4], cs[5], cs[6], cs[7]);
-    s4[0] = make_float4(sn[0], sn[1], sn[2], sn[3]);
-    s4[1] = make_float4(sn[4], sn[5], sn[6], sn[7]);
+  if (local) {
+    if (threadIdx.x < 64) {
+      const int f = threadIdx.x;
+      float c, s;
+      rope_angle(a.inv_freq[f], t < 0 ? 0 : t, c, s);
+      reinterpret_cast<float *>(s_cs)[f] = c;
+      reinterpret_cast<float *>(s_sn)[f] = s;
+      if (a.rope_tab && (a.rope_per_seq || b == 0)) {
+        const size_t trow = (size_t)(a.rope_per_seq ? tok : i) * 128;
+        a.rope_tab[trow + f] = c;
+        a.rope_tab[trow + 64 + f] = s;
+      }
+    }
+    __syncthreads();
+    const int sub = l16 & 7;   // coordinates 8 l16 .. 8 l16 + 7 use angles 8 sub .. 8 sub + 7
+    const float4 c0 = s_cs[2 * sub], c1 = s_cs[2 * sub + 1];
+    const float4 s0 = s_sn[2 * sub], s1 = s_sn[2 * sub + 1];
+    cs[0] = c0.x; cs[1] = c0.y; cs[2] = c0.z; cs[3] = c0.w;
+    cs[4] = c1.x; cs[5] = c1.y; cs[6] = c1.z; cs[7] = c1.w;
+    sn[0] = s0.x; sn[1] = s0.y; sn[2] = s0.z; sn[3] = s0.w;
+    sn[4] = s1.x; sn[5] = s1.y; sn[6] = s1.z; sn[7] = s1.w;
   }
 
   float wq[8], wk[8];
