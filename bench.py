@@ -364,8 +364,8 @@ class ChunkLayer:
         self.flops = vis * HEAD_FLOPS_PER_PAIR
         ctx = [pos0 + T]
         self.bytes = decode_kv_bytes(ctx, kind) + (T - 1) * 2 * 2 * (3 * 6144 + 2 * 1024)
-        # local: ring copy + prologue + split-K + combine; global: prologue + split-K + combine
-        self.launches_per_call = 4 if kind == wl.LOCAL else 3
+        # ring copy (local) or value padding (global), prologue, split-K attention, merge
+        self.launches_per_call = 4
 
     def run(self):
         self.beam.beam_attn_prefill_chunk(self.kind, self.params, self.q, self.k, self.v, self.gate,
@@ -735,11 +735,14 @@ def run_decode_case(args):
     torch.cuda.set_device(0)
     import global_nope_gqa_b200 as beam
     beam.lib()
-    if args.decode_case == "multi8":
-        L = ChunkLayer(torch, beam, wl.GLOBAL, 8, args.context - 8, args.context, args.seed, "case")
+    if args.decode_case in ("multi8", "multi8_local"):
+        glob = args.decode_case == "multi8"
+        kind, slots = (wl.GLOBAL, args.context) if glob else (wl.LOCAL, wl.WINDOW)
+        L = ChunkLayer(torch, beam, kind, 8, args.context - 8, slots, args.seed, "case")
         sec = time_loop(torch, L.run, args.steps, args.warmup)
         assert int(L.status.item()) == 0
-        print(json.dumps({"case": f"global chunk of 8 new tokens, B=1, context {args.context}",
+        print(json.dumps({"case": f"{'global' if glob else 'local'} chunk of 8 new tokens, B=1, "
+                                  f"context {args.context}",
                           "ms": sec * 1e3, "GBps": L.bytes / sec / 1e9}), flush=True)
         return
     fp8 = args.decode_case == "fp8"
@@ -791,7 +794,7 @@ def main(argv=None):
     ap.add_argument("--layers", default="both", choices=["both", "global", "local"],
                     help="prefill layers per step (profiling cases; the headline step is both)")
     ap.add_argument("--batch", type=int, default=0, help="override B (profiling cases)")
-    ap.add_argument("--decode-case", choices=["bf16", "fp8", "multi8"], default=None,
+    ap.add_argument("--decode-case", choices=["bf16", "fp8", "multi8", "multi8_local"], default=None,
                     help="profiling case: time one global decode call at --context only")
     ap.add_argument("--context", type=int, default=wl.MAX_CONTEXT)
     args = ap.parse_args(argv)

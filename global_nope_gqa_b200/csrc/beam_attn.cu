@@ -560,6 +560,12 @@ int beam_attn_prefill_chunk(int kind, const beam_attn_params *p, int32_t B, int3
     da.part_ml = reinterpret_cast<float *>(pw + round_up(parts * kD * 4, 256));
     da.status = dev_status;
     da.kv_slot_major = local ? 0 : 1;
+    // a plan with one split (many sequences, or a short history) needs no merge: the CTA
+    // that sees every key of its (sequence, KV head) writes the gated output itself
+    da.direct = mp.n_split_max == 1;
+    da.gate = static_cast<const uint16_t *>(gate);
+    da.gate_bias = gate_bias;
+    da.out = static_cast<uint16_t *>(out);
     {  // the same test-only fault injection as the prefill kernel's
       const char *f = std::getenv("BEAM_FAULT_INJECT");
       da.fault_stall = f != nullptr && std::strcmp(f, "prefill_wait_stall") == 0;
@@ -567,6 +573,7 @@ int beam_attn_prefill_chunk(int kind, const beam_attn_params *p, int32_t B, int3
     if (mp.n_split_max > 65535 || B > 65535) return BEAM_ERR_UNSUPPORTED;
     decode_tc_kernel<<<dim3(mp.n_split_max, kHkv, B), kDtThreads, kDtSmemBytes, s>>>(tk, tv, da);
     if ((st = launch_status())) return st;
+    if (da.direct) return BEAM_OK;
     MultiCombineArgs mc;
     mc.part_o = da.part_o;
     mc.part_ml = da.part_ml;

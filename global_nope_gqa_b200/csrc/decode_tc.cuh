@@ -64,6 +64,12 @@ struct DecodeTcArgs {
   int split, n_split_max, n_mt;   // split: key coordinates per CTA, a multiple of 128
   float scale_log2, ssmax_base, ssmax_exp;
   float *part_o, *part_ml;    // the layout decode_multi_combine_kernel reads
+  // direct != 0: one CTA covers all of a sequence's keys for its KV head (n_split_max == 1),
+  // so it writes Y = O / l * sigmoid(G + b_h) itself and no merge runs
+  int direct;
+  const uint16_t *gate;       // [B][T][48*128]
+  const float *gate_bias;     // [48]
+  uint16_t *out;              // [B][T][48*128]
   int32_t *status;
   int kv_slot_major;          // K/V maps take (d, slot, head, b) rather than (d, head, t, b)
   int fault_stall;            // tests only: the MMA issuer first waits on a barrier never arrived at
@@ -389,10 +395,44 @@ __global__ void __launch_bounds__(kDtThreads, 1)
       tc::tc_fence_before();
       tc::mbar_arrive(bar(dtd::kPFull + (j & 1)));
     }
+    if (ok) ok = tc_wait(bar(dtd::kOFull), 0u, abort, a.status);
+    if (a.direct) {
+      // the whole key range: Y = O / l * sigmoid(G + b_h) straight to the output row (not
+      // written when a wait ran out)
+      if (ok) {
+        tc::tc_fence_after();
+        const int h = g * kGroup + hh;
+        const size_t orow = (((size_t)b * a.T + (row_ok ? tok : 0)) * kHq + h) * kD;
+        const uint4 *gp = reinterpret_cast<const uint4 *>(a.gate + orow);
+        uint4 *op = reinterpret_cast<uint4 *>(a.out + orow);
+        const float inv = 1.0f / l, bias = a.gate_bias[h];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tc::tmem_ld32(t_o + 32 * c, o);
+          tc::tmem_ld_wait();
+          if (row_ok) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint4 g4 = __ldg(gp + 4 * c + q);
+              const uint32_t gw[4] = {g4.x, g4.y, g4.z, g4.w};
+              uint32_t yw[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float y0 = __uint_as_float(o[8 * q + 2 * e]) * inv / (1.0f + expf(-(bf16_lo(gw[e]) + bias)));
+                const float y1 = __uint_as_float(o[8 * q + 2 * e + 1]) * inv / (1.0f + expf(-(bf16_hi(gw[e]) + bias)));
+                yw[e] = pack_bf16(y0, y1);
+              }
+              op[4 * c + q] = make_uint4(yw[0], yw[1], yw[2], yw[3]);
+            }
+          }
+        }
+      }
+      ok = false;   // nothing more to write
+    }
     const int mt = tok / kMultiTokPerTile, row16 = (tok % kMultiTokPerTile) * kGroup + hh;
     const size_t part = ((((size_t)b * kHkv + g) * a.n_mt + mt) * a.n_split_max + s_idx) * 16 + row16;
-    if (ok) ok = tc_wait(bar(dtd::kOFull), 0u, abort, a.status);
-    if (!ok && row_ok) {   // a wait ran out: the merge turns these rows into NaN
+    if (!ok && row_ok && !a.direct) {   // a wait ran out: the merge turns these rows into NaN
       a.part_ml[part * 2] = __int_as_float(0x7fc00000);
       a.part_ml[part * 2 + 1] = __int_as_float(0x7fc00000);
     }

@@ -165,9 +165,10 @@ BEAM_API size_t beam_prefill_chunk_workspace_bytes(int kind, const beam_attn_par
  * in dev_status and is neither appended nor written to `out`; the others are
  * unaffected.  T > slots_per_seq (global) is BEAM_ERR_CAPACITY before any launch.
  * Up to 16 new tokens (multi-token decode, e.g. verifying a drafted block) run on
- * a split-K tcgen05 kernel that spreads the history over many CTAs; longer chunks
- * on the tcgen05 prefill kernel.  The bounded waits of both behave as in
- * beam_attn_prefill. */
+ * a split-K tcgen05 kernel that spreads the history over many CTAs and a merge
+ * kernel; when the plan gives each (sequence, KV head) a single CTA (many
+ * sequences, or a short history) that CTA applies the gate and writes `out`
+ * itself.  Longer chunks run on the tcgen05 prefill kernel.  The bounded waits of both behave as in beam_attn_prefill. */
 BEAM_API int beam_attn_prefill_chunk(int kind, const beam_attn_params *p, int32_t B, int32_t T,
                                      const void *q, const void *k, const void *v, const void *gate,
                                      const float *q_norm_w, const float *k_norm_w,

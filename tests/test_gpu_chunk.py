@@ -88,11 +88,13 @@ def check_cache(orc, ci, params, kc, vc, skip=()):
     (wl.GLOBAL, [5], 1, 512, 64),
     (wl.GLOBAL, [4000], 130, 512, 4200),          # padding stops at the capacity
     (wl.GLOBAL, [1, 128, 255], 128, 512, 640),
-    # up to 16 new tokens: the split-K multi-token decode path
+    # up to 16 new tokens: the multi-token decode path (one CTA per KV head writing the
+    # gated output when the keys fit it, else split-K partials and a merge)
     (wl.LOCAL, [0, 100, 2000], 8, 512, 512),
     (wl.LOCAL, [37, 5], 3, 100, 100),
     (wl.LOCAL, [3], 16, 1, 1),
     (wl.LOCAL, [510, 511, 520], 16, 512, 512),
+    (wl.LOCAL, [3000, 700], 8, 2048, 2048),       # a wider window: more splits per head
     (wl.GLOBAL, [0, 1000, 127], 16, 512, 2048),
     (wl.GLOBAL, [0, 4090], 5, 512, 4096),
     (wl.GLOBAL, [70000], 2, 512, 70002),
