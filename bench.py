@@ -505,12 +505,17 @@ def bench_long_global_prefill(torch, beam, steps, warmup, seed, pk):
 
 
 _CPU_INPUTS = {}
+PREFILL_WORKLOAD = ("batched_prefill: B={B}, T={T} per GPU, layers={layers} (local: window 512, "
+                    "RoPE; global: NoPE, SSMax), 48 q / 8 kv heads, d=128, fused KV append")
 
 
 def cpu_baseline_prefill(seconds_target=10.0, seconds_cap=30.0, seed=1234):
     """The fp64 oracle, as it stands, on a bounded row sample of the batched-prefill
-    workload (global layer: rows drawn uniformly from 0..8191 of 4 sequences, all 48
-    heads).  Returns TFLOP/s of algorithmic work and the sample description."""
+    workload (B=4, T=8192, both layers): query rows drawn uniformly from 0..8191 of the 4
+    sequences, all 48 heads, alternately from the global and the local layer.  Each layer's
+    rate (algorithmic FLOPs of its sampled rows / its time) is measured separately, and the
+    step's rate combines them by the step's FLOPs: (F_g + F_l) / (F_g / r_g + F_l / r_l).
+    Returns TFLOP/s and the sample description."""
     import oracle
     P = oracle.params()
     B, T = 4, 8192
@@ -521,21 +526,34 @@ def cpu_baseline_prefill(seconds_target=10.0, seconds_cap=30.0, seed=1234):
     inp = _CPU_INPUTS[key]
     rng = np.random.default_rng(seed)
     threads = oracle.n_threads_default()
-    done_flops, done_rows, t0 = 0, 0, time.perf_counter()
+    kinds = ((oracle.GLOBAL, wl.GLOBAL), (oracle.LOCAL, wl.LOCAL))
+    flops = {kw: 0 for _, kw in kinds}
+    secs = {kw: 0.0 for _, kw in kinds}
+    rows = {kw: 0 for _, kw in kinds}
     batch = max(8, threads)
+    t0 = time.perf_counter()
     while True:
-        rb = rng.integers(0, B, size=batch)
-        rt = rng.integers(0, T, size=batch)
-        oracle.prefill_rows(oracle.GLOBAL, P, inp.q, inp.k, inp.v, inp.gate, inp.q_norm_w,
-                            inp.k_norm_w, inp.gate_bias, rb, rt, n_threads=threads)
-        done_flops += int((rt + 1).sum()) * HEAD_FLOPS_PER_PAIR
-        done_rows += batch
+        for ko, kw in kinds:
+            rb = rng.integers(0, B, size=batch)
+            rt = rng.integers(0, T, size=batch)
+            t1 = time.perf_counter()
+            oracle.prefill_rows(ko, P, inp.q, inp.k, inp.v, inp.gate, inp.q_norm_w, inp.k_norm_w,
+                                inp.gate_bias, rb, rt, n_threads=threads)
+            secs[kw] += time.perf_counter() - t1
+            vis = rt + 1 if kw == wl.GLOBAL else np.minimum(rt + 1, wl.WINDOW)
+            flops[kw] += int(vis.sum()) * HEAD_FLOPS_PER_PAIR
+            rows[kw] += batch
         el = time.perf_counter() - t0
         if el >= seconds_target or el >= seconds_cap:
             break
-    return {"value": done_flops / el / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-            "sample": f"{done_rows} query rows x 48 heads of the global layer of batched_prefill "
-                      f"(B=4, T=8192), uniform row positions; {el:.1f} s"}
+    step = {kw: prefill_flops(B, T, kw) for _, kw in kinds}
+    est = sum(step[kw] / (flops[kw] / secs[kw]) for _, kw in kinds)   # oracle seconds per step
+    return {"value": sum(step.values()) / est / 1e12, "unit": "TFLOP/s", "cores": threads,
+            "kind": "oracle",
+            "sample": f"{rows[wl.GLOBAL]} global-layer and {rows[wl.LOCAL]} local-layer query rows "
+                      f"x 48 heads of batched_prefill (B=4, T=8192), uniform row positions, "
+                      f"{secs[wl.GLOBAL]:.1f} s + {secs[wl.LOCAL]:.1f} s; step rate = the two "
+                      "layers' rates combined by the step's FLOPs"}
 
 
 def e2e_prefill(torch, beam, layers, steps, warmup):
@@ -681,9 +699,7 @@ def run_gpu(args):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic: N(0,1) bf16 activations drawn on the device (seeded torch Philox)",
-        "config": {"workload": f"batched_prefill: B={w.B}, T={w.T} per GPU, layers={args.layers} "
-                               "(local: window 512, RoPE; global: NoPE, SSMax), 48 q / 8 kv heads, "
-                               "d=128, fused KV append",
+        "config": {"workload": PREFILL_WORKLOAD.format(B=w.B, T=w.T, layers=args.layers),
                    "global_batch": w.B * world, "seq_len": w.T, "parallelism": f"dp{world}",
                    "l2": "inputs larger than L2 (Q alone is 403 MB per layer)"},
         "pct_of_bf16_peak": round(100 * value / world / pk["bf16_tflops"], 2),
@@ -772,8 +788,9 @@ def run_reference(args):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic: N(0,1) bf16 activations (seeded numpy Philox)",
-        "config": {"workload": "batched_prefill: B=4, T=8192, global layer row sample",
-                   "global_batch": 4, "seq_len": 8192, "parallelism": "none (host cores)"},
+        "config": {"workload": PREFILL_WORKLOAD.format(B=4, T=8192, layers="both"),
+                   "global_batch": 4, "seq_len": 8192, "parallelism": "none (host cores)",
+                   "sample": "query rows of both layers, see cpu_baseline"},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": base["cores"],
                          "kind": "oracle", "sample": base["sample"]},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
