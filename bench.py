@@ -364,8 +364,8 @@ class ChunkLayer:
         self.flops = vis * HEAD_FLOPS_PER_PAIR
         ctx = [pos0 + T]
         self.bytes = decode_kv_bytes(ctx, kind) + (T - 1) * 2 * 2 * (3 * 6144 + 2 * 1024)
-        # ring copy (local) or value padding (global), prologue, split-K attention, merge
-        self.launches_per_call = 4
+        # prologue (with the ring copy or the value padding), split-K attention, merge
+        self.launches_per_call = 3
 
     def run(self):
         self.beam.beam_attn_prefill_chunk(self.kind, self.params, self.q, self.k, self.v, self.gate,
@@ -478,7 +478,7 @@ def bench_prefill_chunk(torch, beam, steps, warmup, seed):
         calls.append((sec, flops))
     assert int(status.item()) == 0, "device status set during the chunked-prefill bench"
     res["tflops"] = sum(f for _, f in calls) / sum(s for s, _ in calls) / 1e12
-    res["gpu_launches_per_step"] = 6   # per layer: ring copy or value padding, prologue, attention
+    res["gpu_launches_per_step"] = 4   # per layer: prologue (with the ring copy or padding), attention
     del x, out
     torch.cuda.empty_cache()
     return res

@@ -470,7 +470,8 @@ int beam_attn_prefill_chunk(int kind, const beam_attn_params *p, int32_t B, int3
                           : nullptr;
   const int prefix = local ? p->window - 1 : 0;
 
-  // 1. the ring rows the chunk still sees (local), or the value padding (global)
+  // the ring rows the chunk still sees (local), or the value padding (global): extra CTAs of
+  // the prologue launch
   ChunkPrepArgs ca;
   ca.pos0 = pos0;
   ca.k_cache = static_cast<const uint16_t *>(k_cache);
@@ -486,12 +487,8 @@ int beam_attn_prefill_chunk(int kind, const beam_attn_params *p, int32_t B, int3
   ca.window = p->window;
   ca.kind = kind;
   const int64_t prep_ctas = (int64_t)B * (local ? prefix : kChunkPadRows);
-  if (prep_ctas > 0) {
-    chunk_prep_kernel<<<(unsigned)prep_ctas, 128, 0, s>>>(ca);
-    if ((st = launch_status())) return st;
-  }
 
-  // 2. prepared keys (and raw values) of the new tokens: into the cache and, for a local
+  // 1. prepared keys (and raw values) of the new tokens: into the cache and, for a local
   //    layer, behind the earlier rows; the RoPE table at each sequence's own positions
   PrologueArgs pa;
   memset(&pa, 0, sizeof pa);
@@ -518,10 +515,14 @@ int beam_attn_prefill_chunk(int kind, const beam_attn_params *p, int32_t B, int3
   pa.window = p->window;
   pa.eps = p->rms_eps;
   fill_inv_freq(pa.inv_freq, p->rope_theta);
-  prologue_kernel<<<(unsigned)((size_t)B * T), 128, 0, s>>>(pa);
+  pa.prep = ca;
+  pa.n_prep = (int)prep_ctas;
+  pa.ring_save = local;
+  if ((int64_t)B * T + prep_ctas > INT32_MAX) return BEAM_ERR_UNSUPPORTED;
+  prologue_kernel<<<(unsigned)((int64_t)B * T + prep_ctas), 128, 0, s>>>(pa);
   if ((st = launch_status())) return st;
 
-  // 3. attention of the new rows over the earlier and the new keys
+  // 2. attention of the new rows over the earlier and the new keys
   if (T <= kMultiMaxT) {
     // a few new tokens (multi-token decode): split the keys across CTAs, then merge
     const MultiPlan mp = multi_plan(kind, p, B, T, layout->slots_per_seq, dev->sm_count);

@@ -21,6 +21,58 @@
 
 namespace beam {
 
+// Before the prologue of a chunked prefill (positions pos0[b] .. pos0[b] + T - 1 after
+// pos0[b] cached tokens).  Local layer: rows e = 0 .. L-1 (L = window - 1) of each
+// sequence's key and value buffers get the ring's rows of positions pos0[b] - L + e, i.e.
+// the earlier keys still inside the window of the chunk's first token, zeros before
+// position 0.  Ring slots the chunk's own tokens overwrite are saved by those tokens' CTAs
+// just before they write them (no other CTA reads or writes such a slot).  Global layer: the
+// value slots from pos0[b] + T up to the next multiple of 128 (within the capacity) are
+// zeroed: the attention kernel reads whole 128-key blocks, and a masked key's weight is
+// exactly 0 but 0 times a non-finite stale value would not be.  Run as extra CTAs of the
+// prologue launch, one CTA of 128 threads per row; thread x moves 8 coordinates of head
+// x / 16.
+constexpr int kChunkPadRows = 128;  // global: CTAs per sequence (at most 127 slots to zero)
+
+struct ChunkPrepArgs {
+  const int64_t *pos0;
+  const uint16_t *k_cache;
+  uint16_t *v_cache;
+  int64_t stride_seq, stride_head, slots;
+  uint16_t *k_ext, *v_ext;   // local: [B][ext_rows][8*128]
+  int ext_rows, prefix, T, window, kind;
+};
+
+__device__ __forceinline__ void chunk_prep_row(const ChunkPrepArgs &a, int cta) {
+  const int per_b = a.kind == BEAM_LOCAL ? a.prefix : kChunkPadRows;
+  const int b = cta / per_b, e = cta - b * per_b;
+  const int head = threadIdx.x >> 4, c = (threadIdx.x & 15) * 8;
+  const int64_t p0 = a.pos0[b];
+  const size_t cache_row = (size_t)b * a.stride_seq + (size_t)head * a.stride_head;
+  if (a.kind == BEAM_LOCAL) {
+    // the token i of this call with i % window == e + 1 that enters the ring takes the slot of
+    // position p0 - L + e and saves that row itself before overwriting it; the tokens that
+    // enter are T - window .. T - 1 (all of them when T < window), so one exists when T >=
+    // window, else when e + 1 <= T - 1
+    if (p0 >= 0 && (a.T >= a.window || e + 1 <= a.T - 1)) return;
+    const int64_t j = p0 - a.prefix + e;
+    uint4 kv = make_uint4(0u, 0u, 0u, 0u), vv = kv;
+    if (p0 >= 0 && j >= 0) {
+      const size_t off = cache_row + (size_t)(j % a.window) * kD + c;
+      kv = *reinterpret_cast<const uint4 *>(a.k_cache + off);
+      vv = *reinterpret_cast<const uint4 *>(a.v_cache + off);
+    }
+    const size_t dst = ((size_t)b * a.ext_rows + e) * (kHkv * kD) + head * kD + c;
+    *reinterpret_cast<uint4 *>(a.k_ext + dst) = kv;
+    *reinterpret_cast<uint4 *>(a.v_ext + dst) = vv;
+  } else {
+    const int64_t end = p0 + a.T, slot = end + e;
+    if (p0 < 0 || end > a.slots || slot >= a.slots || slot >= (end + 127) / 128 * 128) return;
+    *reinterpret_cast<uint4 *>(a.v_cache + cache_row + (size_t)slot * kD + c) =
+        make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
 struct PrologueArgs {
   const uint16_t *q;     // [tokens][48*128] or null (append only)
   const uint16_t *k;     // [tokens][8*128]
@@ -43,6 +95,11 @@ struct PrologueArgs {
   float inv_k_scale, inv_v_scale;
   int32_t *status;
   int T;                 // tokens per sequence in this call
+  // chunked prefill: n_prep extra CTAs after the B * T token CTAs prepare the chunk (the
+  // ring rows it still sees, or the value padding); ring_save: a token that takes the ring
+  // slot of one of those rows copies the row out first
+  ChunkPrepArgs prep;
+  int n_prep, ring_save;
   int kind;
   int window;
   float eps;
@@ -117,6 +174,11 @@ __device__ __forceinline__ void load_weights8(const float *w, int l16, float (&o
 }
 
 __global__ void __launch_bounds__(128) prologue_kernel(const PrologueArgs a) {
+  const int n_tok = (int)gridDim.x - a.n_prep;
+  if ((int)blockIdx.x >= n_tok) {   // a chunk-preparation CTA (the whole CTA returns)
+    chunk_prep_row(a.prep, (int)blockIdx.x - n_tok);
+    return;
+  }
   const int tok = blockIdx.x;
   const int b = tok / a.T;
   const int i = tok - b * a.T;
@@ -225,55 +287,22 @@ __global__ void __launch_bounds__(128) prologue_kernel(const PrologueArgs a) {
               f32x8_to_e4m3(x, is_k ? a.inv_k_scale : a.inv_v_scale);
         } else {
           uint16_t *cache = is_k ? a.k_cache : a.v_cache;
+          const int r = a.ring_save ? i % a.window : 0;
+          if (r >= 1) {
+            // before this call the slot held position q = pos0 + r - window, row r - 1 of the
+            // earlier keys the chunk still sees: save it (zeros before position 0) before
+            // overwriting it
+            const int64_t q = (t - i) + r - a.window;
+            const uint4 old = q >= 0 ? *reinterpret_cast<const uint4 *>(cache + off)
+                                     : make_uint4(0u, 0u, 0u, 0u);
+            uint16_t *ext = is_k ? a.k_out : a.v_out;
+            *reinterpret_cast<uint4 *>(ext + ((size_t)b * a.out_rows + r - 1) * (kHkv * kD) +
+                                       head * kD + l16 * 8) = old;
+          }
           *reinterpret_cast<uint4 *>(cache + off) = res;
         }
       }
     }
-  }
-}
-
-// Before the prologue of a chunked prefill (positions pos0[b] .. pos0[b] + T - 1 after
-// pos0[b] cached tokens).  Local layer: rows e = 0 .. L-1 (L = window - 1) of each
-// sequence's key and value buffers get the ring's rows of positions pos0[b] - L + e, i.e.
-// the earlier keys still inside the window of the chunk's first token, zeros before
-// position 0; this must run before the prologue overwrites ring slots.  Global layer: the
-// value slots from pos0[b] + T up to the next multiple of 128 (within the capacity) are
-// zeroed: the attention kernel reads whole 128-key blocks, and a masked key's weight is
-// exactly 0 but 0 times a non-finite stale value would not be.  One CTA of 128 threads
-// per row; thread x moves 8 coordinates of head x / 16.
-constexpr int kChunkPadRows = 128;  // global: CTAs per sequence (at most 127 slots to zero)
-
-struct ChunkPrepArgs {
-  const int64_t *pos0;
-  const uint16_t *k_cache;
-  uint16_t *v_cache;
-  int64_t stride_seq, stride_head, slots;
-  uint16_t *k_ext, *v_ext;   // local: [B][ext_rows][8*128]
-  int ext_rows, prefix, T, window, kind;
-};
-
-__global__ void __launch_bounds__(128) chunk_prep_kernel(const ChunkPrepArgs a) {
-  const int per_b = a.kind == BEAM_LOCAL ? a.prefix : kChunkPadRows;
-  const int b = blockIdx.x / per_b, e = blockIdx.x - b * per_b;
-  const int head = threadIdx.x >> 4, c = (threadIdx.x & 15) * 8;
-  const int64_t p0 = a.pos0[b];
-  const size_t cache_row = (size_t)b * a.stride_seq + (size_t)head * a.stride_head;
-  if (a.kind == BEAM_LOCAL) {
-    const int64_t j = p0 - a.prefix + e;
-    uint4 kv = make_uint4(0u, 0u, 0u, 0u), vv = kv;
-    if (p0 >= 0 && j >= 0) {
-      const size_t off = cache_row + (size_t)(j % a.window) * kD + c;
-      kv = *reinterpret_cast<const uint4 *>(a.k_cache + off);
-      vv = *reinterpret_cast<const uint4 *>(a.v_cache + off);
-    }
-    const size_t dst = ((size_t)b * a.ext_rows + e) * (kHkv * kD) + head * kD + c;
-    *reinterpret_cast<uint4 *>(a.k_ext + dst) = kv;
-    *reinterpret_cast<uint4 *>(a.v_ext + dst) = vv;
-  } else {
-    const int64_t end = p0 + a.T, slot = end + e;
-    if (p0 < 0 || end > a.slots || slot >= a.slots || slot >= (end + 127) / 128 * 128) return;
-    *reinterpret_cast<uint4 *>(a.v_cache + cache_row + (size_t)slot * kD + c) =
-        make_uint4(0u, 0u, 0u, 0u);
   }
 }
 
