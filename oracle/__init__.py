@@ -89,6 +89,10 @@ def lib():
         L.oracle_prefill_rows.argtypes = [ctypes.c_int, pp, ctypes.c_int, ctypes.c_int, u16p, u16p,
                                           u16p, u16p, fp, fp, fp, ctypes.c_int64, i64p, i64p, dp,
                                           ctypes.c_int]
+        L.oracle_prefill_row_heads.restype = ctypes.c_int
+        L.oracle_prefill_row_heads.argtypes = [ctypes.c_int, pp, ctypes.c_int, ctypes.c_int, u16p,
+                                               u16p, u16p, u16p, fp, fp, fp, ctypes.c_int64, i64p,
+                                               i64p, i64p, dp, ctypes.c_int]
         L.oracle_decode.restype = ctypes.c_int
         L.oracle_decode.argtypes = [ctypes.c_int, pp, ctypes.c_int, u16p, u16p, u16p, u16p, fp, fp,
                                     fp, i64p, u16p, u16p, ctypes.c_int64, dp, ctypes.c_int]
@@ -218,6 +222,29 @@ def prefill_rows(kind, P: Params, q, k, v, gate, q_norm_w, k_norm_w, gate_bias, 
         n_threads or n_threads_default())
     if rc != 0:
         raise ValueError("oracle_prefill_rows rejected its arguments")
+    return out
+
+
+def prefill_row_heads(kind, P: Params, q, k, v, gate, q_norm_w, k_norm_w, gate_bias, rows_b,
+                      rows_t, rows_h, n_threads: int | None = None) -> np.ndarray:
+    """Gated attention output of single query heads: item r is head rows_h[r] of row
+    (rows_b[r], rows_t[r]); [n_items, d] float64.  Same arithmetic as prefill_rows."""
+    q, k, v, gate = _u16(q), _u16(k), _u16(v), _u16(gate)
+    B, T = q.shape[0], q.shape[1]
+    rows_b = np.ascontiguousarray(rows_b, dtype=np.int64)
+    rows_t = np.ascontiguousarray(rows_t, dtype=np.int64)
+    rows_h = np.ascontiguousarray(rows_h, dtype=np.int64)
+    assert rows_b.size == rows_t.size == rows_h.size
+    qw, kw, bias = _f32(q_norm_w), _f32(k_norm_w), _f32(gate_bias)
+    out = np.empty((rows_b.size, P.head_dim), dtype=np.float64)
+    rc = lib().oracle_prefill_row_heads(
+        kind, ctypes.byref(P), B, T, _ptr(q, ctypes.c_uint16), _ptr(k, ctypes.c_uint16),
+        _ptr(v, ctypes.c_uint16), _ptr(gate, ctypes.c_uint16), _ptr(qw, ctypes.c_float),
+        _ptr(kw, ctypes.c_float), _ptr(bias, ctypes.c_float), rows_b.size,
+        _ptr(rows_b, ctypes.c_int64), _ptr(rows_t, ctypes.c_int64), _ptr(rows_h, ctypes.c_int64),
+        _ptr(out, ctypes.c_double), n_threads or n_threads_default())
+    if rc != 0:
+        raise ValueError("oracle_prefill_row_heads rejected its arguments")
     return out
 
 

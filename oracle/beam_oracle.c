@@ -249,6 +249,7 @@ typedef struct {
   const double *qw, *kw;
   const float *bias;
   const int64_t *rows_b, *rows_t;
+  const int64_t *rows_h;   /* oracle_prefill_row_heads: the one query head of each item */
   double *out;
   double **khat;   /* per sequence: [T][Hkv][d] prepared keys (NULL if unused) */
   double **vd;     /* per sequence: [T][Hkv][d] values as doubles */
@@ -326,6 +327,66 @@ int oracle_prefill_rows(int kind, const oracle_params *P, int B, int T,
     run_parallel(prefill_key_job, &c, T, n_threads);
   }
   run_parallel(prefill_row_job, &c, n_rows, n_threads);
+  for (int b = 0; b < B; ++b) { free(c.khat[b]); free(c.vd[b]); }
+  free(c.khat); free(c.vd); free(qw); free(kw);
+  return 0;
+}
+
+/* The same output as oracle_prefill_rows for single (row, head) items: item r is
+ * query head rows_h[r] of row (rows_b[r], rows_t[r]); out is [n_items][d].  Long
+ * rows then cost one head instead of 48, so a parity sample can reach deep into a
+ * 131,072-token sequence and still spread over every head. */
+static void prefill_row_head_job(void *vctx, int64_t r) {
+  prefill_ctx *c = (prefill_ctx *)vctx;
+  const oracle_params *P = c->P;
+  int d = P->head_dim, Hq = P->n_q_heads, Hkv = P->n_kv_heads, G = Hq / Hkv;
+  int64_t b = c->rows_b[r], t = c->rows_t[r];
+  int h = (int)c->rows_h[r], g = h / G;
+  int64_t lo = 0;
+  while (!oracle_visible(c->kind, t, lo, P->window)) ++lo;  /* first visible key */
+  int64_t n = t - lo + 1;
+  double *q = (double *)malloc(sizeof(double) * d);
+  double *scores = (double *)malloc(sizeof(double) * n);
+  kv_view view = {c->khat[b] + ((size_t)lo * Hkv + g) * d, c->vd[b] + ((size_t)lo * Hkv + g) * d,
+                  (int64_t)Hkv * d, d};
+  size_t q_off = (((size_t)b * c->T + t) * Hq + h) * d;
+  prepare_query(c->kind, P, c->q + q_off, c->qw, t, q);
+  attend_one(P, q, n, kv_view_row, &view, c->gate + q_off, (double)c->bias[h], scores,
+             c->out + (size_t)r * d);
+  free(q); free(scores);
+}
+
+int oracle_prefill_row_heads(int kind, const oracle_params *P, int B, int T,
+                             const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                             const uint16_t *gate, const float *q_norm_w, const float *k_norm_w,
+                             const float *gate_bias, int64_t n_items, const int64_t *rows_b,
+                             const int64_t *rows_t, const int64_t *rows_h, double *out,
+                             int n_threads) {
+  if (!P || P->n_kv_heads <= 0 || P->n_q_heads % P->n_kv_heads) return -1;
+  for (int64_t r = 0; r < n_items; ++r)
+    if (rows_b[r] < 0 || rows_b[r] >= B || rows_t[r] < 0 || rows_t[r] >= T || rows_h[r] < 0 ||
+        rows_h[r] >= P->n_q_heads)
+      return -1;
+  int d = P->head_dim, Hkv = P->n_kv_heads;
+  double *qw = (double *)malloc(sizeof(double) * d), *kw = (double *)malloc(sizeof(double) * d);
+  for (int i = 0; i < d; ++i) { qw[i] = q_norm_w[i]; kw[i] = k_norm_w[i]; }
+  prefill_ctx c;
+  memset(&c, 0, sizeof c);
+  c.kind = kind; c.P = P; c.B = B; c.T = T;
+  c.q = q; c.k = k; c.v = v; c.gate = gate; c.qw = qw; c.kw = kw; c.bias = gate_bias;
+  c.rows_b = rows_b; c.rows_t = rows_t; c.rows_h = rows_h; c.out = out;
+  c.khat = (double **)calloc(B, sizeof(double *));
+  c.vd = (double **)calloc(B, sizeof(double *));
+  for (int b = 0; b < B; ++b) {
+    int used = 0;
+    for (int64_t r = 0; r < n_items && !used; ++r) used = rows_b[r] == b;
+    if (!used) continue;
+    c.khat[b] = (double *)malloc(sizeof(double) * (size_t)T * Hkv * d);
+    c.vd[b] = (double *)malloc(sizeof(double) * (size_t)T * Hkv * d);
+    c.key_b = b;
+    run_parallel(prefill_key_job, &c, T, n_threads);
+  }
+  run_parallel(prefill_row_head_job, &c, n_items, n_threads);
   for (int b = 0; b < B; ++b) { free(c.khat[b]); free(c.vd[b]); }
   free(c.khat); free(c.vd); free(qw); free(kw);
   return 0;

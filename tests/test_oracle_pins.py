@@ -154,6 +154,44 @@ def test_gqa_equals_explicitly_repeated_kv(orc, kind):
     assert np.max(np.abs(yb - yg)) > 1e-2
 
 
+@pytest.mark.parametrize("kind", [wl.LOCAL, wl.GLOBAL])
+def test_single_head_items_equal_repeated_kv_rows(orc, kind):
+    """prefill_row_heads (one query head per item) against the full-row function run
+    with every query head given its own copy of KV head h // 3: the item's head picks
+    both its KV head and its output, so a wrong mapping or index fails here."""
+    T, d = 30, 16
+    Pg = orc.params(n_q_heads=6, n_kv_heads=2, head_dim=d, window=9)
+    Pr = orc.params(n_q_heads=6, n_kv_heads=6, head_dim=d, window=9)
+    q, gate = _rand((2, T, 6 * d), 8, "q"), _rand((2, T, 6 * d), 8, "g")
+    k, v = _rand((2, T, 2, d), 8, "k"), _rand((2, T, 2, d), 8, "v")
+    kr, vr = np.repeat(k, 3, axis=2), np.repeat(v, 3, axis=2)
+    w1, w2 = wl.norm_weight(8, "qw")[:d], wl.norm_weight(8, "kw")[:d]
+    bias = np.linspace(-1, 1, 6).astype(np.float32)
+    rng = np.random.default_rng(4)
+    rb, rt, rh = rng.integers(0, 2, 40), rng.integers(0, T, 40), rng.integers(0, 6, 40)
+    got = orc.prefill_row_heads(kind, Pg, q, k.reshape(2, T, -1), v.reshape(2, T, -1), gate, w1,
+                                w2, bias, rb, rt, rh)
+    full = orc.prefill_rows(kind, Pr, q, kr.reshape(2, T, -1), vr.reshape(2, T, -1), gate, w1, w2,
+                            bias, rb, rt)
+    np.testing.assert_allclose(got, full[np.arange(40), rh], rtol=1e-13, atol=1e-15)
+
+
+def test_single_head_items_window_of_one_closed_form(orc):
+    """Window 1: each item is its own value row of KV head h // 6, gated per
+    coordinate with its head's bias -- written out in numpy."""
+    T = 12
+    P = orc.params(window=1)
+    inp = wl.prefill_inputs(1, T, 3, layer="w1heads")
+    rt = np.arange(T)
+    rh = (7 * rt + 5) % 48
+    got = orc.prefill_row_heads(wl.LOCAL, P, inp.q, inp.k, inp.v, inp.gate, inp.q_norm_w,
+                                inp.k_norm_w, inp.gate_bias, np.zeros(T, np.int64), rt, rh)
+    v = wl.bf16_bits_to_f32(inp.v[0]).astype(np.float64).reshape(T, 8, 128)
+    g = wl.bf16_bits_to_f32(inp.gate[0]).astype(np.float64).reshape(T, 48, 128)
+    expect = v[rt, rh // 6] / (1.0 + np.exp(-(g[rt, rh] + inp.gate_bias[rh][:, None])))
+    np.testing.assert_allclose(got, expect, rtol=1e-14, atol=1e-15)
+
+
 # ---------------------------------------------------------------- softmax
 def test_softmax_toy_distractor_model(orc):
     """Section 'What scalable softmax changes mathematically': P ~ 6.17e-6."""
