@@ -741,8 +741,6 @@ int decode_call(int kind, const beam_attn_params *p, int32_t B, const void *q, c
   d8.base = da;
   d8.k_scale = k_scale;
   d8.v_scale = v_scale;
-  d8.inv_k_scale = 1.0f / k_scale;
-  d8.inv_v_scale = 1.0f / v_scale;
 
   if (kind == BEAM_LOCAL) {
     // one launch: the ring's splits form a cluster that also merges through distributed
@@ -852,8 +850,8 @@ int beam_kv_append_fp8(int kind, const beam_attn_params *p, int32_t B, int32_t T
   pa.slots = layout->slots_per_seq;
   pa.pos0 = pos0;
   pa.cache_fp8 = 1;
-  pa.inv_k_scale = 1.0f / k_scale;
-  pa.inv_v_scale = 1.0f / v_scale;
+  pa.k_scale = k_scale;
+  pa.v_scale = v_scale;
   pa.status = dev_status;
   pa.T = T;
   pa.kind = kind;

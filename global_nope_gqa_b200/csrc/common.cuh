@@ -83,7 +83,38 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
   return (uint32_t)h.x | ((uint32_t)h.y << 16);
 }
 
-// Eight fp32 values -> eight E4M3 codes (value * inv_scale, nearest, saturating), in order.
+// x / scale rounded to fp32 by round-to-odd: the quotient is formed by IEEE fp64 division
+// (correctly rounded), truncated to fp32, and the last significand bit is set when the
+// truncation dropped anything.  Rounding that fp32 value once more to nearest at 4
+// significant bits (E4M3) gives the nearest E4M3 value of the fp64 quotient -- no double
+// rounding -- because 24 >= 4 + 2 (round-to-odd: S. Boldo, G. Melquiond, "Emulation of
+// FMA and correctly rounded sums: proved algorithms using rounding to odd", IEEE Trans.
+// Computers 57(4), 2008).  Magnitudes past the fp32 range truncate to FLT_MAX, which the
+// saturating conversion maps to 448 like any other value past 448.
+__device__ __forceinline__ float div_to_f32_odd(float x, double scale) {
+  const double q = (double)x / scale;
+  float f = __double2float_rz(q);
+  if ((double)f != q) f = __uint_as_float(__float_as_uint(f) | 1u);
+  return f;
+}
+
+// Eight fp32 values -> eight cache codes E4M3(x / scale) (nearest, ties to even, saturating
+// at +-448), in order: the quotient of the value and the cache's scale, not of the value
+// and a rounded reciprocal, so a code matches the nearest code of the exact quotient at any
+// finite positive scale.
+__device__ __forceinline__ uint2 f32x8_to_e4m3_div(const float (&x)[8], float scale) {
+  const double s = (double)scale;
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    w[i] = __nv_cvt_float2_to_fp8x2(
+        make_float2(div_to_f32_odd(x[2 * i], s), div_to_f32_odd(x[2 * i + 1], s)),
+        __NV_SATFINITE, __NV_E4M3);
+  return make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
+}
+
+// Eight fp32 values -> eight E4M3 codes (value * mul, nearest, saturating), in order.  Used
+// with power-of-two factors (the decode query's two-term split), where the product is exact.
 __device__ __forceinline__ uint2 f32x8_to_e4m3(const float (&x)[8], float inv_scale) {
   uint32_t w[4];
 #pragma unroll

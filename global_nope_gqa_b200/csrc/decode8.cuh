@@ -50,8 +50,7 @@ constexpr int kDec8Smem = kDec8Stages * 2 * kDec8TileBytes;   // 64 KiB: three C
 
 struct Decode8Args {
   DecodeArgs base;          // caches are the code arrays (k_cache / v_cache as bytes)
-  float k_scale, v_scale;   // value = code * scale
-  float inv_k_scale, inv_v_scale;
+  float k_scale, v_scale;   // value = code * scale; code = E4M3(value / scale)
 };
 
 __device__ __forceinline__ uint32_t swz128(int row, int chunk) {  // byte offset in a tile
@@ -213,7 +212,7 @@ __global__ void __launch_bounds__(kDecThreads) decode8_attn_kernel(const Decode8
       *reinterpret_cast<uint2 *>(q_hi + row * kD + l16 * 8) = hi;
       *reinterpret_cast<uint2 *>(q_lo + row * kD + l16 * 8) = f32x8_to_e4m3(r, 1.0f);
     } else if (slot / a.split == s_idx) {
-      const uint2 codes = f32x8_to_e4m3(x, row == kGroup ? A.inv_k_scale : A.inv_v_scale);
+      const uint2 codes = f32x8_to_e4m3_div(x, row == kGroup ? A.k_scale : A.v_scale);
       uint8_t *cache = row == kGroup ? kbase : vbase;
       *reinterpret_cast<uint2 *>(cache + (size_t)slot * kD + l16 * 8) = codes;
       const int rel = (int)(slot - key_lo);

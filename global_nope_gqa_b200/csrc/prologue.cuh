@@ -91,8 +91,8 @@ struct PrologueArgs {
   float *rope_tab;       // local layers, or null: cos (64) then sin (64) of each token's angles
   int rope_per_seq;      // rope_tab is [B][T][128] (own positions) rather than [T][128] (0 .. T-1)
   int whole_seq;         // a sequence whose tokens do not all fit is not written at all
-  int cache_fp8;         // the caches hold E4M3 codes of value * inv scale (one byte each)
-  float inv_k_scale, inv_v_scale;
+  int cache_fp8;         // the caches hold E4M3 codes of value / scale (one byte each)
+  float k_scale, v_scale;
   int32_t *status;
   int T;                 // tokens per sequence in this call
   // chunked prefill: n_prep extra CTAs after the B * T token CTAs prepare the chunk (the
@@ -284,7 +284,7 @@ __global__ void __launch_bounds__(128) prologue_kernel(const PrologueArgs a) {
         if (a.cache_fp8) {   // codes of the fp32 rows, not of their bf16 rounding
           uint8_t *cache = reinterpret_cast<uint8_t *>(is_k ? a.k_cache : a.v_cache);
           *reinterpret_cast<uint2 *>(cache + off) =
-              f32x8_to_e4m3(x, is_k ? a.inv_k_scale : a.inv_v_scale);
+              f32x8_to_e4m3_div(x, is_k ? a.k_scale : a.v_scale);
         } else {
           uint16_t *cache = is_k ? a.k_cache : a.v_cache;
           const int r = a.ring_save ? i % a.window : 0;

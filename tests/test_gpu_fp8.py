@@ -3,9 +3,12 @@
 Cache contents are seeded E4M3 codes given to both sides.  The FP8 decode is
 compared with oracle_decode_fp8 at the parity bar of the other GPU tests.  Codes
 the device writes are compared with the oracle's expected codes: value codes bit
-for bit (raw bf16 values divided by a power-of-two scale are exact in fp32, so
-both sides round the same number), key codes within one E4M3 step (the device
-rounds its fp32 normalised key, the oracle the exact one).
+for bit at any finite positive scale (both sides take the nearest code of the
+exact quotient value / scale: the oracle divides in fp64, the device divides in
+fp64 and reaches fp32 by round-to-odd, so its one E4M3 rounding is exact), key
+codes within one E4M3 step (the device rounds its fp32 normalised key, the oracle
+the exact one).  The scales include ones an amax / 448 rule gives (0.0173, 3.7,
+not powers of two) and one that makes large values saturate at 448 (0.0051).
 """
 import numpy as np
 import pytest
@@ -33,7 +36,8 @@ def _f8_layout(beam, kind, params, B, slots):
 
 
 @pytest.mark.parametrize("kind", [wl.GLOBAL, wl.LOCAL])
-@pytest.mark.parametrize("k_scale,v_scale", [(0.5, 1.0), (1.0, 0.25)])
+@pytest.mark.parametrize("k_scale,v_scale", [(0.5, 1.0), (1.0, 0.25), (0.0173, 3.7),
+                                             (3.7, 0.0051)])
 def test_kv_append_fp8_codes(env, kind, k_scale, v_scale):
     torch, beam, orc = env
     params = beam.default_params()
@@ -90,7 +94,8 @@ def run_decode_fp8(torch, beam, di, kc0, vc0, k_scale, v_scale, params=None, sta
     (wl.GLOBAL, [1, 2, 63, 64, 65, 700, 4097, 9000], 9000),
     (wl.LOCAL, [1, 3, 511, 512, 513, 2000, 70], 512),
 ])
-@pytest.mark.parametrize("k_scale,v_scale", [(0.5, 2.0), (1.0, 1.0)])
+@pytest.mark.parametrize("k_scale,v_scale", [(0.5, 2.0), (1.0, 1.0), (0.0173, 3.7),
+                                             (3.7, 0.0051)])
 def test_decode_fp8_matches_oracle_and_appends(env, kind, ctx, slots, k_scale, v_scale):
     torch, beam, orc = env
     params = beam.default_params()
