@@ -237,6 +237,10 @@ int decode_split(int kind, const beam_attn_params *p, int32_t B, int64_t slots, 
   return (int)split;
 }
 
+// What beam_decode_workspace_bytes reports for a local layer, which needs no workspace:
+// a small nonzero size, because 0 reports invalid arguments.
+constexpr size_t kDecodeNoWorkspace = 16;
+
 struct DecodeWorkspace {
   float *part_o;
   float *part_ml;
@@ -660,6 +664,8 @@ int beam_kv_append(int kind, const beam_attn_params *p, int32_t B, int32_t T, co
 size_t beam_decode_workspace_bytes(int kind, const beam_attn_params *p, int32_t B,
                                    const beam_kv_layout_t *layout) {
   if (check_params(kind, p) || !layout || B <= 0 || layout->slots_per_seq < 1) return 0;
+  // a ring decode merges its splits in distributed shared memory: no workspace
+  if (kind == BEAM_LOCAL) return kDecodeNoWorkspace;
   DeviceInfo *dev = nullptr;
   int sm = 148;
   if (device_info(&dev) == BEAM_OK) sm = dev->sm_count;
@@ -701,8 +707,9 @@ int decode_call(int kind, const beam_attn_params *p, int32_t B, const void *q, c
   const int split = decode_split(kind, p, B, layout->slots_per_seq, dev->sm_count, fp8);
   const int64_t vis_max = kind == BEAM_LOCAL ? p->window : layout->slots_per_seq;
   const int n_split_max = (int)((vis_max + split - 1) / split);
+  // only the split-K path of a global layer keeps partial results in the workspace
   DecodeWorkspace w = decode_workspace(workspace, B, n_split_max);
-  if (!workspace || workspace_bytes < w.bytes) return BEAM_ERR_WORKSPACE;
+  if (kind == BEAM_GLOBAL && (!workspace || workspace_bytes < w.bytes)) return BEAM_ERR_WORKSPACE;
   if (n_split_max > 65535) return BEAM_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
 
@@ -904,9 +911,13 @@ int beam_attn_decode_noalloc(int kind, const beam_attn_params *p, int32_t B, con
   if (B < 0) return BEAM_ERR_INVALID_ARG;
   if (B == 0) return BEAM_OK;
   if ((st = check_layout(kind, p, layout))) return st;
-  const size_t need = beam_decode_workspace_bytes(kind, p, B, layout);
-  if (need == 0) return BEAM_ERR_CUDA;
-  if (need > kNoAllocScratchBytes) return BEAM_ERR_SCRATCH_LIMIT;
+  // a local (ring) decode keeps nothing in the scratch; a global one needs the
+  // split-K partials of all its sequences to fit
+  if (kind == BEAM_GLOBAL) {
+    const size_t need = beam_decode_workspace_bytes(kind, p, B, layout);
+    if (need == 0) return BEAM_ERR_CUDA;
+    if (need > kNoAllocScratchBytes) return BEAM_ERR_SCRATCH_LIMIT;
+  }
   void *scratch = nullptr;
   if ((st = noalloc_scratch(&scratch))) return st;
   return beam_attn_decode(kind, p, B, q, k, v, gate, q_norm_w, k_norm_w, gate_bias, pos, k_cache,

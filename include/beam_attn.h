@@ -188,8 +188,10 @@ BEAM_API int beam_kv_append(int kind, const beam_attn_params *p, int32_t B, int3
                    void *v_cache, const beam_kv_layout_t *layout, int32_t *dev_status,
                    beam_stream_t stream);
 
-/* Workspace of one decode call (bytes): the split-K partial results, sized from
- * the layout's slots per sequence. */
+/* Workspace of one decode call (bytes): for a global layer the split-K partial
+ * results, sized from the layout's slots per sequence (0: invalid arguments).  A
+ * local layer's decode merges its splits on chip and needs no workspace: the
+ * function returns 16 and the call accepts any workspace, null included. */
 BEAM_API size_t beam_decode_workspace_bytes(int kind, const beam_attn_params *p, int32_t B,
                                    const beam_kv_layout_t *layout);
 
@@ -260,14 +262,18 @@ BEAM_API int beam_attn_decode_fp8(int kind, const beam_attn_params *p, int32_t B
  * This entry point computes exactly what beam_attn_decode computes, with the
  * same arguments minus the workspace.  Its scratch is a fixed array of
  * 8 MiB (8,388,608 bytes) of device memory inside the library, which every GPU
- * that loads the library holds until the process exits.  A call whose
- * beam_decode_workspace_bytes() would exceed 8 MiB returns
- * BEAM_ERR_SCRATCH_LIMIT before any launch (roughly: B * 8 * splits * 3.1 KB +
- * B * 12 KB; B = 64 at a 32K-slot cache or B = 1 at a 1M-slot cache fit).
+ * that loads the library holds until the process exits.  A global-layer call
+ * whose beam_decode_workspace_bytes() would exceed 8 MiB returns
+ * BEAM_ERR_SCRATCH_LIMIT before any launch (roughly: B * 8 * splits * 3.1 KB;
+ * B = 64 at a 32K-slot cache or B = 1 at a 1M-slot cache fit).  A local-layer
+ * call uses no scratch and takes any batch.
  *
  * The first call on each device looks up the array's device address (with that
  * device current) and caches it; make that first call before any stream
- * capture.  All calls share the one array and it keeps whatever the last call
+ * capture.  The library caches per-device state (this address, the kernels'
+ * shared-memory opt-ins) for the life of the process: after cudaDeviceReset
+ * of a device, do not call the library on that device again in the same
+ * process.  All calls share the one array and it keeps whatever the last call
  * left in it; nothing in it needs to start at zero, because every value read
  * is written earlier in the same call.  Calls whose kernels overlap on the GPU
  * (on different streams, or from several threads) race on the array: issue

@@ -153,6 +153,9 @@ def test_host_validation_rejects_before_launch(beam):
     glob = beam.beam_kv_layout(beam.GLOBAL, p, 2, 4096)
     dws = beam.beam_decode_workspace_bytes(beam.GLOBAL, p, 2, glob)
     assert dws > 2 * 48 * 128 * 2
+    # a local (ring) decode merges on chip: a small nonzero size, whatever the batch
+    ring512 = beam.beam_kv_layout(beam.LOCAL, p, 4096, 512)
+    assert beam.beam_decode_workspace_bytes(beam.LOCAL, p, 4096, ring512) == 16
     dargs = lambda **kw: [kw.get("kind", 1), P, kw.get("B", 2), A, A, A, A, A, A, A,
                           kw.get("pos", A), A, A, kw.get("layout", ctypes.byref(glob)), A,
                           kw.get("ws", A), kw.get("ws_bytes", dws), None, None]
