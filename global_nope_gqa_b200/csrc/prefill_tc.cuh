@@ -109,29 +109,6 @@ __device__ __forceinline__ float tanh_approx(float x) {
   return y;
 }
 
-// exp2 of two values on the FMA and integer pipes, to take part of the exponentials off the
-// MUFU unit: 2^y = 2^k * 2^f with k = round(y) (found by adding 1.5 * 2^23, which leaves k
-// in the low mantissa bits), f = y - k in [-1/2, 1/2], 2^f from a cubic fitted for least
-// maximum relative error (7.5e-5, far below bf16's 2^-9; fit_exp2_poly.py), and 2^k
-// applied by adding k to the exponent field.  y is clamped at -120 first, so masked
-// (-inf) scores give 2^-120 instead of 0 -- negligible against the row's weights.
-constexpr int kTcEmuPairs = 0;  // pairs per 16 emulated in each 32-score chunk
-__device__ __forceinline__ void exp2_poly_pair(float y0, float y1, float &p0, float &p1) {
-  const uint64_t y = tc::f2_pack(fmaxf(y0, -120.0f), fmaxf(y1, -120.0f));
-  const uint64_t t = tc::f2_add(y, tc::f2_pack(12582912.0f, 12582912.0f));
-  const uint64_t kf = tc::f2_add(t, tc::f2_pack(-12582912.0f, -12582912.0f));
-  const uint64_t f = tc::f2_fma(kf, tc::f2_pack(-1.0f, -1.0f), y);
-  uint64_t q = tc::f2_fma(tc::f2_pack(5.517166853e-02f, 5.517166853e-02f), f,
-                          tc::f2_pack(2.426111251e-01f, 2.426111251e-01f));
-  q = tc::f2_fma(q, f, tc::f2_pack(6.932609677e-01f, 6.932609677e-01f));
-  q = tc::f2_fma(q, f, tc::f2_pack(9.999280572e-01f, 9.999280572e-01f));
-  float q0, q1, t0, t1;
-  tc::f2_unpack(q, q0, q1);
-  tc::f2_unpack(t, t0, t1);
-  p0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
-  p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
-}
-
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
@@ -671,13 +648,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                                  __uint_as_float(sr[c][i + 1])),
                                      f2, nm2),
                           y0, y1);
-            float p0, p1;
-            if ((i >> 1) < kTcEmuPairs) {
-              exp2_poly_pair(y0, y1, p0, p1);
-            } else {
-              p0 = ex2_approx(y0);
-              p1 = ex2_approx(y1);
-            }
+            const float p0 = ex2_approx(y0), p1 = ex2_approx(y1);
             acc[(i >> 1) & 3] = tc::f2_add(acc[(i >> 1) & 3], tc::f2_pack(p0, p1));
             pk[i >> 1] = pack_bf16(p0, p1);
           }

@@ -170,12 +170,16 @@ def test_prefill_masks_bit_exact(env, kind, T, window):
 
 
 def _rows_sample(B, T, seed, n_random):
+    """Per sequence: both rows at every 128-row tile boundary (128k - 1, 128k), the rows
+    at the window's edges (the first rows whose window is full, 510 .. 514), the first and
+    last rows, and n_random seeded rows."""
     rng = np.random.default_rng(seed)
     rows = []
+    edges = [0, 1, 2, 510, 511, 512, 513, 514, T - 1]
+    tiles = [t for k in range(1, (T + 127) // 128) for t in (128 * k - 1, 128 * k)]
     for b in range(B):
-        fixed = [0, 1, 511, 512, 513, T - 1]
         rnd = rng.integers(0, T, size=n_random)
-        rows += [(b, int(t)) for t in sorted(set([t for t in fixed if t < T] + list(rnd)))]
+        rows += [(b, int(t)) for t in sorted(set([t for t in edges + tiles if t < T] + list(rnd)))]
     return np.array([r[0] for r in rows]), np.array([r[1] for r in rows])
 
 
@@ -193,8 +197,9 @@ def _device_prefill_inputs(torch, B, T, seed, tag):
 
 @pytest.mark.parametrize("kind", [wl.LOCAL, wl.GLOBAL])
 def test_prefill_batched_workload_sampled_rows(env, kind):
-    """Batched prefill workload (B=4, T=8192) in the bench's launch configuration;
-    sampled rows (window edges, last token, random) against the oracle."""
+    """Batched prefill workload (B=4, T=8192) in the bench's launch configuration: over
+    540 rows (every 128-row tile boundary and the window edges of each sequence, plus
+    random rows), all 48 heads, against the oracle."""
     torch, beam, orc = env
     w = wl.workload("batched_prefill")
     x, inp = _device_prefill_inputs(torch, w.B, w.T, w.seed, f"bp{kind}")
@@ -209,6 +214,7 @@ def test_prefill_batched_workload_sampled_rows(env, kind):
                            vc, layout)
     torch.cuda.synchronize()
     rb, rt = _rows_sample(w.B, w.T, 3, 6)
+    assert rb.size >= 512
     qh = host_bits(x["q"]); kh = host_bits(x["k"]); vh = host_bits(x["v"]); gh = host_bits(x["gate"])
     ref = orc.prefill_rows(kind, oracle_params(orc, params), qh, kh, vh, gh, inp.q_norm_w,
                            inp.k_norm_w, inp.gate_bias, rb, rt)
@@ -217,7 +223,11 @@ def test_prefill_batched_workload_sampled_rows(env, kind):
 
 
 def test_prefill_long_global_sampled_rows(env):
-    """Long-context global prefill (B=1, T=131072): a(p) up to p = 131072."""
+    """Long-context global prefill (B=1, T=131072): a(p) up to p = 131072.  A stratified
+    sample of 2,048 rows: the first 512 rows with all 48 heads, then the last 512 rows and
+    1,024 seeded random rows, each with the two heads of one work unit (head pair r mod
+    24, so every pair is covered many times over) -- a row near the end reads 131,072
+    keys, and one head pair keeps the fp64 oracle within tens of seconds."""
     torch, beam, orc = env
     w = wl.workload("long_global_prefill")
     x, inp = _device_prefill_inputs(torch, w.B, w.T, w.seed, "long")
@@ -227,12 +237,23 @@ def test_prefill_long_global_sampled_rows(env):
     out = torch.empty_like(x["q"])
     beam.beam_attn_prefill(wl.GLOBAL, params, x["q"], x["k"], x["v"], x["gate"], qw, kw, bias, out)
     torch.cuda.synchronize()
-    rt = np.array([0, 1, 2047, 65535, 100000, 131071])
-    rb = np.zeros_like(rt)
-    ref = orc.prefill_rows(wl.GLOBAL, oracle_params(orc, params), host_bits(x["q"]),
-                           host_bits(x["k"]), host_bits(x["v"]), host_bits(x["gate"]),
-                           inp.q_norm_w, inp.k_norm_w, inp.gate_bias, rb, rt)
-    assert_close(host_bits(out)[rb, rt].reshape(ref.shape), ref, "long global")
+    T = w.T
+    qh, kh, vh, gh = (host_bits(x[n]) for n in ("q", "k", "v", "gate"))
+    got = host_bits(out)
+    P = oracle_params(orc, params)
+    first = np.arange(512)
+    ref = orc.prefill_rows(wl.GLOBAL, P, qh, kh, vh, gh, inp.q_norm_w, inp.k_norm_w,
+                           inp.gate_bias, np.zeros_like(first), first)
+    assert_close(got[0, first].reshape(ref.shape), ref, "long global, first 512 rows")
+    rnd = np.random.default_rng(17).choice(np.arange(512, T - 512), 1024, replace=False)
+    deep = np.concatenate([np.arange(T - 512, T), np.sort(rnd)])
+    pair = np.arange(deep.size) % 24
+    rt = np.repeat(deep, 2)
+    rh = np.stack([2 * pair, 2 * pair + 1], axis=1).ravel()
+    ref = orc.prefill_row_heads(wl.GLOBAL, P, qh, kh, vh, gh, inp.q_norm_w, inp.k_norm_w,
+                                inp.gate_bias, np.zeros_like(rt), rt, rh)
+    g = got[0].reshape(T, 48, 128)[rt, rh]
+    assert_close(g, ref, "long global, last 512 and 1,024 random rows")
 
 
 # ------------------------------------------------------------------ caches
@@ -354,22 +375,21 @@ def test_decode_edge_contexts(env, kind):
     np.testing.assert_array_equal(vh, expect)
 
 
-def test_decode_batched_workload_sampled_sequences(env):
+def test_decode_batched_workload_all_sequences(env):
     """Batched decode workload: 64 sequences, contexts uniform in [1024, 32768],
-    one local and one global layer; every output of 16 sampled sequences."""
+    one local and one global layer; every output element of all 64 sequences."""
     torch, beam, orc = env
     w = wl.workload("batched_decode")
     ctx = np.array(w.ctx)
     params = beam.default_params()
     P = oracle_params(orc, params)
-    pick = np.random.default_rng(0).choice(w.B, 16, replace=False)
     for kind, slots in ((wl.GLOBAL, w.extra["global_slots"]), (wl.LOCAL, 512)):
         di = wl.decode_inputs(kind, ctx, slots, w.seed, layer=f"bd{kind}")
-        k0, v0 = di.k_cache[pick].copy(), di.v_cache[pick].copy()
+        k0, v0 = di.k_cache.copy(), di.v_cache.copy()
         out, *_ = run_decode(torch, beam, di)
-        ref = orc.decode(kind, P, di.q[pick], di.k[pick], di.v[pick], di.gate[pick], di.q_norm_w,
-                         di.k_norm_w, di.gate_bias, di.pos[pick], k0, v0)
-        assert_close(host_bits(out)[pick].reshape(ref.shape), ref, f"batched decode kind={kind}")
+        ref = orc.decode(kind, P, di.q, di.k, di.v, di.gate, di.q_norm_w, di.k_norm_w,
+                         di.gate_bias, di.pos, k0, v0)
+        assert_close(host_bits(out).reshape(ref.shape), ref, f"batched decode kind={kind}")
 
 
 def test_decode_1m_context(env):
