@@ -111,6 +111,12 @@ def lib():
             ctypes.c_int, pp, ctypes.c_int, u16p, u16p, u16p, u16p, fp, fp, fp,
             ctypes.POINTER(ctypes.c_int64), u8p, u8p, ctypes.c_int64, ctypes.c_double,
             ctypes.c_double, dp, ctypes.c_int]
+        L.oracle_prefill_chunk_rows_fp8.restype = ctypes.c_int
+        L.oracle_prefill_chunk_rows_fp8.argtypes = [
+            ctypes.c_int, pp, ctypes.c_int, ctypes.c_int, u16p, u16p, u16p, u16p, fp, fp, fp,
+            ctypes.POINTER(ctypes.c_int64), u8p, u8p, ctypes.c_int64, ctypes.c_double,
+            ctypes.c_double, ctypes.c_int64, ctypes.POINTER(ctypes.c_int64),
+            ctypes.POINTER(ctypes.c_int64), dp, ctypes.c_int]
         L.oracle_kv_row_fp8.restype = None
         L.oracle_kv_row_fp8.argtypes = [ctypes.c_int, pp, u16p, u16p, fp, ctypes.c_int64,
                                         ctypes.c_double, ctypes.c_double, u8p, u8p]
@@ -347,6 +353,47 @@ def decode_fp8(kind, P: Params, q, k, v, gate, q_norm_w, k_norm_w, gate_bias, po
     if rc != 0:
         raise ValueError("oracle_decode_fp8 rejected its arguments")
     return out
+
+
+def prefill_chunk_rows_fp8(kind, P: Params, q, k, v, gate, q_norm_w, k_norm_w, gate_bias, pos0,
+                           k_codes, v_codes, k_scale: float, v_scale: float, rows_b, rows_i,
+                           n_threads: int | None = None) -> np.ndarray:
+    """Chunked prefill over FP8 E4M3 caches (uint8 codes [B, Hkv, slots, d] as they were
+    before the call, one scale per tensor) for the listed (b, new token i) rows:
+    [n_rows, Hq, d] float64.  The chunk's own keys and values are quantised first."""
+    q, k, v, gate = _u16(q), _u16(k), _u16(v), _u16(gate)
+    k_codes = np.ascontiguousarray(k_codes, dtype=np.uint8)
+    v_codes = np.ascontiguousarray(v_codes, dtype=np.uint8)
+    B, T = q.shape[0], q.shape[1]
+    slots = k_codes.shape[2]
+    pos0 = np.ascontiguousarray(pos0, dtype=np.int64)
+    rows_b = np.ascontiguousarray(rows_b, dtype=np.int64)
+    rows_i = np.ascontiguousarray(rows_i, dtype=np.int64)
+    qw, kw, bias = _f32(q_norm_w), _f32(k_norm_w), _f32(gate_bias)
+    out = np.empty((rows_b.size, P.n_q_heads, P.head_dim), dtype=np.float64)
+    i64 = ctypes.c_int64
+    rc = lib().oracle_prefill_chunk_rows_fp8(
+        kind, ctypes.byref(P), B, T, _ptr(q, ctypes.c_uint16), _ptr(k, ctypes.c_uint16),
+        _ptr(v, ctypes.c_uint16), _ptr(gate, ctypes.c_uint16), _ptr(qw, ctypes.c_float),
+        _ptr(kw, ctypes.c_float), _ptr(bias, ctypes.c_float), _ptr(pos0, i64),
+        _ptr(k_codes, ctypes.c_uint8), _ptr(v_codes, ctypes.c_uint8), slots, float(k_scale),
+        float(v_scale), rows_b.size, _ptr(rows_b, i64), _ptr(rows_i, i64),
+        _ptr(out, ctypes.c_double), n_threads or n_threads_default())
+    if rc != 0:
+        raise ValueError("oracle_prefill_chunk_rows_fp8 rejected its arguments")
+    return out
+
+
+def prefill_chunk_fp8(kind, P: Params, q, k, v, gate, q_norm_w, k_norm_w, gate_bias, pos0,
+                      k_codes, v_codes, k_scale: float, v_scale: float,
+                      n_threads: int | None = None) -> np.ndarray:
+    """All rows of a chunk over FP8 caches: [B, T, Hq, d] float64."""
+    B, T = q.shape[0], q.shape[1]
+    bb, ii = np.meshgrid(np.arange(B), np.arange(T), indexing="ij")
+    out = prefill_chunk_rows_fp8(kind, P, q, k, v, gate, q_norm_w, k_norm_w, gate_bias, pos0,
+                                 k_codes, v_codes, k_scale, v_scale, bb.ravel(), ii.ravel(),
+                                 n_threads)
+    return out.reshape(B, T, P.n_q_heads, P.head_dim)
 
 
 def kv_row_fp8(kind, P: Params, k_token, v_token, k_norm_w, j, k_scale: float, v_scale: float):

@@ -37,6 +37,10 @@ typedef struct {
 
 enum { ORACLE_LOCAL = 0, ORACLE_GLOBAL = 1 };
 
+/* FP8 E4M3 codes (defined with the FP8 cache functions below) */
+double oracle_e4m3_decode(uint8_t code);
+uint8_t oracle_e4m3_encode(double x);
+
 /* ---------------------------------------------------------------- scalars */
 
 double oracle_bf16_to_double(uint16_t bits) {
@@ -508,6 +512,12 @@ typedef struct {
   int64_t slots;
   const int64_t *rows_b, *rows_i;
   double *out;
+  /* FP8 E4M3 caches (oracle_prefill_chunk_rows_fp8): cached rows are
+   * E4M3^-1(code) * scale, and the chunk's own keys and values are first
+   * written as codes, so the queries see them read back from the cache too */
+  int fp8;
+  const uint8_t *k_codes, *v_codes;
+  double k_scale, v_scale;
 } chunk_ctx;
 
 typedef struct {
@@ -529,8 +539,13 @@ static void chunk_row(const void *vctx, int64_t idx, double *k_row, double *v_ro
   int64_t s = oracle_cache_slot(c->kind, j, c->slots);
   size_t off = (((size_t)r->b * c->P->n_kv_heads + r->g) * c->slots + s) * d;
   for (int i = 0; i < d; ++i) {
-    k_row[i] = oracle_bf16_to_double(c->k_cache[off + i]);
-    v_row[i] = oracle_bf16_to_double(c->v_cache[off + i]);
+    if (c->fp8) {
+      k_row[i] = oracle_e4m3_decode(c->k_codes[off + i]) * c->k_scale;
+      v_row[i] = oracle_e4m3_decode(c->v_codes[off + i]) * c->v_scale;
+    } else {
+      k_row[i] = oracle_bf16_to_double(c->k_cache[off + i]);
+      v_row[i] = oracle_bf16_to_double(c->v_cache[off + i]);
+    }
   }
 }
 
@@ -554,9 +569,14 @@ static void chunk_job(void *vctx, int64_t r) {
     if (h % G == 0) {
       for (int64_t m = m0; m <= i; ++m) {
         size_t in_off = (((size_t)b * c->T + m) * Hkv + g) * d;
-        prepare_key(c->kind, P, c->k + in_off, c->kw, c->pos0[b] + m, kv_new + (size_t)m * d);
-        for (int e = 0; e < d; ++e)
-          kv_new[(size_t)(i + 1) * d + (size_t)m * d + e] = oracle_bf16_to_double(c->v[in_off + e]);
+        double *kn = kv_new + (size_t)m * d, *vn = kv_new + (size_t)(i + 1) * d + (size_t)m * d;
+        prepare_key(c->kind, P, c->k + in_off, c->kw, c->pos0[b] + m, kn);
+        for (int e = 0; e < d; ++e) vn[e] = oracle_bf16_to_double(c->v[in_off + e]);
+        if (c->fp8)   /* written as codes first, read back from the cache */
+          for (int e = 0; e < d; ++e) {
+            kn[e] = oracle_e4m3_decode(oracle_e4m3_encode(kn[e] / c->k_scale)) * c->k_scale;
+            vn[e] = oracle_e4m3_decode(oracle_e4m3_encode(vn[e] / c->v_scale)) * c->v_scale;
+          }
       }
     }
     chunk_view view = {c, b, g, lo, kv_new, kv_new + (size_t)(i + 1) * d};
@@ -587,7 +607,7 @@ int oracle_prefill_chunk_rows(int kind, const oracle_params *P, int B, int T,
   double *qw = (double *)malloc(sizeof(double) * d), *kw = (double *)malloc(sizeof(double) * d);
   for (int i = 0; i < d; ++i) { qw[i] = q_norm_w[i]; kw[i] = k_norm_w[i]; }
   chunk_ctx c = {kind, P, B, T, q, k, v, gate, qw, kw, gate_bias, pos0, k_cache, v_cache, slots,
-                 rows_b, rows_i, out};
+                 rows_b, rows_i, out, 0, NULL, NULL, 1.0, 1.0};
   run_parallel(chunk_job, &c, n_rows, n_threads);
   free(qw); free(kw);
   return 0;
@@ -711,6 +731,40 @@ int oracle_decode_fp8(int kind, const oracle_params *P, int B, const uint16_t *q
   decode8_ctx c = {{kind, P, B, q, k, v, gate, qw, kw, gate_bias, pos, NULL, NULL, slots, out},
                    k_codes, v_codes, k_scale, v_scale};
   run_parallel(decode8_job, &c, (int64_t)B * P->n_q_heads, n_threads);
+  free(qw); free(kw);
+  return 0;
+}
+
+/* Chunked prefill over FP8 E4M3 caches (section "KV memory": the FP8 cache, and a
+ * call that continues a sequence reads its earlier keys from the cache): as
+ * oracle_prefill_chunk_rows, but a cached row is E4M3^-1(code) * scale and the
+ * chunk's own keys and values are written as codes first (code = E4M3(x / scale)
+ * of the exact prepared key and of the raw value), so the queries see them read
+ * back from the cache -- the order oracle_decode_fp8 takes for one new token.
+ * Caches are head-major [B][Hkv][slots][d] codes as they were before the call. */
+int oracle_prefill_chunk_rows_fp8(int kind, const oracle_params *P, int B, int T,
+                                  const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                                  const uint16_t *gate, const float *q_norm_w,
+                                  const float *k_norm_w, const float *gate_bias,
+                                  const int64_t *pos0, const uint8_t *k_codes,
+                                  const uint8_t *v_codes, int64_t slots, double k_scale,
+                                  double v_scale, int64_t n_rows, const int64_t *rows_b,
+                                  const int64_t *rows_i, double *out, int n_threads) {
+  if (!P || P->n_kv_heads <= 0 || P->n_q_heads % P->n_kv_heads) return -1;
+  if (!(k_scale > 0.0) || !(v_scale > 0.0)) return -1;
+  for (int b = 0; b < B; ++b) {
+    if (pos0[b] < 0) return -1;
+    if (kind == ORACLE_GLOBAL && pos0[b] + T > slots) return -1;
+    if (kind == ORACLE_LOCAL && slots < P->window) return -1;
+  }
+  for (int64_t r = 0; r < n_rows; ++r)
+    if (rows_b[r] < 0 || rows_b[r] >= B || rows_i[r] < 0 || rows_i[r] >= T) return -1;
+  int d = P->head_dim;
+  double *qw = (double *)malloc(sizeof(double) * d), *kw = (double *)malloc(sizeof(double) * d);
+  for (int i = 0; i < d; ++i) { qw[i] = q_norm_w[i]; kw[i] = k_norm_w[i]; }
+  chunk_ctx c = {kind, P, B, T, q, k, v, gate, qw, kw, gate_bias, pos0, NULL, NULL, slots,
+                 rows_b, rows_i, out, 1, k_codes, v_codes, k_scale, v_scale};
+  run_parallel(chunk_job, &c, n_rows, n_threads);
   free(qw); free(kw);
   return 0;
 }

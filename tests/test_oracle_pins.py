@@ -554,6 +554,52 @@ def test_decode_fp8_window_of_one_is_the_quantised_new_value(orc):
     np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-14)
 
 
+def _nan_free_codes(rng, shape):
+    c = rng.integers(0, 256, size=shape).astype(np.uint8)
+    c[(c & 0x7F) == 0x7F] ^= 0x01        # no NaN codes
+    return c
+
+
+@pytest.mark.parametrize("kind", [0, 1])
+def test_chunk_fp8_of_one_token_equals_fp8_decode(orc, kind):
+    """A one-token chunk over FP8 caches is an FP8 decode step (pinned above): the new
+    key and value quantised first, cached codes read back with their scales.  Scales
+    that are not powers of two (an amax / 448 rule gives such)."""
+    d, Hq, Hkv, W = 16, 6, 2, 8
+    P = orc.params(n_q_heads=Hq, n_kv_heads=Hkv, head_dim=d, window=W)
+    pos = np.array([0, 3, 8, 29], np.int64)
+    B, slots = pos.size, (W if kind == orc.LOCAL else 40)
+    q, k, v, gate, qw, kw, bias = _small_chunk_problem(B, 1, 23)
+    rng = np.random.default_rng(23)
+    kc, vc = _nan_free_codes(rng, (B, Hkv, slots, d)), _nan_free_codes(rng, (B, Hkv, slots, d))
+    ks, vs = 0.0173, 3.7
+    got = orc.prefill_chunk_fp8(kind, P, q, k, v, gate, qw, kw, bias, pos, kc, vc, ks, vs)[:, 0]
+    ref = orc.decode_fp8(kind, P, q[:, 0], k[:, 0], v[:, 0], gate[:, 0], qw, kw, bias, pos, kc,
+                         vc, ks, vs)
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("kind", [0, 1])
+def test_chunk_fp8_equals_bf16_chunk_of_the_dequantised_cache(orc, kind):
+    """With the chunk's keys zero (RMSNorm keeps them zero, an exact code) and its values
+    on the E4M3 grid, the FP8 chunk is the BF16 chunk (pinned above) over caches holding
+    the dequantised codes: same slots, windows across the ring's wrap, power-of-two
+    scales (2 and 1/2) so the dequantised values are exact in bf16."""
+    d, Hq, Hkv, W, T = 16, 6, 2, 8, 5
+    P = orc.params(n_q_heads=Hq, n_kv_heads=Hkv, head_dim=d, window=W)
+    pos0 = np.array([0, 3, 8, 29], np.int64)
+    B, slots = pos0.size, (W if kind == orc.LOCAL else 40)
+    q, k, v, gate, qw, kw, bias = _small_chunk_problem(B, T, 24)
+    k[:] = 0
+    rng = np.random.default_rng(24)
+    v = _grid_bf16(orc, _nan_free_codes(rng, v.shape), 0.5)
+    kc, vc = _nan_free_codes(rng, (B, Hkv, slots, d)), _nan_free_codes(rng, (B, Hkv, slots, d))
+    got = orc.prefill_chunk_fp8(kind, P, q, k, v, gate, qw, kw, bias, pos0, kc, vc, 2.0, 0.5)
+    ref = orc.prefill_chunk(kind, P, q, k, v, gate, qw, kw, bias, pos0, _grid_bf16(orc, kc, 2.0),
+                            _grid_bf16(orc, vc, 0.5))
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-13)
+
+
 def test_kv_row_fp8_codes_are_nearest_to_the_exact_rows(orc):
     """Each code's value is within half an E4M3 step of the exact prepared key / raw
     value (relative 2^-4 in the normal range); a value on the grid is exact."""
