@@ -348,10 +348,12 @@ def bench_decode_1m(torch, beam, steps, warmup, seed, fp8=False):
 
 
 class ChunkLayer:
-    """One chunk call (T new tokens after pos0 cached ones, B = 1) with its own caches."""
+    """One chunk call (T new tokens after pos0 cached ones, B = 1) with its own caches
+    (BF16, or FP8 E4M3 codes with one scale per cache tensor)."""
 
-    def __init__(self, torch, beam, kind, T, pos0, slots, seed, tag):
-        self.beam, self.kind = beam, kind
+    def __init__(self, torch, beam, kind, T, pos0, slots, seed, tag, fp8=False):
+        self.beam, self.kind, self.fp8 = beam, kind, fp8
+        self.k_scale, self.v_scale = 0.0173, 3.7   # scales an amax / 448 rule gives
         self.params = beam.default_params()
         dev = "cuda"
         ci = wl.chunk_inputs(kind, T, [pos0], slots, seed, layer=tag, with_cache=False)
@@ -363,38 +365,56 @@ class ChunkLayer:
         self.kw = torch.from_numpy(ci.k_norm_w).to(dev)
         self.bias = torch.from_numpy(ci.gate_bias).to(dev)
         self.pos0 = torch.from_numpy(ci.pos0).to(dev)
-        self.layout = beam.beam_kv_layout(kind, self.params, 1, slots)
-        self.kc = torch.empty(self.layout.bytes_k // 2, dtype=torch.bfloat16, device=dev)
-        self.vc = torch.empty_like(self.kc)
-        wl.device_normal_bf16_(self.kc, seed, f"{tag}/kc")
-        wl.device_normal_bf16_(self.vc, seed, f"{tag}/vc")
+        if fp8:
+            self.layout = beam.beam_kv_layout_fp8(kind, self.params, 1, slots)
+            self.kc = torch.empty(self.layout.bytes_k, dtype=torch.uint8, device=dev)
+            self.vc = torch.empty_like(self.kc)
+            wl.device_normal_e4m3_(self.kc, seed, f"{tag}/kc", self.k_scale)
+            wl.device_normal_e4m3_(self.vc, seed, f"{tag}/vc", self.v_scale)
+            ws = beam.beam_prefill_chunk_fp8_workspace_bytes(kind, self.params, 1, T, self.layout)
+        else:
+            self.layout = beam.beam_kv_layout(kind, self.params, 1, slots)
+            self.kc = torch.empty(self.layout.bytes_k // 2, dtype=torch.bfloat16, device=dev)
+            self.vc = torch.empty_like(self.kc)
+            wl.device_normal_bf16_(self.kc, seed, f"{tag}/kc")
+            wl.device_normal_bf16_(self.vc, seed, f"{tag}/vc")
+            ws = beam.beam_prefill_chunk_workspace_bytes(kind, self.params, 1, T, self.layout)
         self.out = torch.empty_like(self.q)
-        self.ws = torch.empty(max(16, beam.beam_prefill_chunk_workspace_bytes(
-            kind, self.params, 1, T, self.layout)), dtype=torch.uint8, device=dev)
+        self.ws = torch.empty(max(16, ws), dtype=torch.uint8, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         vis = wl.chunk_visible_pairs(T, pos0, wl.WINDOW if kind == wl.LOCAL else None)
         self.flops = vis * HEAD_FLOPS_PER_PAIR
         ctx = [pos0 + T]
-        self.bytes = decode_kv_bytes(ctx, kind) + (T - 1) * 2 * 2 * (3 * 6144 + 2 * 1024)
-        # prologue (with the ring copy or the value padding), split-K attention, merge
-        self.launches_per_call = 3
+        self.bytes = decode_kv_bytes(ctx, kind, elem_bytes=1 if fp8 else 2) + \
+            (T - 1) * 2 * 2 * (3 * 6144 + 2 * 1024)
+        # prologue (with the ring copy or the value padding), split-K attention, and for a
+        # global layer at 1M context (37 runs per KV head) the merge kernel; a local layer's
+        # 5 runs are merged by the attention kernel's last CTA
+        self.launches_per_call = 2 if kind == wl.LOCAL else 3
 
     def run(self):
+        if self.fp8:
+            self.beam.beam_attn_prefill_chunk_fp8(
+                self.kind, self.params, self.q, self.k, self.v, self.gate, self.qw, self.kw,
+                self.bias, self.pos0, self.out, self.kc, self.vc, self.layout, self.k_scale,
+                self.v_scale, workspace=self.ws, dev_status=self.status)
+            return
         self.beam.beam_attn_prefill_chunk(self.kind, self.params, self.q, self.k, self.v, self.gate,
                                           self.qw, self.kw, self.bias, self.pos0, self.out,
                                           self.kc, self.vc, self.layout, workspace=self.ws,
                                           dev_status=self.status)
 
 
-def bench_decode_multi_1m(torch, beam, steps, warmup, seed, T=8):
+def bench_decode_multi_1m(torch, beam, steps, warmup, seed, T=8, fp8=False):
     """52-layer step verifying T = 8 drafted tokens at context 1,048,576 (the last T positions
-    of the 1M window): every layer is one chunk call of T new tokens; one CUDA graph."""
+    of the 1M window): every layer is one chunk call of T new tokens; one CUDA graph.  With
+    fp8, over FP8 E4M3 caches (9 global caches of 2 GiB)."""
     pos0 = wl.MAX_CONTEXT - T
     layers = []
     for i in range(1, wl.N_LAYERS + 1):
         kind = wl.layer_kind(i)
         slots = wl.MAX_CONTEXT if kind == wl.GLOBAL else wl.WINDOW
-        layers.append(ChunkLayer(torch, beam, kind, T, pos0, slots, seed, f"dm/L{i}"))
+        layers.append(ChunkLayer(torch, beam, kind, T, pos0, slots, seed, f"dm/L{i}", fp8=fp8))
 
     def step():
         for L in layers:
@@ -412,8 +432,10 @@ def bench_decode_multi_1m(torch, beam, steps, warmup, seed, T=8):
     assert all(int(L.status.item()) == 0 for L in layers)
     total_bytes = sum(L.bytes for L in layers)
     res = {
-        "workload": f"decode_multi_1m: B=1, {T} new tokens per step after {pos0} cached, 52 layers "
-                    "(9 global 4 GiB caches, 43 x 512-slot rings)",
+        "workload": (f"decode_multi_1m_fp8: B=1, {T} new tokens per step after {pos0} cached, 52 "
+                     "layers, FP8 E4M3 caches (9 global 2 GiB caches, 43 x 512-slot rings)") if fp8
+        else (f"decode_multi_1m: B=1, {T} new tokens per step after {pos0} cached, 52 layers "
+              "(9 global 4 GiB caches, 43 x 512-slot rings)"),
         "ms_per_step": sec * 1e3,
         "tokens_per_s": T / sec,
         "kv_read_GBps": total_bytes / sec / 1e9,
@@ -748,6 +770,8 @@ def run_gpu(args):
         result["decode_1m_fp8"] = hbm_fracs(d8)
         dm = bench_decode_multi_1m(torch, beam, args.steps, args.warmup, args.seed)
         result["decode_multi_1m"] = hbm_fracs(dm)
+        dm8 = bench_decode_multi_1m(torch, beam, args.steps, args.warmup, args.seed, fp8=True)
+        result["decode_multi_1m_fp8"] = hbm_fracs(dm8)
         pc = bench_prefill_chunk(torch, beam, args.steps, args.warmup, args.seed)
         pc["pct_of_bf16_peak"] = round(100 * pc["tflops"] / pk["bf16_tflops"], 2)
         result["prefill_chunk"] = pc

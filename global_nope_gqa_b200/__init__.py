@@ -29,6 +29,7 @@ EXPORTS = (
     "beam_kv_append", "beam_decode_workspace_bytes", "beam_attn_decode", "beam_status_string",
     "beam_attn_decode_noalloc", "beam_prefill_chunk_workspace_bytes", "beam_attn_prefill_chunk",
     "beam_kv_layout_fp8", "beam_kv_append_fp8", "beam_attn_decode_fp8",
+    "beam_prefill_chunk_fp8_workspace_bytes", "beam_attn_prefill_chunk_fp8",
 )
 
 
@@ -83,6 +84,12 @@ def lib() -> ctypes.CDLL:
         L.beam_attn_prefill_chunk.restype = ctypes.c_int
         L.beam_attn_prefill_chunk.argtypes = [ctypes.c_int, pp, i32, i32, vp, vp, vp, vp, vp, vp, vp,
                                               vp, vp, vp, vp, lp, vp, sz, vp, vp]
+        L.beam_prefill_chunk_fp8_workspace_bytes.restype = sz
+        L.beam_prefill_chunk_fp8_workspace_bytes.argtypes = [ctypes.c_int, pp, i32, i32, lp]
+        L.beam_attn_prefill_chunk_fp8.restype = ctypes.c_int
+        L.beam_attn_prefill_chunk_fp8.argtypes = [ctypes.c_int, pp, i32, i32, vp, vp, vp, vp, vp,
+                                                  vp, vp, vp, vp, vp, vp, lp, ctypes.c_float,
+                                                  ctypes.c_float, vp, sz, vp, vp]
         L.beam_kv_append.restype = ctypes.c_int
         L.beam_kv_append.argtypes = [ctypes.c_int, pp, i32, i32, vp, vp, vp, vp, vp, vp, lp, vp, vp]
         L.beam_decode_workspace_bytes.restype = sz
@@ -200,6 +207,31 @@ def beam_attn_prefill_chunk(kind, params, q, k, v, gate, q_norm_w, k_norm_w, gat
         _ptr(k_norm_w), _ptr(gate_bias), _ptr(pos0), _ptr(out), _ptr(k_cache), _ptr(v_cache),
         ctypes.byref(layout), _ptr(workspace), ws_bytes, _ptr(dev_status), _stream(stream))
     _check("beam_attn_prefill_chunk", rc)
+    return out
+
+
+def beam_prefill_chunk_fp8_workspace_bytes(kind: int, params: Params, B: int, T: int,
+                                           layout: KVLayout) -> int:
+    return lib().beam_prefill_chunk_fp8_workspace_bytes(kind, ctypes.byref(params), B, T,
+                                                        ctypes.byref(layout))
+
+
+def beam_attn_prefill_chunk_fp8(kind, params, q, k, v, gate, q_norm_w, k_norm_w, gate_bias, pos0,
+                                out, k_cache, v_cache, layout: KVLayout, k_scale: float,
+                                v_scale: float, workspace=None, dev_status=None, stream=None):
+    """Chunked prefill over FP8 E4M3 caches (uint8 code arrays, FP8 layout, one scale per
+    cache tensor); otherwise as beam_attn_prefill_chunk."""
+    B, T = q.shape[0], q.shape[1]
+    need = beam_prefill_chunk_fp8_workspace_bytes(kind, params, B, T, layout)
+    if workspace is None and need:
+        workspace = _workspace(need, q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib().beam_attn_prefill_chunk_fp8(
+        kind, ctypes.byref(params), B, T, _ptr(q), _ptr(k), _ptr(v), _ptr(gate), _ptr(q_norm_w),
+        _ptr(k_norm_w), _ptr(gate_bias), _ptr(pos0), _ptr(out), _ptr(k_cache), _ptr(v_cache),
+        ctypes.byref(layout), float(k_scale), float(v_scale), _ptr(workspace), ws_bytes,
+        _ptr(dev_status), _stream(stream))
+    _check("beam_attn_prefill_chunk_fp8", rc)
     return out
 
 

@@ -67,11 +67,11 @@ int device_info(DeviceInfo **out) {
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem),
                           "decode shared-memory opt-in")))
       return st;
-    if ((st = cuda_status(cudaFuncSetAttribute(decode_tc_kernel,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               kDtSmemBytes),
-                          "multi-token decode shared-memory opt-in")))
-      return st;
+    for (auto kernel : {decode_tc_kernel<false>, decode_tc_kernel<true>})
+      if ((st = cuda_status(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 kDtSmemBytes),
+                            "multi-token decode shared-memory opt-in")))
+        return st;
     if ((st = cuda_status(cudaFuncSetAttribute(decode8_attn_kernel<false>,
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, kDec8Smem),
                           "FP8 decode shared-memory opt-in")))
@@ -180,19 +180,37 @@ int make_cache_map(CUtensorMap *map, const void *base, const beam_kv_layout_t *L
   return r == CUDA_SUCCESS ? BEAM_OK : BEAM_ERR_CUDA;
 }
 
+// 4-D map over an FP8 cache [B][8][slots][128] of one-byte codes: coordinates (d, slot,
+// head, b), 128-byte swizzled boxes of 128 codes x 128 slots; slots past the capacity read
+// as zero codes.
+int make_cache_map_u8(CUtensorMap *map, const void *base, const beam_kv_layout_t *L, int B) {
+  const cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)L->slots_per_seq, (cuuint64_t)kHkv,
+                              (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)L->stride_slot, (cuuint64_t)L->stride_head,
+                                 (cuuint64_t)L->stride_seq};
+  const cuuint32_t box[4] = {(cuuint32_t)kD, (cuuint32_t)kTcBN, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = g_encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void *>(base),
+                              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? BEAM_OK : BEAM_ERR_CUDA;
+}
+
 // The persistent tcgen05 attention kernel over B sequences of T query rows.  The caller
 // fills the pointers and the chunk fields of `fa`; the shape and scale fields are set here.
+// k_scale: the keys' factor over an FP8 cache (1 for bf16), folded into the score scale.
 int launch_prefill_attention(int kind, const beam_attn_params *p, int32_t B, int32_t T,
                              const CUtensorMap &tm_q, const CUtensorMap &tm_k,
                              const CUtensorMap &tm_v, PrefillTcArgs fa, const DeviceInfo *dev,
-                             cudaStream_t s) {
+                             cudaStream_t s, float k_scale = 1.0f) {
   fa.eps = p->rms_eps;
   fa.B = B;
   fa.T = T;
   fa.kind = kind;
   fa.window = p->window;
   fa.n_qblocks = (T + kTcBM - 1) / kTcBM;
-  fa.scale_log2 = p->softmax_scale * kLog2e;
+  fa.scale_log2 = p->softmax_scale * kLog2e * k_scale;
   fa.ssmax_base = p->ssmax_base;
   fa.ssmax_exp = p->ssmax_exp;
   // Fault injection for tests of the device-timeout path: with BEAM_FAULT_INJECT set to
@@ -335,12 +353,9 @@ int beam_attn_prefill(int kind, const beam_attn_params *p, int32_t B, int32_t T,
 
   PrologueArgs pa;
   memset(&pa, 0, sizeof pa);
-  pa.q = static_cast<const uint16_t *>(q);
   pa.k = static_cast<const uint16_t *>(k);
   pa.v = static_cast<const uint16_t *>(v);
-  pa.qw = q_norm_w;
-  pa.kw = k_norm_w;
-  pa.q_out = nullptr;  // queries are normalised inside the attention kernel
+  pa.kw = k_norm_w;   // queries are normalised inside the attention kernel
   pa.k_out = kn;
   pa.rope_tab = kind == BEAM_LOCAL ? rope_tab : nullptr;
   pa.k_cache = static_cast<uint16_t *>(k_cache);
@@ -373,6 +388,7 @@ int beam_attn_prefill(int kind, const beam_attn_params *p, int32_t B, int32_t T,
   fa.gate_bias = gate_bias;
   fa.out = static_cast<uint16_t *>(out);
   fa.status = dev_status;
+  fa.v_scale = 1.0f;
   return launch_prefill_attention(kind, p, B, T, tm_q, tm_k, tm_v, fa, dev, s);
 }
 
@@ -406,17 +422,80 @@ MultiPlan multi_plan(int kind, const beam_attn_params *p, int32_t B, int32_t T, 
   return m;
 }
 
-size_t multi_partial_bytes(int32_t B, const MultiPlan &m) {
-  const size_t parts = (size_t)B * kHkv * m.n_mt * m.n_split_max * 16;
-  return round_up(parts * kD * 4, 256) + round_up(parts * 2 * 4, 256);
+// One bf16 view of an FP8 cache (the cache's element strides, two bytes an element).
+size_t fp8_view_bytes(int32_t B, const beam_kv_layout_t *layout) {
+  return round_up((size_t)B * (size_t)layout->stride_seq * 2, 256);
 }
 
+// Runs per sequence up to which the multi-token kernel merges them itself (the last CTA of
+// each (sequence, KV head)); beyond it a merge kernel spreads the work over many CTAs.
+constexpr int kFoldMaxSplits = 8;
+
+// partials o [B][8][n_mt][n_split_max][16][128] and (m, l), then the merge tickets [B][8]
+size_t multi_partial_bytes(int32_t B, const MultiPlan &m) {
+  const size_t parts = (size_t)B * kHkv * m.n_mt * m.n_split_max * 16;
+  return round_up(parts * kD * 4, 256) + round_up(parts * 2 * 4, 256) +
+         round_up((size_t)B * kHkv * 4, 256);
+}
+
+size_t chunk_workspace_bytes(int kind, const beam_attn_params *p, int32_t B, int32_t T,
+                             const beam_kv_layout_t *layout, bool fp8);
+int chunk_call(int kind, const beam_attn_params *p, int32_t B, int32_t T, const void *q,
+               const void *k, const void *v, const void *gate, const float *q_norm_w,
+               const float *k_norm_w, const float *gate_bias, const int64_t *pos0, void *out,
+               void *k_cache, void *v_cache, const beam_kv_layout_t *layout, void *workspace,
+               size_t workspace_bytes, int32_t *dev_status, beam_stream_t stream, bool fp8,
+               float k_scale, float v_scale);
+
 }  // namespace
+
 
 extern "C" {
 
 size_t beam_prefill_chunk_workspace_bytes(int kind, const beam_attn_params *p, int32_t B,
                                           int32_t T, const beam_kv_layout_t *layout) {
+  return chunk_workspace_bytes(kind, p, B, T, layout, false);
+}
+
+size_t beam_prefill_chunk_fp8_workspace_bytes(int kind, const beam_attn_params *p, int32_t B,
+                                              int32_t T, const beam_kv_layout_t *layout) {
+  if (kind == BEAM_GLOBAL && !layout) return 0;
+  return chunk_workspace_bytes(kind, p, B, T, layout, true);
+}
+
+int beam_attn_prefill_chunk(int kind, const beam_attn_params *p, int32_t B, int32_t T,
+                            const void *q, const void *k, const void *v, const void *gate,
+                            const float *q_norm_w, const float *k_norm_w, const float *gate_bias,
+                            const int64_t *pos0, void *out, void *k_cache, void *v_cache,
+                            const beam_kv_layout_t *layout, void *workspace,
+                            size_t workspace_bytes, int32_t *dev_status, beam_stream_t stream) {
+  return chunk_call(kind, p, B, T, q, k, v, gate, q_norm_w, k_norm_w, gate_bias, pos0, out,
+                    k_cache, v_cache, layout, workspace, workspace_bytes, dev_status, stream,
+                    false, 1.0f, 1.0f);
+}
+
+int beam_attn_prefill_chunk_fp8(int kind, const beam_attn_params *p, int32_t B, int32_t T,
+                                const void *q, const void *k, const void *v, const void *gate,
+                                const float *q_norm_w, const float *k_norm_w,
+                                const float *gate_bias, const int64_t *pos0, void *out,
+                                void *k_cache, void *v_cache, const beam_kv_layout_t *layout,
+                                float k_scale, float v_scale, void *workspace,
+                                size_t workspace_bytes, int32_t *dev_status, beam_stream_t stream) {
+  return chunk_call(kind, p, B, T, q, k, v, gate, q_norm_w, k_norm_w, gate_bias, pos0, out,
+                    k_cache, v_cache, layout, workspace, workspace_bytes, dev_status, stream,
+                    true, k_scale, v_scale);
+}
+
+}  // extern "C"
+
+namespace {
+
+// Workspace of a chunk call: for a local layer the ring rows it still sees and the new rows
+// ([B][window - 1 + T][8][128] bf16, keys and values) and the RoPE table [B][T][128] fp32;
+// for T <= 16 the split-K partials and merge tickets; for a global layer over an FP8 cache
+// the bf16 view of the cache (keys and values, the cache's element strides) at the end.
+size_t chunk_workspace_bytes(int kind, const beam_attn_params *p, int32_t B, int32_t T,
+                             const beam_kv_layout_t *layout, bool fp8) {
   if (!p || B <= 0 || T <= 0 || p->window < 1) return 0;
   size_t bytes = 0;
   if (kind == BEAM_LOCAL) {
@@ -432,15 +511,18 @@ size_t beam_prefill_chunk_workspace_bytes(int kind, const beam_attn_params *p, i
     const int64_t slots = layout ? layout->slots_per_seq : (int64_t)p->window;
     bytes += multi_partial_bytes(B, multi_plan(kind, p, B, T, slots, sm));
   }
+  // a long global chunk over an FP8 cache reads a bf16 view; a few-token one widens the
+  // code tiles in the kernel
+  if (fp8 && kind == BEAM_GLOBAL && T > kMultiMaxT) bytes += 2 * fp8_view_bytes(B, layout);
   return bytes;
 }
 
-int beam_attn_prefill_chunk(int kind, const beam_attn_params *p, int32_t B, int32_t T,
-                            const void *q, const void *k, const void *v, const void *gate,
-                            const float *q_norm_w, const float *k_norm_w, const float *gate_bias,
-                            const int64_t *pos0, void *out, void *k_cache, void *v_cache,
-                            const beam_kv_layout_t *layout, void *workspace,
-                            size_t workspace_bytes, int32_t *dev_status, beam_stream_t stream) {
+int chunk_call(int kind, const beam_attn_params *p, int32_t B, int32_t T, const void *q,
+               const void *k, const void *v, const void *gate, const float *q_norm_w,
+               const float *k_norm_w, const float *gate_bias, const int64_t *pos0, void *out,
+               void *k_cache, void *v_cache, const beam_kv_layout_t *layout, void *workspace,
+               size_t workspace_bytes, int32_t *dev_status, beam_stream_t stream, bool fp8,
+               float k_scale, float v_scale) {
   int st = check_params(kind, p);
   if (st) return st;
   if (B < 0 || T < 0) return BEAM_ERR_INVALID_ARG;
@@ -452,11 +534,12 @@ int beam_attn_prefill_chunk(int kind, const beam_attn_params *p, int32_t B, int3
       !aligned16(q_norm_w) || !aligned16(k_norm_w) || !aligned16(k_cache) || !aligned16(v_cache) ||
       !aligned16(workspace) || (reinterpret_cast<uintptr_t>(pos0) & 7u))
     return BEAM_ERR_ALIGNMENT;
-  if ((st = check_layout(kind, p, layout))) return st;
+  if ((st = fp8 ? check_layout_fp8(kind, p, layout) : check_layout(kind, p, layout))) return st;
+  if (fp8 && (!valid_scale(k_scale) || !valid_scale(v_scale))) return BEAM_ERR_INVALID_ARG;
   const bool local = kind == BEAM_LOCAL;
   if (!local && layout->slots_per_seq < T) return BEAM_ERR_CAPACITY;
   if (!local && layout->slots_per_seq > INT32_MAX - kTcBN) return BEAM_ERR_UNSUPPORTED;
-  const size_t need = beam_prefill_chunk_workspace_bytes(kind, p, B, T, layout);
+  const size_t need = chunk_workspace_bytes(kind, p, B, T, layout, fp8);
   if (need && (!workspace || workspace_bytes < need)) return BEAM_ERR_WORKSPACE;
   const int64_t ext_rows = local ? (int64_t)p->window - 1 + T : T;
   if ((int64_t)B * ext_rows > INT32_MAX) return BEAM_ERR_UNSUPPORTED;
@@ -479,7 +562,9 @@ int beam_attn_prefill_chunk(int kind, const beam_attn_params *p, int32_t B, int3
   ChunkPrepArgs ca;
   ca.pos0 = pos0;
   ca.k_cache = static_cast<const uint16_t *>(k_cache);
-  ca.v_cache = static_cast<uint16_t *>(v_cache);
+  ca.v_cache = static_cast<uint16_t *>(v_cache);   // the view instead for an FP8 cache (below)
+  ca.v_ring = static_cast<const uint16_t *>(v_cache);
+  ca.fp8 = fp8;
   ca.stride_seq = layout->stride_seq;
   ca.stride_head = layout->stride_head;
   ca.slots = layout->slots_per_seq;
@@ -492,13 +577,58 @@ int beam_attn_prefill_chunk(int kind, const beam_attn_params *p, int32_t B, int3
   ca.kind = kind;
   const int64_t prep_ctas = (int64_t)B * (local ? prefix : kChunkPadRows);
 
+  // the few-token path's plan and workspace (split-K partials, merge tickets)
+  const bool few = T <= kMultiMaxT;
+  MultiPlan mp{};
+  uint8_t *pw = nullptr;
+  size_t parts = 0;
+  bool fold = false;
+  if (few) {
+    mp = multi_plan(kind, p, B, T, layout->slots_per_seq, dev->sm_count);
+    pw = static_cast<uint8_t *>(workspace) +
+         (local ? 2 * ext_bytes + round_up((size_t)B * T * 128 * 4, 256) : 0);
+    parts = (size_t)B * kHkv * mp.n_mt * mp.n_split_max * 16;
+    fold = mp.n_split_max > 1 && mp.n_split_max <= kFoldMaxSplits;
+  }
+  uint32_t *tickets = few ? reinterpret_cast<uint32_t *>(pw + round_up(parts * kD * 4, 256) +
+                                                         round_up(parts * 2 * 4, 256))
+                          : nullptr;
+  // a global layer over an FP8 cache: the attention reads a bf16 view of the cache (the
+  // codes' unscaled values) at the end of the workspace; the cached rows are converted
+  // first, the prologue writes the new rows into both
+  uint16_t *k_view = nullptr, *v_view = nullptr;
+  const bool widen_in_kernel = fp8 && !local && few;   // decode_tc_kernel<true>
+  if (fp8 && !local && !few) {
+    const size_t vb = fp8_view_bytes(B, layout);
+    uint8_t *end = static_cast<uint8_t *>(workspace) + need;
+    k_view = reinterpret_cast<uint16_t *>(end - 2 * vb);
+    v_view = reinterpret_cast<uint16_t *>(end - vb);
+    Fp8ViewArgs fv;
+    fv.pos0 = pos0;
+    fv.k_codes = static_cast<const uint8_t *>(k_cache);
+    fv.v_codes = static_cast<const uint8_t *>(v_cache);
+    fv.k_view = k_view;
+    fv.v_view = v_view;
+    fv.stride_seq = layout->stride_seq;
+    fv.stride_head = layout->stride_head;
+    fv.slots = layout->slots_per_seq;
+    const int64_t blocks = (layout->slots_per_seq + kViewSlots - 1) / kViewSlots;
+    if (blocks > INT32_MAX || B > 65535) return BEAM_ERR_UNSUPPORTED;
+    fp8_view_kernel<<<dim3((unsigned)blocks, kHkv, B), 256, 0, s>>>(fv);
+    if ((st = launch_status())) return st;
+  }
+  // the caches the attention kernels read as bf16
+  void *k_att = k_view ? static_cast<void *>(k_view) : k_cache;
+  void *v_att = v_view ? static_cast<void *>(v_view) : v_cache;
+  ca.v_cache = static_cast<uint16_t *>(v_att);   // global: the value padding the attention reads
+
   // 1. prepared keys (and raw values) of the new tokens: into the cache and, for a local
-  //    layer, behind the earlier rows; the RoPE table at each sequence's own positions
+  //    layer, behind the earlier rows; the RoPE table at each sequence's own positions (and
+  //    the merge tickets of the few-token path zeroed)
   PrologueArgs pa;
   memset(&pa, 0, sizeof pa);
   pa.k = static_cast<const uint16_t *>(k);
   pa.v = static_cast<const uint16_t *>(v);
-  pa.qw = q_norm_w;
   pa.kw = k_norm_w;
   pa.k_out = k_ext;
   pa.v_out = v_ext;
@@ -520,28 +650,35 @@ int beam_attn_prefill_chunk(int kind, const beam_attn_params *p, int32_t B, int3
   pa.eps = p->rms_eps;
   fill_inv_freq(pa.inv_freq, p->rope_theta);
   pa.prep = ca;
-  pa.n_prep = (int)prep_ctas;
+  // the in-kernel widening zeroes keys past the last visible one itself: no value padding
+  // (which would treat the code array as bf16)
+  pa.n_prep = widen_in_kernel ? 0 : (int)prep_ctas;
   pa.ring_save = local;
-  if ((int64_t)B * T + prep_ctas > INT32_MAX) return BEAM_ERR_UNSUPPORTED;
-  prologue_kernel<<<(unsigned)((int64_t)B * T + prep_ctas), 128, 0, s>>>(pa);
+  pa.tickets = fold ? tickets : nullptr;
+  pa.cache_fp8 = fp8;
+  pa.k_scale = k_scale;
+  pa.v_scale = v_scale;
+  pa.k_view = k_view;
+  pa.v_view = v_view;
+  if ((int64_t)B * T + pa.n_prep > INT32_MAX) return BEAM_ERR_UNSUPPORTED;
+  prologue_kernel<<<(unsigned)((int64_t)B * T + pa.n_prep), 128, 0, s>>>(pa);
   if ((st = launch_status())) return st;
 
   // 2. attention of the new rows over the earlier and the new keys
-  if (T <= kMultiMaxT) {
-    // a few new tokens (multi-token decode): split the keys across CTAs, then merge
-    const MultiPlan mp = multi_plan(kind, p, B, T, layout->slots_per_seq, dev->sm_count);
-    uint8_t *pw = static_cast<uint8_t *>(workspace) + (local ? 2 * ext_bytes +
-                                                       round_up((size_t)B * T * 128 * 4, 256)
-                                                             : 0);
-    const size_t parts = (size_t)B * kHkv * mp.n_mt * mp.n_split_max * 16;
+  if (few) {
+    // a few new tokens (multi-token decode): split the keys across CTAs, then merge (in the
+    // same kernel when a sequence's keys span at most kFoldMaxSplits runs)
     if ((st = encode_fn())) return st;
     CUtensorMap tk, tv;
     if (local) {
       if ((st = make_head_map(&tk, k_ext, kHkv, (int)ext_rows, B))) return st;
       if ((st = make_head_map(&tv, v_ext, kHkv, (int)ext_rows, B))) return st;
+    } else if (widen_in_kernel) {
+      if ((st = make_cache_map_u8(&tk, k_cache, layout, B))) return st;
+      if ((st = make_cache_map_u8(&tv, v_cache, layout, B))) return st;
     } else {
-      if ((st = make_cache_map(&tk, k_cache, layout, B))) return st;
-      if ((st = make_cache_map(&tv, v_cache, layout, B))) return st;
+      if ((st = make_cache_map(&tk, k_att, layout, B))) return st;
+      if ((st = make_cache_map(&tv, v_att, layout, B))) return st;
     }
     DecodeTcArgs da;
     memset(&da, 0, sizeof da);
@@ -568,6 +705,10 @@ int beam_attn_prefill_chunk(int kind, const beam_attn_params *p, int32_t B, int3
     // a plan with one split (many sequences, or a short history) needs no merge: the CTA
     // that sees every key of its (sequence, KV head) writes the gated output itself
     da.direct = mp.n_split_max == 1;
+    da.fold = fold;
+    da.tickets = tickets;
+    da.k_scale = k_scale;
+    da.v_scale = v_scale;
     da.gate = static_cast<const uint16_t *>(gate);
     da.gate_bias = gate_bias;
     da.out = static_cast<uint16_t *>(out);
@@ -576,9 +717,14 @@ int beam_attn_prefill_chunk(int kind, const beam_attn_params *p, int32_t B, int3
       da.fault_stall = f != nullptr && std::strcmp(f, "prefill_wait_stall") == 0;
     }
     if (mp.n_split_max > 65535 || B > 65535) return BEAM_ERR_UNSUPPORTED;
-    decode_tc_kernel<<<dim3(mp.n_split_max, kHkv, B), kDtThreads, kDtSmemBytes, s>>>(tk, tv, da);
+    if (widen_in_kernel)
+      decode_tc_kernel<true><<<dim3(mp.n_split_max, kHkv, B), DtCfg<true>::kThreads, kDtSmemBytes,
+                               s>>>(tk, tv, da);
+    else
+      decode_tc_kernel<false><<<dim3(mp.n_split_max, kHkv, B), DtCfg<false>::kThreads,
+                                kDtSmemBytes, s>>>(tk, tv, da);
     if ((st = launch_status())) return st;
-    if (da.direct) return BEAM_OK;
+    if (da.direct || da.fold) return BEAM_OK;
     MultiCombineArgs mc;
     mc.part_o = da.part_o;
     mc.part_ml = da.part_ml;
@@ -604,8 +750,8 @@ int beam_attn_prefill_chunk(int kind, const beam_attn_params *p, int32_t B, int3
     if ((st = make_head_map(&tm_k, k_ext, kHkv, (int)ext_rows, B))) return st;
     if ((st = make_head_map(&tm_v, v_ext, kHkv, (int)ext_rows, B))) return st;
   } else {
-    if ((st = make_cache_map(&tm_k, k_cache, layout, B))) return st;
-    if ((st = make_cache_map(&tm_v, v_cache, layout, B))) return st;
+    if ((st = make_cache_map(&tm_k, k_att, layout, B))) return st;
+    if ((st = make_cache_map(&tm_v, v_att, layout, B))) return st;
   }
   PrefillTcArgs fa;
   memset(&fa, 0, sizeof fa);
@@ -620,8 +766,13 @@ int beam_attn_prefill_chunk(int kind, const beam_attn_params *p, int32_t B, int3
   fa.slots = layout->slots_per_seq;
   fa.ext_prefix = prefix;
   fa.kv_slot_major = local ? 0 : 1;
-  return launch_prefill_attention(kind, p, B, T, tm_q, tm_k, tm_v, fa, dev, s);
+  fa.v_scale = v_scale;
+  return launch_prefill_attention(kind, p, B, T, tm_q, tm_k, tm_v, fa, dev, s, k_scale);
 }
+
+}  // namespace
+
+extern "C" {
 
 int beam_kv_append(int kind, const beam_attn_params *p, int32_t B, int32_t T, const void *k,
                    const void *v, const float *k_norm_w, const int64_t *pos0, void *k_cache,
@@ -643,7 +794,6 @@ int beam_kv_append(int kind, const beam_attn_params *p, int32_t B, int32_t T, co
   memset(&pa, 0, sizeof pa);
   pa.k = static_cast<const uint16_t *>(k);
   pa.v = static_cast<const uint16_t *>(v);
-  pa.qw = k_norm_w;  // unused: no query rows
   pa.kw = k_norm_w;
   pa.k_cache = static_cast<uint16_t *>(k_cache);
   pa.v_cache = static_cast<uint16_t *>(v_cache);
@@ -848,7 +998,6 @@ int beam_kv_append_fp8(int kind, const beam_attn_params *p, int32_t B, int32_t T
   memset(&pa, 0, sizeof pa);
   pa.k = static_cast<const uint16_t *>(k);
   pa.v = static_cast<const uint16_t *>(v);
-  pa.qw = k_norm_w;  // unused: no query rows
   pa.kw = k_norm_w;
   pa.k_cache = static_cast<uint16_t *>(k_cache);
   pa.v_cache = static_cast<uint16_t *>(v_cache);

@@ -83,34 +83,62 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
   return (uint32_t)h.x | ((uint32_t)h.y << 16);
 }
 
-// x / scale rounded to fp32 by round-to-odd: the quotient is formed by IEEE fp64 division
-// (correctly rounded), truncated to fp32, and the last significand bit is set when the
-// truncation dropped anything.  Rounding that fp32 value once more to nearest at 4
-// significant bits (E4M3) gives the nearest E4M3 value of the fp64 quotient -- no double
-// rounding -- because 24 >= 4 + 2 (round-to-odd: S. Boldo, G. Melquiond, "Emulation of
-// FMA and correctly rounded sums: proved algorithms using rounding to odd", IEEE Trans.
-// Computers 57(4), 2008).  Magnitudes past the fp32 range truncate to FLT_MAX, which the
-// saturating conversion maps to 448 like any other value past 448.
-__device__ __forceinline__ float div_to_f32_odd(float x, double scale) {
-  const double q = (double)x / scale;
-  float f = __double2float_rz(q);
-  if ((double)f != q) f = __uint_as_float(__float_as_uint(f) | 1u);
-  return f;
+// Eight E4M3 codes (low byte first) -> their eight values as bf16, exactly (an E4M3 value
+// has 4 significant bits and an exponent within bf16's range): the unscaled values an
+// FP8 cache row holds, in the form the bf16 tensor-core kernels read.
+__device__ __forceinline__ uint4 e4m3x8_to_bf16x8(const uint2 codes) {
+  const uint32_t pairs[4] = {codes.x & 0xFFFFu, codes.x >> 16, codes.y & 0xFFFFu, codes.y >> 16};
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t h = e4m3x2_to_f16x2(pairs[i]);
+    w[i] = pack_bf16(__half2float(__ushort_as_half((unsigned short)(h & 0xFFFFu))),
+                     __half2float(__ushort_as_half((unsigned short)(h >> 16))));
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// The nearest E4M3 code of a double, ties to the even code, magnitudes from 448 up
+// saturating to 448 (OCP E4M3: sign, 4 exponent bits with bias 7, 3 fraction bits,
+// subnormals m * 2^-9, no infinities; S.1111.111 is NaN and never produced).  Written from
+// that definition in integer arithmetic on the double's 53-bit significand, so the one
+// rounding sees every bit of its input.
+__device__ __forceinline__ uint32_t e4m3_rne(double q) {
+  const uint64_t bits = (uint64_t)__double_as_longlong(q);
+  const uint32_t sign = (uint32_t)(bits >> 63) << 7;
+  const uint64_t mag = bits & 0x7FFFFFFFFFFFFFFFull;
+  if (mag >= 0x407C000000000000ull) return sign | 0x7Eu;   // |q| >= 448 = 1.75 * 2^8
+  const int e = (int)(mag >> 52) - 1023;                    // |q| in [2^e, 2^(e + 1))
+  if (e < -21) return sign;                                 // below 2^-11: rounds to zero
+  const uint64_t sig = (1ull << 52) | (mag & ((1ull << 52) - 1));
+  if (e >= -6) {   // a normal code: keep 3 fraction bits
+    uint64_t m = sig >> 49;                                 // 8 .. 15
+    const uint64_t rem = sig & ((1ull << 49) - 1), half = 1ull << 48;
+    if (rem > half || (rem == half && (m & 1))) ++m;
+    int ee = e;
+    if (m == 16) { m = 8; ++ee; }                           // cannot pass 448 (checked above)
+    return sign | ((uint32_t)(ee + 7) << 3) | (uint32_t)(m - 8);
+  }
+  // a subnormal code: |q| in units of 2^-9 (8 is the smallest normal, code 0x08)
+  const int shift = 43 - e;                                 // 50 .. 64
+  uint64_t m = shift >= 64 ? 0 : sig >> shift;
+  const uint64_t rem = shift >= 64 ? sig : sig & ((1ull << shift) - 1);
+  const uint64_t half = 1ull << (shift - 1);
+  if (rem > half || (rem == half && (m & 1))) ++m;
+  return sign | (uint32_t)m;
 }
 
 // Eight fp32 values -> eight cache codes E4M3(x / scale) (nearest, ties to even, saturating
-// at +-448), in order: the quotient of the value and the cache's scale, not of the value
-// and a rounded reciprocal, so a code matches the nearest code of the exact quotient at any
-// finite positive scale.
+// at +-448), in order: the quotient of the value and the cache's scale, formed in fp64
+// (IEEE division, exact to 53 bits), not the product with a rounded reciprocal, so a code
+// is the nearest code of the quotient at any finite positive scale.
 __device__ __forceinline__ uint2 f32x8_to_e4m3_div(const float (&x)[8], float scale) {
   const double s = (double)scale;
-  uint32_t w[4];
+  uint32_t c[8];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
-    w[i] = __nv_cvt_float2_to_fp8x2(
-        make_float2(div_to_f32_odd(x[2 * i], s), div_to_f32_odd(x[2 * i + 1], s)),
-        __NV_SATFINITE, __NV_E4M3);
-  return make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
+  for (int i = 0; i < 8; ++i) c[i] = e4m3_rne((double)x[i] / s);
+  return make_uint2(c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24),
+                    c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24));
 }
 
 // Eight fp32 values -> eight E4M3 codes (value * mul, nearest, saturating), in order.  Used

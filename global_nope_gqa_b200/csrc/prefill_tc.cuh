@@ -91,6 +91,9 @@ struct PrefillTcArgs {
   int ext_prefix;         // local: rows of earlier keys in front of the new ones (window - 1)
   int kv_slot_major;      // K/V maps take coordinates (d, slot, head, b), not (d, head, t, b)
   int rope_rows;          // rows per sequence in rope_tab (0: one table for all sequences)
+  // Output factor: v_scale over an FP8 cache, whose K/V maps read the unscaled values of the
+  // codes (k_scale is folded into scale_log2 by the host); 1 for a bf16 cache
+  float v_scale;
 };
 
 namespace tcd {
@@ -702,7 +705,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       if (!(ok = tc_wait(bar(tcd::kOFull + t), n & 1, abort, a.status))) break;
       tc::tc_fence_after();
-      const float inv = 0.5f / l;
+      const float inv = (0.5f / l) * a.v_scale;
       const float hb = 0.5f * a.gate_bias[h];
       if constexpr (kStage) {
         // row r of the tile, with the row's swizzle (r % 8) in the chunk bits: the row starts

@@ -13,8 +13,9 @@
 // token is formed once, by one thread, in fp64 (t * frequency, then reduced to
 // [-pi, pi]), because in fp32 t * frequency is off by up to ~0.06 rad at t ~ 1e6;
 // the reduced angle then goes through fp32 sincosf, and the cos / sin values reach
-// the other threads through shared memory.  Rows: 48 query heads, 8 key heads, and
-// 8 value heads when a cache is written (copied unchanged).
+// the other threads through shared memory.  Rows: the 8 key heads, and the 8 value heads
+// when a cache is written (copied unchanged); queries are prepared inside the attention
+// kernels.
 #pragma once
 
 #include "common.cuh"
@@ -36,11 +37,13 @@ constexpr int kChunkPadRows = 128;  // global: CTAs per sequence (at most 127 sl
 
 struct ChunkPrepArgs {
   const int64_t *pos0;
-  const uint16_t *k_cache;
-  uint16_t *v_cache;
+  const uint16_t *k_cache;   // local: the ring (E4M3 codes when fp8)
+  uint16_t *v_cache;         // global: the bf16 values the attention reads (cache or FP8 view)
+  const uint16_t *v_ring;    // local: the ring's values (E4M3 codes when fp8)
   int64_t stride_seq, stride_head, slots;
   uint16_t *k_ext, *v_ext;   // local: [B][ext_rows][8*128]
   int ext_rows, prefix, T, window, kind;
+  int fp8;                   // the ring holds E4M3 codes: copy their unscaled values as bf16
 };
 
 __device__ __forceinline__ void chunk_prep_row(const ChunkPrepArgs &a, int cta) {
@@ -59,8 +62,15 @@ __device__ __forceinline__ void chunk_prep_row(const ChunkPrepArgs &a, int cta) 
     uint4 kv = make_uint4(0u, 0u, 0u, 0u), vv = kv;
     if (p0 >= 0 && j >= 0) {
       const size_t off = cache_row + (size_t)(j % a.window) * kD + c;
-      kv = *reinterpret_cast<const uint4 *>(a.k_cache + off);
-      vv = *reinterpret_cast<const uint4 *>(a.v_cache + off);
+      if (a.fp8) {
+        kv = e4m3x8_to_bf16x8(*reinterpret_cast<const uint2 *>(
+            reinterpret_cast<const uint8_t *>(a.k_cache) + off));
+        vv = e4m3x8_to_bf16x8(*reinterpret_cast<const uint2 *>(
+            reinterpret_cast<const uint8_t *>(a.v_ring) + off));
+      } else {
+        kv = *reinterpret_cast<const uint4 *>(a.k_cache + off);
+        vv = *reinterpret_cast<const uint4 *>(a.v_ring + off);
+      }
     }
     const size_t dst = ((size_t)b * a.ext_rows + e) * (kHkv * kD) + head * kD + c;
     *reinterpret_cast<uint4 *>(a.k_ext + dst) = kv;
@@ -74,12 +84,9 @@ __device__ __forceinline__ void chunk_prep_row(const ChunkPrepArgs &a, int cta) 
 }
 
 struct PrologueArgs {
-  const uint16_t *q;     // [tokens][48*128] or null (append only)
   const uint16_t *k;     // [tokens][8*128]
   const uint16_t *v;     // [tokens][8*128] (read only when a cache is written)
-  const float *qw;       // [128]
   const float *kw;       // [128]
-  uint16_t *q_out;       // [tokens][48*128] prepared queries, or null
   uint16_t *k_out;       // prepared keys [B][out_rows][8*128], or null
   uint16_t *v_out;       // raw values copied to [B][out_rows][8*128], or null
   int out_rows;          // rows per sequence in k_out / v_out (0: T)
@@ -93,6 +100,10 @@ struct PrologueArgs {
   int whole_seq;         // a sequence whose tokens do not all fit is not written at all
   int cache_fp8;         // the caches hold E4M3 codes of value / scale (one byte each)
   float k_scale, v_scale;
+  // FP8 chunk: the rows the attention reads (k_out / v_out, and the global view) hold the
+  // unscaled values of the written codes as bf16; k_view / v_view: a global layer's bf16 view
+  // of the cache (same element strides), or null
+  uint16_t *k_view, *v_view;
   int32_t *status;
   int T;                 // tokens per sequence in this call
   // chunked prefill: n_prep extra CTAs after the B * T token CTAs prepare the chunk (the
@@ -100,6 +111,7 @@ struct PrologueArgs {
   // slot of one of those rows copies the row out first
   ChunkPrepArgs prep;
   int n_prep, ring_save;
+  uint32_t *tickets;     // or null: [B][8] merge tickets of the multi-token kernel, zeroed here
   int kind;
   int window;
   float eps;
@@ -173,7 +185,7 @@ __device__ __forceinline__ void load_weights8(const float *w, int l16, float (&o
   out[4] = x1.x; out[5] = x1.y; out[6] = x1.z; out[7] = x1.w;
 }
 
-__global__ void __launch_bounds__(128) prologue_kernel(const PrologueArgs a) {
+__global__ void __launch_bounds__(128, 8) prologue_kernel(const PrologueArgs a) {
   const int n_tok = (int)gridDim.x - a.n_prep;
   if ((int)blockIdx.x >= n_tok) {   // a chunk-preparation CTA (the whole CTA returns)
     chunk_prep_row(a.prep, (int)blockIdx.x - n_tok);
@@ -182,6 +194,7 @@ __global__ void __launch_bounds__(128) prologue_kernel(const PrologueArgs a) {
   const int tok = blockIdx.x;
   const int b = tok / a.T;
   const int i = tok - b * a.T;
+  if (a.tickets && i == 0 && threadIdx.x < kHkv) a.tickets[(size_t)b * kHkv + threadIdx.x] = 0u;
   const int64_t t = (a.pos0 ? a.pos0[b] : 0) + i;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int half = lane >> 4, l16 = lane & 15;
@@ -213,6 +226,16 @@ __global__ void __launch_bounds__(128) prologue_kernel(const PrologueArgs a) {
     }
   }
 
+  // Rows: half-warp w * 2 + half (0 .. 7) owns key head w * 2 + half and value head
+  // w * 2 + half.  Their loads are issued first, so that their latency overlaps the angle
+  // computation below.
+  const int head = warp * 2 + half;
+  const bool k_on = a.k_out != nullptr || write_cache;
+  const bool v_on = write_cache || a.v_out != nullptr;
+  const size_t src_off = (size_t)tok * (kHkv * kD) + head * kD + l16 * 8;
+  const uint4 raw_k = k_on ? *reinterpret_cast<const uint4 *>(a.k + src_off) : make_uint4(0u, 0u, 0u, 0u);
+  const uint4 raw_v = v_on ? *reinterpret_cast<const uint4 *>(a.v + src_off) : make_uint4(0u, 0u, 0u, 0u);
+
   // The token's 64 angles, one per thread of warps 0-1, shared through shared memory: every
   // row of the token uses the same angles (and, for the table at positions 0 .. T-1,
   // every sequence).
@@ -241,68 +264,106 @@ __global__ void __launch_bounds__(128) prologue_kernel(const PrologueArgs a) {
     sn[4] = s1.x; sn[5] = s1.y; sn[6] = s1.z; sn[7] = s1.w;
   }
 
-  float wq[8], wk[8];
-  load_weights8(a.qw, l16, wq);
+  float wk[8];
   load_weights8(a.kw, l16, wk);
 
   const unsigned half_mask = 0xFFFFu << (half * 16);  // shuffles stay inside the half-warp
-  const int n_rows = kHq + kHkv + kHkv;  // q heads, k heads, v heads
-  for (int row = warp * 2 + half; row < n_rows; row += 8) {
-    const bool is_q = row < kHq;
-    const bool is_k = !is_q && row < kHq + kHkv;
-    const bool is_v = row >= kHq + kHkv;
-    if (is_q && (a.q == nullptr || a.q_out == nullptr)) continue;
-    if (is_k && a.k_out == nullptr && !write_cache) continue;
-    if (is_v && !write_cache && a.v_out == nullptr) continue;
-    const int head = is_q ? row : (is_k ? row - kHq : row - kHq - kHkv);
-    const uint16_t *src = is_q ? a.q + (size_t)tok * (kHq * kD) + head * kD
-                               : (is_k ? a.k : a.v) + (size_t)tok * (kHkv * kD) + head * kD;
-    uint4 raw = *reinterpret_cast<const uint4 *>(src + l16 * 8);
+#pragma unroll
+  for (int kv = 0; kv < 2; ++kv) {
+    const bool is_k = kv == 0;
+    if (!(is_k ? k_on : v_on)) continue;   // the same for the whole CTA
+    const uint4 raw = is_k ? raw_k : raw_v;
     float x[8];
-    if (is_v) {
+    if (!is_k) {
       x[0] = bf16_lo(raw.x); x[1] = bf16_hi(raw.x); x[2] = bf16_lo(raw.y); x[3] = bf16_hi(raw.y);
       x[4] = bf16_lo(raw.z); x[5] = bf16_hi(raw.z); x[6] = bf16_lo(raw.w); x[7] = bf16_hi(raw.w);
     } else {
-      norm_rope_f32(raw, is_q ? wq : wk, local, cs, sn, l16, half_mask, a.eps, x);
+      norm_rope_f32(raw, wk, local, cs, sn, l16, half_mask, a.eps, x);
     }
     uint4 res = raw;
-    if (!is_v) {
+    if (is_k) {
       res.x = pack_bf16(x[0], x[1]); res.y = pack_bf16(x[2], x[3]);
       res.z = pack_bf16(x[4], x[5]); res.w = pack_bf16(x[6], x[7]);
     }
-    if (is_q) {
-      *reinterpret_cast<uint4 *>(a.q_out + (size_t)tok * (kHq * kD) + head * kD + l16 * 8) = res;
-    } else {
-      uint16_t *dst = is_k ? a.k_out : a.v_out;
-      if (dst) {
-        const size_t orow = (size_t)b * (a.out_rows ? a.out_rows : a.T) + a.out_row0 + i;
-        *reinterpret_cast<uint4 *>(dst + orow * (kHkv * kD) + head * kD + l16 * 8) = res;
-      }
-      if (write_cache) {
-        const size_t off = (size_t)b * a.stride_seq + (size_t)head * a.stride_head +
-                           (size_t)slot * kD + l16 * 8;
-        if (a.cache_fp8) {   // codes of the fp32 rows, not of their bf16 rounding
-          uint8_t *cache = reinterpret_cast<uint8_t *>(is_k ? a.k_cache : a.v_cache);
-          *reinterpret_cast<uint2 *>(cache + off) =
-              f32x8_to_e4m3_div(x, is_k ? a.k_scale : a.v_scale);
-        } else {
-          uint16_t *cache = is_k ? a.k_cache : a.v_cache;
-          const int r = a.ring_save ? i % a.window : 0;
-          if (r >= 1) {
-            // before this call the slot held position q = pos0 + r - window, row r - 1 of the
-            // earlier keys the chunk still sees: save it (zeros before position 0) before
-            // overwriting it
-            const int64_t q = (t - i) + r - a.window;
-            const uint4 old = q >= 0 ? *reinterpret_cast<const uint4 *>(cache + off)
-                                     : make_uint4(0u, 0u, 0u, 0u);
-            uint16_t *ext = is_k ? a.k_out : a.v_out;
-            *reinterpret_cast<uint4 *>(ext + ((size_t)b * a.out_rows + r - 1) * (kHkv * kD) +
-                                       head * kD + l16 * 8) = old;
-          }
-          *reinterpret_cast<uint4 *>(cache + off) = res;
+    uint16_t *dst = is_k ? a.k_out : a.v_out;
+    // an FP8 cache stores codes of the fp32 rows, not of their bf16 rounding; the attention
+    // of an FP8 chunk reads the codes' unscaled values (its scales apply in the kernel)
+    uint2 codes = make_uint2(0u, 0u);
+    if (a.cache_fp8 && (write_cache || dst)) codes = f32x8_to_e4m3_div(x, is_k ? a.k_scale : a.v_scale);
+    const uint4 att = a.cache_fp8 ? e4m3x8_to_bf16x8(codes) : res;
+    if (dst) {
+      const size_t orow = (size_t)b * (a.out_rows ? a.out_rows : a.T) + a.out_row0 + i;
+      *reinterpret_cast<uint4 *>(dst + orow * (kHkv * kD) + head * kD + l16 * 8) = att;
+    }
+    if (write_cache) {
+      const size_t off = (size_t)b * a.stride_seq + (size_t)head * a.stride_head +
+                         (size_t)slot * kD + l16 * 8;
+      if (a.cache_fp8) {
+        uint8_t *cache = reinterpret_cast<uint8_t *>(is_k ? a.k_cache : a.v_cache);
+        const int r = a.ring_save ? i % a.window : 0;
+        if (r >= 1) {   // as below, for a ring of codes: its old row's values go to the workspace
+          const int64_t q = (t - i) + r - a.window;
+          const uint4 old = q >= 0 ? e4m3x8_to_bf16x8(*reinterpret_cast<const uint2 *>(cache + off))
+                                   : make_uint4(0u, 0u, 0u, 0u);
+          uint16_t *ext = is_k ? a.k_out : a.v_out;
+          *reinterpret_cast<uint4 *>(ext + ((size_t)b * a.out_rows + r - 1) * (kHkv * kD) +
+                                     head * kD + l16 * 8) = old;
         }
+        *reinterpret_cast<uint2 *>(cache + off) = codes;
+        uint16_t *view = is_k ? a.k_view : a.v_view;
+        if (view) *reinterpret_cast<uint4 *>(view + off) = att;
+      } else {
+        uint16_t *cache = is_k ? a.k_cache : a.v_cache;
+        const int r = a.ring_save ? i % a.window : 0;
+        if (r >= 1) {
+          // before this call the slot held position q = pos0 + r - window, row r - 1 of the
+          // earlier keys the chunk still sees: save it (zeros before position 0) before
+          // overwriting it
+          const int64_t q = (t - i) + r - a.window;
+          const uint4 old = q >= 0 ? *reinterpret_cast<const uint4 *>(cache + off)
+                                   : make_uint4(0u, 0u, 0u, 0u);
+          uint16_t *ext = is_k ? a.k_out : a.v_out;
+          *reinterpret_cast<uint4 *>(ext + ((size_t)b * a.out_rows + r - 1) * (kHkv * kD) +
+                                     head * kD + l16 * 8) = old;
+        }
+        *reinterpret_cast<uint4 *>(cache + off) = res;
       }
     }
+  }
+}
+
+// The cached rows of an FP8 global cache that a chunk reads (positions 0 .. pos0[b] - 1)
+// as bf16 values of their codes, unscaled, into a view with the cache's element strides: the
+// tcgen05 attention kernels then read the view as they read a bf16 cache, and the scales
+// apply inside them.  Grid (slot blocks of 64, KV head, sequence); 256 threads move 16 codes
+// each, twice; a block past the sequence's cached rows returns at once.
+constexpr int kViewSlots = 64;
+
+struct Fp8ViewArgs {
+  const int64_t *pos0;
+  const uint8_t *k_codes, *v_codes;
+  uint16_t *k_view, *v_view;
+  int64_t stride_seq, stride_head, slots;
+};
+
+__global__ void __launch_bounds__(256) fp8_view_kernel(const Fp8ViewArgs a) {
+  const int g = blockIdx.y, b = blockIdx.z;
+  const int64_t s0 = (int64_t)blockIdx.x * kViewSlots;
+  const int64_t n = min(max(a.pos0[b], (int64_t)0), a.slots);   // cached rows of the sequence
+  if (s0 >= n) return;
+  const size_t row0 = (size_t)b * a.stride_seq + (size_t)g * a.stride_head;
+#pragma unroll
+  for (int rep = 0; rep < 2; ++rep) {
+    const int item = rep * 256 + (int)threadIdx.x;
+    const int64_t slot = s0 + item / 8;
+    if (slot >= n) continue;
+    const size_t off = row0 + (size_t)slot * kD + (item % 8) * 16;
+    const uint4 kc = *reinterpret_cast<const uint4 *>(a.k_codes + off);
+    const uint4 vc = *reinterpret_cast<const uint4 *>(a.v_codes + off);
+    *reinterpret_cast<uint4 *>(a.k_view + off) = e4m3x8_to_bf16x8(make_uint2(kc.x, kc.y));
+    *reinterpret_cast<uint4 *>(a.k_view + off + 8) = e4m3x8_to_bf16x8(make_uint2(kc.z, kc.w));
+    *reinterpret_cast<uint4 *>(a.v_view + off) = e4m3x8_to_bf16x8(make_uint2(vc.x, vc.y));
+    *reinterpret_cast<uint4 *>(a.v_view + off + 8) = e4m3x8_to_bf16x8(make_uint2(vc.z, vc.w));
   }
 }
 

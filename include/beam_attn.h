@@ -249,6 +249,34 @@ BEAM_API int beam_attn_decode_fp8(int kind, const beam_attn_params *p, int32_t B
                                   size_t workspace_bytes, int32_t *dev_status,
                                   beam_stream_t stream);
 
+/* Workspace beam_attn_prefill_chunk_fp8 needs (bytes): what
+ * beam_prefill_chunk_workspace_bytes gives for the same shapes and, for a global
+ * layer, a bf16 view of the cache (keys and values, two bytes for every element of
+ * the FP8 layout, 4 * bytes_k in all) at the end of the workspace. */
+BEAM_API size_t beam_prefill_chunk_fp8_workspace_bytes(int kind, const beam_attn_params *p,
+                                                       int32_t B, int32_t T,
+                                                       const beam_kv_layout_t *layout);
+
+/* beam_attn_prefill_chunk over FP8 E4M3 caches (layout from beam_kv_layout_fp8; one
+ * scale per cache tensor as for beam_attn_decode_fp8).  The chunk's new keys and
+ * values are written as codes first; the queries then attend over every visible key
+ * and value read back from the cache, the new ones included (the order the FP8
+ * decode takes for one new token).  Cached codes are widened to bf16 (their
+ * unscaled values, exact) in the workspace -- the ring rows a local chunk sees, or,
+ * for a global layer, the rows before each sequence's pos0 in a bf16 view of the
+ * cache -- and the tensor-core kernels of the bf16 path read them, with k_scale
+ * folded into the score scale and v_scale into the output.  Positions, status,
+ * capacity and the T <= 16 path as in beam_attn_prefill_chunk. */
+BEAM_API int beam_attn_prefill_chunk_fp8(int kind, const beam_attn_params *p, int32_t B, int32_t T,
+                                         const void *q, const void *k, const void *v,
+                                         const void *gate, const float *q_norm_w,
+                                         const float *k_norm_w, const float *gate_bias,
+                                         const int64_t *pos0, void *out, void *k_cache,
+                                         void *v_cache, const beam_kv_layout_t *layout,
+                                         float k_scale, float v_scale, void *workspace,
+                                         size_t workspace_bytes, int32_t *dev_status,
+                                         beam_stream_t stream);
+
 /* Decode without any allocation, for callers that cannot call cudaMalloc.
  *
  * There is no counterpart in the paper: this is a deployment convenience.  Some

@@ -4,11 +4,11 @@ Cache contents are seeded E4M3 codes given to both sides.  The FP8 decode is
 compared with oracle_decode_fp8 at the parity bar of the other GPU tests.  Codes
 the device writes are compared with the oracle's expected codes: value codes bit
 for bit at any finite positive scale (both sides take the nearest code of the
-exact quotient value / scale: the oracle divides in fp64, the device divides in
-fp64 and reaches fp32 by round-to-odd, so its one E4M3 rounding is exact), key
-codes within one E4M3 step (the device rounds its fp32 normalised key, the oracle
-the exact one).  The scales include ones an amax / 448 rule gives (0.0173, 3.7,
-not powers of two) and one that makes large values saturate at 448 (0.0051).
+quotient value / scale formed in fp64, rounding it once to E4M3), key codes within
+one E4M3 step (the device rounds its fp32 normalised key, the oracle the exact one).
+The scales include ones an amax / 448 rule gives (0.0173, 3.7, not powers of two)
+and one that makes large values saturate at 448 (0.0051).  One test writes every
+finite bf16 value through the append and checks each code.
 """
 import numpy as np
 import pytest
@@ -71,6 +71,37 @@ def test_kv_append_fp8_codes(env, kind, k_scale, v_scale):
             written[b, s] = True
     assert np.all(kh.transpose(0, 2, 1, 3)[~written] == 0x5A)
     assert np.all(vh.transpose(0, 2, 1, 3)[~written] == 0x5A)
+
+
+@pytest.mark.parametrize("v_scale", [3.7, 0.0173, 1.0, 0.0051])
+def test_kv_append_fp8_every_bf16_value(env, v_scale):
+    """Every finite bf16 bit pattern (non-finite ones replaced by zero) as a value, 64
+    tokens of 1024: each written code must be the oracle's nearest code of value / scale --
+    the ties, the subnormal codes and the saturation at 448 included."""
+    torch, beam, orc = env
+    params = beam.default_params()
+    P = oracle_params(orc, params)
+    T = 64
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    vals = wl.bf16_bits_to_f32(bits)
+    bits = np.where(np.isfinite(vals), bits, 0).astype(np.uint16)
+    v = bits.reshape(1, T, 1024)
+    k = wl.normal_bf16((1, T, 1024), 5, "allk")
+    kw = wl.norm_weight(5, "allkw")
+    layout = _f8_layout(beam, wl.GLOBAL, params, 1, T)
+    kc = torch.zeros((layout.bytes_k,), dtype=torch.uint8, device="cuda")
+    vc = torch.zeros_like(kc)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    beam.beam_kv_append_fp8(wl.GLOBAL, params, dev(torch, k), dev(torch, v),
+                            torch.from_numpy(kw).cuda(),
+                            torch.zeros(1, dtype=torch.int64, device="cuda"), kc, vc, layout, 1.0,
+                            v_scale, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    vh = vc.cpu().numpy().reshape(8, T, 128).transpose(1, 0, 2)   # [token][head][d]
+    for t in range(T):
+        _, vr = orc.kv_row_fp8(wl.GLOBAL, P, k[0, t], v[0, t], kw, t, 1.0, v_scale)
+        np.testing.assert_array_equal(vh[t].reshape(-1), vr.reshape(-1), err_msg=f"token {t}")
 
 
 def run_decode_fp8(torch, beam, di, kc0, vc0, k_scale, v_scale, params=None, status=None):

@@ -86,10 +86,12 @@ def gate_bias(seed: int, tag: str = "gate_bias") -> np.ndarray:
 
 def normal_e4m3(shape, seed: int, tag: str, scale: float = 1.0) -> np.ndarray:
     """FP8 E4M3 codes (uint8) of seeded N(0,1) draws divided by `scale` -- synthetic
-    cache contents; the draw is rounded to the nearest code by PyTorch's float8_e4m3fn
-    cast (values stay far inside the finite range)."""
+    cache contents; the draw is clamped to the finite range +-448 (a small scale pushes
+    the tails past it, and the cast would make those NaN) and rounded to the nearest code
+    by PyTorch's float8_e4m3fn cast."""
     import torch
     x = rng(seed, tag).standard_normal(size=shape, dtype=np.float32) / np.float32(scale)
+    x = np.clip(x, -448.0, 448.0)
     return torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
 
 
@@ -103,7 +105,8 @@ def device_normal_e4m3_(tensor_u8, seed: int, tag: str, scale: float = 1.0):
     for s in range(0, flat.numel(), chunk):
         part = flat[s:s + chunk]
         x = torch.randn(part.numel(), device=tensor_u8.device, dtype=torch.float32, generator=g)
-        part.copy_((x / scale).to(torch.float8_e4m3fn).view(torch.uint8))
+        x = (x / scale).clamp_(-448.0, 448.0)   # the cast would turn values past 448 into NaN
+        part.copy_(x.to(torch.float8_e4m3fn).view(torch.uint8))
     return tensor_u8
 
 
