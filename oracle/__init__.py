@@ -126,6 +126,12 @@ def lib():
     return _lib
 
 
+def _scale32(x) -> float:
+    """An FP8 cache scale as the library takes it: a float32 (the C ABI's `float`), so
+    that both sides divide by the same number."""
+    return float(np.float32(x))
+
+
 def _ptr(a: np.ndarray, ctype):
     assert a.flags["C_CONTIGUOUS"], "oracle inputs must be C-contiguous"
     return a.ctypes.data_as(ctypes.POINTER(ctype))
@@ -348,7 +354,7 @@ def decode_fp8(kind, P: Params, q, k, v, gate, q_norm_w, k_norm_w, gate_bias, po
         kind, ctypes.byref(P), B, _ptr(q, ctypes.c_uint16), _ptr(k, ctypes.c_uint16),
         _ptr(v, ctypes.c_uint16), _ptr(gate, ctypes.c_uint16), _ptr(qw, ctypes.c_float),
         _ptr(kw, ctypes.c_float), _ptr(bias, ctypes.c_float), _ptr(pos, ctypes.c_int64),
-        _ptr(k_codes, u8), _ptr(v_codes, u8), slots, float(k_scale), float(v_scale),
+        _ptr(k_codes, u8), _ptr(v_codes, u8), slots, _scale32(k_scale), _scale32(v_scale),
         _ptr(out, ctypes.c_double), n_threads or n_threads_default())
     if rc != 0:
         raise ValueError("oracle_decode_fp8 rejected its arguments")
@@ -376,8 +382,8 @@ def prefill_chunk_rows_fp8(kind, P: Params, q, k, v, gate, q_norm_w, k_norm_w, g
         kind, ctypes.byref(P), B, T, _ptr(q, ctypes.c_uint16), _ptr(k, ctypes.c_uint16),
         _ptr(v, ctypes.c_uint16), _ptr(gate, ctypes.c_uint16), _ptr(qw, ctypes.c_float),
         _ptr(kw, ctypes.c_float), _ptr(bias, ctypes.c_float), _ptr(pos0, i64),
-        _ptr(k_codes, ctypes.c_uint8), _ptr(v_codes, ctypes.c_uint8), slots, float(k_scale),
-        float(v_scale), rows_b.size, _ptr(rows_b, i64), _ptr(rows_i, i64),
+        _ptr(k_codes, ctypes.c_uint8), _ptr(v_codes, ctypes.c_uint8), slots, _scale32(k_scale),
+        _scale32(v_scale), rows_b.size, _ptr(rows_b, i64), _ptr(rows_i, i64),
         _ptr(out, ctypes.c_double), n_threads or n_threads_default())
     if rc != 0:
         raise ValueError("oracle_prefill_chunk_rows_fp8 rejected its arguments")
@@ -404,7 +410,7 @@ def kv_row_fp8(kind, P: Params, k_token, v_token, k_norm_w, j, k_scale: float, v
     u8 = ctypes.c_uint8
     lib().oracle_kv_row_fp8(kind, ctypes.byref(P), _ptr(k_token, ctypes.c_uint16),
                             _ptr(v_token, ctypes.c_uint16), _ptr(kw, ctypes.c_float), int(j),
-                            float(k_scale), float(v_scale), _ptr(kr, u8), _ptr(vr, u8))
+                            _scale32(k_scale), _scale32(v_scale), _ptr(kr, u8), _ptr(vr, u8))
     return kr, vr
 
 
