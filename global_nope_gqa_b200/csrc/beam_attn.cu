@@ -227,8 +227,10 @@ int launch_prefill_attention(int kind, const beam_attn_params *p, int32_t B, int
   if (int st = make_head_map(&tm_o, fa.out, kHq, T, B)) return st;
   // persistent: one CTA per SM (the kernel's shared memory admits one per SM)
   const int grid = (int)std::min<int64_t>(n_units, dev->sm_count);
-  const bool wide = ((reinterpret_cast<uintptr_t>(fa.gate) | reinterpret_cast<uintptr_t>(fa.out) |
-                      reinterpret_cast<uintptr_t>(fa.rope_tab)) & 31u) == 0;
+  // 32-byte row accesses need the gate and output rows 32-byte aligned (the RoPE table is
+  // read in 8-byte pieces)
+  const bool wide = ((reinterpret_cast<uintptr_t>(fa.gate) | reinterpret_cast<uintptr_t>(fa.out)) &
+                     31u) == 0;
   auto kernel = kind == BEAM_GLOBAL ? (wide ? prefill_tc_kernel<true, true> : prefill_tc_kernel<true, false>)
                                     : (wide ? prefill_tc_kernel<false, true> : prefill_tc_kernel<false, false>);
   kernel<<<grid, kTcThreads, kTcSmemBytes, s>>>(tm_q, tm_k, tm_v, tm_o, fa);

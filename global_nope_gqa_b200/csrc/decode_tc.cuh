@@ -397,8 +397,11 @@ __global__ void __launch_bounds__(DtCfg<kFp8>::kThreads, 1)
       }
       const float inv = rsqrtf(ss * (1.0f / kD) + a.eps);
       const float4 *w4p = reinterpret_cast<const float4 *>(a.qw);
-      const float4 *tab = local ? reinterpret_cast<const float4 *>(
-                                      a.rope_tab + ((size_t)b * a.T + (row_ok ? tok : 0)) * 128)
+      // the RoPE table is angle-major: (cos, sin) of angle i of this token's row at
+      // i * (B * T) + b * T + tok
+      const size_t rope_stride = (size_t)gridDim.z * a.T;
+      const float2 *tab = local ? reinterpret_cast<const float2 *>(a.rope_tab) +
+                                      (size_t)b * a.T + (row_ok ? tok : 0)
                                 : nullptr;
 #pragma unroll
       for (int c = 0; c < 8; ++c) {   // coordinates 8c .. 8c+7 and their partners + 64
@@ -417,15 +420,12 @@ __global__ void __launch_bounds__(DtCfg<kFp8>::kThreads, 1)
           xh[2 * e + 1] = bf16_hi(hw[e]) * inv * wh[2 * e + 1];
         }
         if (local) {  // rotate-half: coordinate i < 64 pairs with i + 64
-          const float4 c0 = __ldg(tab + 2 * c), c1 = __ldg(tab + 2 * c + 1);
-          const float4 s0 = __ldg(tab + 16 + 2 * c), s1 = __ldg(tab + 16 + 2 * c + 1);
-          const float cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-          const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
+            const float2 cs = __ldg(tab + (size_t)(8 * c + e) * rope_stride);
             const float a0 = xl[e], b0 = xh[e];
-            xl[e] = a0 * cv[e] - b0 * sv[e];
-            xh[e] = b0 * cv[e] + a0 * sv[e];
+            xl[e] = a0 * cs.x - b0 * cs.y;
+            xh[e] = b0 * cs.x + a0 * cs.y;
           }
         }
         const uint32_t sw = (uint32_t)((c ^ (r & 7)) << 4);

@@ -76,7 +76,7 @@ constexpr uint32_t kTcDrainLimit = 1u << 22;    // polls for in-flight work afte
 
 struct PrefillTcArgs {
   const float *q_norm_w;  // [128]
-  const float *rope_tab;  // local: [T][128] cos then sin of position t; null for global
+  const float *rope_tab;  // local: angle-major float2 (cos, sin) [64][rows]; null for global
   float eps;
   const uint16_t *gate;   // [B][T][48*128]
   const float *gate_bias; // [48]
@@ -90,7 +90,7 @@ struct PrefillTcArgs {
   int64_t slots;          // global: cache slots per sequence (the K/V maps cover the cache)
   int ext_prefix;         // local: rows of earlier keys in front of the new ones (window - 1)
   int kv_slot_major;      // K/V maps take coordinates (d, slot, head, b), not (d, head, t, b)
-  int rope_rows;          // rows per sequence in rope_tab (0: one table for all sequences)
+  int rope_rows;          // rows per sequence in rope_tab (0: one table of T rows for all)
   // Output factor: v_scale over an FP8 cache, whose K/V maps read the unscaled values of the
   // codes (k_scale is folded into scale_log2 by the host); 1 for a bf16 cache
   float v_scale;
@@ -468,36 +468,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   } else if (warp >= 12) {
     // ------------------------------------------------------------ Q preparation
     // RMSNorm of each raw Q row in shared memory (in place), then RoPE for a local layer;
-    // thread r owns row r of both tiles (same position, so the same angles).  The cos/sin
-    // values of a row are fetched ahead: chunks 0-1 before the Q tiles land, chunk c + 2
-    // as soon as chunk c is done.
+    // thread r owns row r of both tiles (same position, so the same angles).  The RoPE table
+    // is angle-major (entry (i, row) = (cos, sin) at i * stride + row), so the 32 rows of a
+    // warp read one contiguous run per angle; chunk 0 is fetched before the Q tiles land,
+    // chunk c + 1 while chunk c is worked.
     asm volatile("setmaxnreg.dec.sync.aligned.u32 104;\n" ::: "memory");
     const int r = threadIdx.x - 384;
     const float4 *w4 = reinterpret_cast<const float4 *>(a.q_norm_w);
+    const float2 *tab2 = reinterpret_cast<const float2 *>(a.rope_tab);
+    const size_t rope_stride = a.rope_rows ? (size_t)a.B * a.rope_rows : (size_t)a.T;
     bool ok = true;
     for (int u = blockIdx.x, n = 0; ok && u < a.n_units; u += gridDim.x, ++n) {
       const TcUnit w = tc_unit(a, u);
       const int tok = w.q0 + r;
-      const float4 *tab =
-          local ? reinterpret_cast<const float4 *>(
-                      a.rope_tab + ((size_t)w.b * a.rope_rows + min(tok, a.T - 1)) * 128)
-                : nullptr;
-      float4 tb[8];   // per slot: cos lo, cos hi, sin lo, sin hi of one chunk of 8
-      auto tab_load = [&](int c, int slot) {
-        if constexpr (kWide) {
-          tc::ld_nc_v8(tab + 2 * c, tb[4 * slot + 0], tb[4 * slot + 1]);
-          tc::ld_nc_v8(tab + 16 + 2 * c, tb[4 * slot + 2], tb[4 * slot + 3]);
-        } else {
-          tb[4 * slot + 0] = __ldg(tab + 2 * c);
-          tb[4 * slot + 1] = __ldg(tab + 2 * c + 1);
-          tb[4 * slot + 2] = __ldg(tab + 16 + 2 * c);
-          tb[4 * slot + 3] = __ldg(tab + 16 + 2 * c + 1);
+      // a global layer (kStage) has no RoPE: its instantiation carries none of this code
+      const bool rope = !kStage && local;
+      const float2 *tab =
+          rope ? tab2 + (size_t)(a.rope_rows ? w.b * a.rope_rows : 0) + min(tok, a.T - 1) : nullptr;
+      float2 tb[8];   // (cos, sin) of the 8 angles of the chunk in hand
+      const float2 *tab_next = tab;   // angle 8 c of the next chunk to fetch
+      auto tab_load = [&]() {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          tb[e] = __ldg(tab_next);
+          tab_next += rope_stride;
         }
       };
-      if (local) {
-        tab_load(0, 0);
-        tab_load(1, 1);
-      }
+      if (rope) tab_load();
       const int qset = n & 1;
       if (!(ok = tc_wait(bar(tcd::kQFull + qset), (n >> 1) & 1, abort, a.status))) break;
       auto chunk = [&](int t, int hf, int c) -> uint4 * {   // 8 bf16 at d = 64 hf + 8 c
@@ -524,20 +521,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
-        const int slot = c & 1;
         const float4 wl0 = __ldg(w4 + 2 * c), wl1 = __ldg(w4 + 2 * c + 1);
         const float4 wh0 = __ldg(w4 + 16 + 2 * c), wh1 = __ldg(w4 + 16 + 2 * c + 1);
         const float wl[8] = {wl0.x, wl0.y, wl0.z, wl0.w, wl1.x, wl1.y, wl1.z, wl1.w};
         const float wh[8] = {wh0.x, wh0.y, wh0.z, wh0.w, wh1.x, wh1.y, wh1.z, wh1.w};
         float cv[8], sv[8];
-        if (local) {
-          const float4 c0 = tb[4 * slot], c1 = tb[4 * slot + 1];
-          const float4 s0 = tb[4 * slot + 2], s1 = tb[4 * slot + 3];
-          cv[0] = c0.x; cv[1] = c0.y; cv[2] = c0.z; cv[3] = c0.w;
-          cv[4] = c1.x; cv[5] = c1.y; cv[6] = c1.z; cv[7] = c1.w;
-          sv[0] = s0.x; sv[1] = s0.y; sv[2] = s0.z; sv[3] = s0.w;
-          sv[4] = s1.x; sv[5] = s1.y; sv[6] = s1.z; sv[7] = s1.w;
-          if (c < 6) tab_load(c + 2, slot);
+        if (rope) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            cv[e] = tb[e].x;
+            sv[e] = tb[e].y;
+          }
+          if (c < 7) tab_load();   // the next chunk's angles, while this chunk is worked
         }
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
@@ -551,7 +546,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             xh[2 * e] = bf16_lo(hw[e]) * inv[t] * wh[2 * e];
             xh[2 * e + 1] = bf16_hi(hw[e]) * inv[t] * wh[2 * e + 1];
           }
-          if (local) {  // rotate-half: coordinate i < 64 pairs with i + 64
+          if (rope) {  // rotate-half: coordinate i < 64 pairs with i + 64
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
               const float a0 = xl[e], b0 = xh[e];

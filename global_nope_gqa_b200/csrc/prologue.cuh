@@ -95,7 +95,8 @@ struct PrologueArgs {
   uint16_t *v_cache;
   int64_t stride_seq, stride_head, slots;
   const int64_t *pos0;   // device [B]: position of token 0 of each sequence, or null (= 0)
-  float *rope_tab;       // local layers, or null: cos (64) then sin (64) of each token's angles
+  float *rope_tab;       // local layers, or null: (cos, sin) of each token's 64 angles,
+                         // angle-major [64][rows] float2 (rows: T, or B * T with rope_per_seq)
   int rope_per_seq;      // rope_tab is [B][T][128] (own positions) rather than [T][128] (0 .. T-1)
   int whole_seq;         // a sequence whose tokens do not all fit is not written at all
   int cache_fp8;         // the caches hold E4M3 codes of value / scale (one byte each)
@@ -249,9 +250,10 @@ __global__ void __launch_bounds__(128, 8) prologue_kernel(const PrologueArgs a) 
       reinterpret_cast<float *>(s_cs)[f] = c;
       reinterpret_cast<float *>(s_sn)[f] = s;
       if (a.rope_tab && (a.rope_per_seq || b == 0)) {
-        const size_t trow = (size_t)(a.rope_per_seq ? tok : i) * 128;
-        a.rope_tab[trow + f] = c;
-        a.rope_tab[trow + 64 + f] = s;
+        // angle-major: (cos, sin) of angle f at row f * rows + (the token's row)
+        const size_t rows = a.rope_per_seq ? (size_t)n_tok : (size_t)a.T;
+        reinterpret_cast<float2 *>(a.rope_tab)[(size_t)f * rows + (a.rope_per_seq ? tok : i)] =
+            make_float2(c, s);
       }
     }
     __syncthreads();
