@@ -792,14 +792,15 @@ def run_decode_case(args):
     torch.cuda.set_device(0)
     import global_nope_gqa_b200 as beam
     beam.lib()
-    if args.decode_case in ("multi8", "multi8_local"):
-        glob = args.decode_case == "multi8"
+    if args.decode_case in ("multi8", "multi8_local", "multi8_fp8"):
+        glob = args.decode_case != "multi8_local"
+        fp8 = args.decode_case == "multi8_fp8"
         kind, slots = (wl.GLOBAL, args.context) if glob else (wl.LOCAL, wl.WINDOW)
-        L = ChunkLayer(torch, beam, kind, 8, args.context - 8, slots, args.seed, "case")
+        L = ChunkLayer(torch, beam, kind, 8, args.context - 8, slots, args.seed, "case", fp8=fp8)
         sec = time_loop(torch, L.run, args.steps, args.warmup)
         assert int(L.status.item()) == 0
         print(json.dumps({"case": f"{'global' if glob else 'local'} chunk of 8 new tokens, B=1, "
-                                  f"context {args.context}",
+                                  f"context {args.context}{', FP8 E4M3 cache' if fp8 else ''}",
                           "ms": sec * 1e3, "GBps": L.bytes / sec / 1e9}), flush=True)
         return
     fp8 = args.decode_case == "fp8"
@@ -852,7 +853,7 @@ def main(argv=None):
     ap.add_argument("--layers", default="both", choices=["both", "global", "local"],
                     help="prefill layers per step (profiling cases; the headline step is both)")
     ap.add_argument("--batch", type=int, default=0, help="override B (profiling cases)")
-    ap.add_argument("--decode-case", choices=["bf16", "fp8", "multi8", "multi8_local"], default=None,
+    ap.add_argument("--decode-case", choices=["bf16", "fp8", "multi8", "multi8_local", "multi8_fp8"], default=None,
                     help="profiling case: time one global decode call at --context only")
     ap.add_argument("--context", type=int, default=wl.MAX_CONTEXT)
     args = ap.parse_args(argv)

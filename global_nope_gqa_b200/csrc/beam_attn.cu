@@ -49,7 +49,24 @@ int cuda_status(cudaError_t e, const char *what) {
 }
 
 
-// Per-device attributes: SM count and the dynamic shared-memory opt-ins.
+// A warp-specialised kernel redistributes its registers between roles (setmaxnreg); the
+// roles' shares must fit in what the CTA is launched with, or the increase never completes.
+// Checked against the compiled per-thread count once per device, before any launch.
+int check_register_pool(const void *kernel, int threads, int pool) {
+  cudaFuncAttributes fa;
+  int st = cuda_status(cudaFuncGetAttributes(&fa, kernel), "kernel attributes");
+  if (st) return st;
+  if ((int64_t)fa.numRegs * threads < pool) {
+    if (verbose())
+      std::fprintf(stderr, "beam_attn: %d registers x %d threads < register split %d\n", fa.numRegs,
+                   threads, pool);
+    return BEAM_ERR_UNSUPPORTED;
+  }
+  return BEAM_OK;
+}
+
+// Per-device attributes: SM count, the dynamic shared-memory opt-ins and the register
+// pools of the warp-specialised kernels.
 int device_info(DeviceInfo **out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BEAM_ERR_CUDA;
@@ -84,7 +101,11 @@ int device_info(DeviceInfo **out) {
                         prefill_tc_kernel<false, true>, prefill_tc_kernel<false, false>})
       if ((st = cuda_status(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  kTcSmemBytes),
-                            "prefill shared-memory opt-in")))
+                            "prefill shared-memory opt-in")) ||
+          (st = check_register_pool(reinterpret_cast<const void *>(kernel), kTcThreads, kTcRegPool)))
+        return st;
+    for (auto kernel : {decode_tc_kernel<false>, decode_tc_kernel<true>})
+      if ((st = check_register_pool(reinterpret_cast<const void *>(kernel), kDtThreads, kDtRegPool)))
         return st;
     d.ready = true;
   }
@@ -133,6 +154,24 @@ void fill_inv_freq(double (&f)[64], double theta) {
 }
 
 int launch_status() { return cuda_status(cudaGetLastError(), "kernel launch"); }
+
+// A launch with programmatic stream serialization: the kernel may start while the one before
+// it in the stream finishes; it calls pdl_wait() before it touches that kernel's results.
+template <typename... KArgs, typename... Args>
+int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+               Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_status(cudaLaunchKernelEx(&cfg, kernel, args...), "kernel launch");
+}
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link to libcuda).
 PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
@@ -431,7 +470,7 @@ size_t fp8_view_bytes(int32_t B, const beam_kv_layout_t *layout) {
 
 // Runs per sequence up to which the multi-token kernel merges them itself (the last CTA of
 // each (sequence, KV head)); beyond it a merge kernel spreads the work over many CTAs.
-constexpr int kFoldMaxSplits = 8;
+constexpr int kFoldMaxSplits = kFoldMaxSplitsDev;
 
 // partials o [B][8][n_mt][n_split_max][16][128] and (m, l), then the merge tickets [B][8]
 size_t multi_partial_bytes(int32_t B, const MultiPlan &m) {
@@ -663,8 +702,9 @@ int chunk_call(int kind, const beam_attn_params *p, int32_t B, int32_t T, const 
   pa.k_view = k_view;
   pa.v_view = v_view;
   if ((int64_t)B * T + pa.n_prep > INT32_MAX) return BEAM_ERR_UNSUPPORTED;
-  prologue_kernel<<<(unsigned)((int64_t)B * T + pa.n_prep), 128, 0, s>>>(pa);
-  if ((st = launch_status())) return st;
+  if ((st = launch_pdl(prologue_kernel, dim3((unsigned)((int64_t)B * T + pa.n_prep)), dim3(128), 0,
+                       s, pa)))
+    return st;
 
   // 2. attention of the new rows over the earlier and the new keys
   if (few) {
@@ -719,13 +759,10 @@ int chunk_call(int kind, const beam_attn_params *p, int32_t B, int32_t T, const 
       da.fault_stall = f != nullptr && std::strcmp(f, "prefill_wait_stall") == 0;
     }
     if (mp.n_split_max > 65535 || B > 65535) return BEAM_ERR_UNSUPPORTED;
-    if (widen_in_kernel)
-      decode_tc_kernel<true><<<dim3(mp.n_split_max, kHkv, B), DtCfg<true>::kThreads, kDtSmemBytes,
-                               s>>>(tk, tv, da);
-    else
-      decode_tc_kernel<false><<<dim3(mp.n_split_max, kHkv, B), DtCfg<false>::kThreads,
-                                kDtSmemBytes, s>>>(tk, tv, da);
-    if ((st = launch_status())) return st;
+    if ((st = launch_pdl(widen_in_kernel ? decode_tc_kernel<true> : decode_tc_kernel<false>,
+                         dim3(mp.n_split_max, kHkv, B), dim3(kDtThreads), kDtSmemBytes, s, tk, tv,
+                         da)))
+      return st;
     if (da.direct || da.fold) return BEAM_OK;
     MultiCombineArgs mc;
     mc.part_o = da.part_o;

@@ -152,6 +152,16 @@ __device__ __forceinline__ uint2 f32x8_to_e4m3(const float (&x)[8], float inv_sc
   return make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
 }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream serialization
+// may start while the kernel before it in the stream is still running; pdl_wait() returns
+// once that kernel has completed and its memory writes are visible (at once for a kernel
+// launched without the attribute).  pdl_trigger() lets the next kernel's CTAs be scheduled
+// as soon as every CTA of this one has issued it or exited.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+
 // 2^x on the special-function unit (flushes subnormal results to zero; 2^-inf = 0).
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;

@@ -61,6 +61,10 @@
 namespace beam {
 
 constexpr int kTcThreads = 512;
+// Register split (setmaxnreg) per 128 threads: warps 0-3 56 each, the two softmax warpgroups
+// 176, the Q-preparation warpgroup 104 -- exactly the 512 x 128 registers of the launch.
+constexpr int kTcRegPool = 128 * (56 + 176 + 176 + 104);
+static_assert(kTcRegPool <= kTcThreads * 128, "the split must fit the launch's registers");
 constexpr int kTcBM = 128;      // query rows per tile
 constexpr int kTcBN = 128;      // keys per block
 constexpr uint32_t kTcTileBytes = 128 * 128 * 2;   // 32 KiB: one 128 x 128 bf16 tile

@@ -187,6 +187,10 @@ __device__ __forceinline__ void load_weights8(const float *w, int l16, float (&o
 }
 
 __global__ void __launch_bounds__(128, 8) prologue_kernel(const PrologueArgs a) {
+  // the workspace and the caches may still be in use by the kernel before this one (the
+  // previous call on the stream); the attention kernel after this one waits for all of it
+  pdl_wait();
+  pdl_trigger();
   const int n_tok = (int)gridDim.x - a.n_prep;
   if ((int)blockIdx.x >= n_tok) {   // a chunk-preparation CTA (the whole CTA returns)
     chunk_prep_row(a.prep, (int)blockIdx.x - n_tok);
