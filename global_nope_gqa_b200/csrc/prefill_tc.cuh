@@ -598,19 +598,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int c = 0; c < 4; ++c) tc::tmem_ld32(t_s + 32 * c, sr[c]);
         tc::tmem_ld_wait();
         const int k0 = (w.kb_lo + j) * kTcBN;
-        // masked only where the block holds a key outside this row's range (a warp whose
-        // rows disagree takes the masking path)
-        if (k0 + kTcBN - 1 > hi_base || k0 < lo_base) {
-          // key k0 + i is visible to row r iff lo <= i <= hi
+        // masked only where the block holds a key outside this row's range.  Key k0 + i is
+        // visible to row r iff lo <= i <= hi; the window start and the causal edge move by
+        // one key per row, so in most 32-key chunks a warp's 32 rows agree: a chunk whose
+        // keys are all visible to every row of the warp is passed over.
+        if (__any_sync(0xffffffffu, k0 + kTcBN - 1 > hi_base || k0 < lo_base)) {
           const int hi = hi_base - k0;
           const int lo = lo_base - k0;
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
+          for (int c = 0; c < 4; ++c) {
+            const bool all_in = __all_sync(0xffffffffu, lo <= 32 * c && hi >= 32 * c + 31);
+            const bool all_out = __all_sync(0xffffffffu, hi < 32 * c || lo > 32 * c + 31);
+            if (!all_in) {   // (an all-invisible chunk takes an empty range)
+              const int lo_c = all_out ? 32 : lo - 32 * c, hi_c = hi - 32 * c;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int kk = c * 32 + i;
-              sr[c][i] = (kk >= lo && kk <= hi) ? sr[c][i] : 0xFF800000u;  // -inf
+              for (int i = 0; i < 32; ++i)
+                sr[c][i] = (i >= lo_c && i <= hi_c) ? sr[c][i] : 0xFF800000u;  // -inf
             }
+          }
         }
         // row max of the raw scores: eight independent chains of 3-input max
         float mc[8];
