@@ -251,8 +251,8 @@ BEAM_API int beam_attn_decode_fp8(int kind, const beam_attn_params *p, int32_t B
 
 /* Workspace beam_attn_prefill_chunk_fp8 needs (bytes): what
  * beam_prefill_chunk_workspace_bytes gives for the same shapes and, for a global
- * layer, a bf16 view of the cache (keys and values, two bytes for every element of
- * the FP8 layout, 4 * bytes_k in all) at the end of the workspace. */
+ * layer with T > 16, a bf16 view of the cache (keys and values, two bytes for every
+ * element of the FP8 layout, 4 * bytes_k in all) at the end of the workspace. */
 BEAM_API size_t beam_prefill_chunk_fp8_workspace_bytes(int kind, const beam_attn_params *p,
                                                        int32_t B, int32_t T,
                                                        const beam_kv_layout_t *layout);
@@ -261,12 +261,15 @@ BEAM_API size_t beam_prefill_chunk_fp8_workspace_bytes(int kind, const beam_attn
  * scale per cache tensor as for beam_attn_decode_fp8).  The chunk's new keys and
  * values are written as codes first; the queries then attend over every visible key
  * and value read back from the cache, the new ones included (the order the FP8
- * decode takes for one new token).  Cached codes are widened to bf16 (their
- * unscaled values, exact) in the workspace -- the ring rows a local chunk sees, or,
- * for a global layer, the rows before each sequence's pos0 in a bf16 view of the
- * cache -- and the tensor-core kernels of the bf16 path read them, with k_scale
- * folded into the score scale and v_scale into the output.  Positions, status,
- * capacity and the T <= 16 path as in beam_attn_prefill_chunk. */
+ * decode takes for one new token).  The codes are read as their unscaled values
+ * (exact), with k_scale folded into the score scale and v_scale into the output:
+ * a local chunk widens the ring rows it sees to bf16 in the workspace, and a global
+ * chunk of more than 16 tokens widens the rows before each sequence's pos0 into a
+ * bf16 view of the cache, both then read by the tensor-core kernels of the bf16
+ * path; a global chunk of at most 16 tokens reads the codes themselves (keys in
+ * E4M3 MMAs against a two-term E4M3 split of each query row, values widened to f16
+ * on chip).  Positions, status, capacity and the T <= 16 path as in
+ * beam_attn_prefill_chunk. */
 BEAM_API int beam_attn_prefill_chunk_fp8(int kind, const beam_attn_params *p, int32_t B, int32_t T,
                                          const void *q, const void *k, const void *v,
                                          const void *gate, const float *q_norm_w,
