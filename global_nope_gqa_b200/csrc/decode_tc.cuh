@@ -187,8 +187,10 @@ __global__ void __launch_bounds__(kDtThreads, 1)
   const bool local = a.kind == BEAM_LOCAL;
 
   // key coordinates of the sequence (see above); an out-of-range pos0 has set the status in
-  // the prologue and does nothing here (the whole CTA returns together)
-  const int64_t p0 = a.pos0[b];
+  // the prologue and does nothing here (the whole CTA returns together).  pos0 is read before
+  // pdl_wait() (the prologue does not write it; the kernels before the prologue have ended
+  // when this one starts) and through L2, past any stale copy in this SM's L1.
+  const int64_t p0 = __ldcg(a.pos0 + b);
   if (p0 < 0 || (!local && p0 + a.T > a.slots)) return;
   int64_t kq, lo_all;
   if (local) {
