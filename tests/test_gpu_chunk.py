@@ -243,3 +243,36 @@ def test_chunk_out_of_range_sequences_set_status_and_write_nothing(env):
         kh = host_bits(kc).reshape(2, 8, slots, 128)
         vh = host_bits(vc).reshape(2, 8, slots, 128)
         assert np.array_equal(kh[1], ci.k_cache[1]) and np.array_equal(vh[1], ci.v_cache[1])
+
+
+@pytest.mark.parametrize("kind,T", [(wl.LOCAL, 8), (wl.GLOBAL, 8), (wl.LOCAL, 300),
+                                    (wl.GLOBAL, 300)])
+def test_back_to_back_calls_sharing_one_workspace(env, kind, T):
+    """Three chunk calls issued on one stream with no synchronisation between them, all
+    with the same workspace: a call's prologue must not overwrite the workspace rows, RoPE
+    table or merge tickets that the previous call's attention kernel still reads (the
+    launches overlap under programmatic dependent launch).  Each output against the oracle."""
+    torch, beam, orc = env
+    params = beam.default_params()
+    slots = 512 if kind == wl.LOCAL else 4096
+    cases = [wl.chunk_inputs(kind, T, pos0, slots, 81 + n, layer=f"b2b{kind}{T}/{n}")
+             for n, pos0 in enumerate(([700, 3], [3000, 1200], [40, 2500]))]
+    layout = beam.beam_kv_layout(kind, params, 2, slots)
+    need = max(beam.beam_prefill_chunk_workspace_bytes(kind, params, 2, T, layout), 256)
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    outs = []
+    for ci in cases:
+        q, k, v, g = (dev(torch, x) for x in (ci.q, ci.k, ci.v, ci.gate))
+        kc = dev(torch, ci.k_cache).view(-1)
+        vc = dev(torch, ci.v_cache).view(-1)
+        out = torch.full((2, T, 48 * 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+        beam.beam_attn_prefill_chunk(kind, params, q, k, v, g, torch.from_numpy(ci.q_norm_w).cuda(),
+                                     torch.from_numpy(ci.k_norm_w).cuda(),
+                                     torch.from_numpy(ci.gate_bias).cuda(),
+                                     torch.from_numpy(ci.pos0).cuda(), out, kc, vc, layout,
+                                     workspace=ws)
+        outs.append((out, q, k, v, g, kc, vc))   # keep every buffer alive until the sync
+    torch.cuda.synchronize()
+    for n, (ci, o) in enumerate(zip(cases, outs)):
+        ref = oracle_chunk(orc, beam, ci, params)
+        assert_close(host_bits(o[0]).reshape(ref.shape), ref, f"back-to-back call {n}")
