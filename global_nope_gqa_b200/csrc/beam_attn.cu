@@ -947,23 +947,23 @@ int decode_call(int kind, const beam_attn_params *p, int32_t B, const void *q, c
     cfg.blockDim = dim3(kDecThreads);
     cfg.dynamicSmemBytes = fp8 ? kDec8Smem : kDecSmem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)n_split_max;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cuda_status(fp8 ? cudaLaunchKernelEx(&cfg, decode8_attn_kernel<true>, d8)
                            : cudaLaunchKernelEx(&cfg, decode_attn_kernel<true>, da),
                        "ring decode launch");
   }
 
-  if (fp8)
-    decode8_attn_kernel<false><<<grid, kDecThreads, kDec8Smem, s>>>(d8);
-  else
-    decode_attn_kernel<false><<<grid, kDecThreads, kDecSmem, s>>>(da);
-  if ((st = launch_status())) return st;
+  if ((st = fp8 ? launch_pdl(decode8_attn_kernel<false>, grid, dim3(kDecThreads), kDec8Smem, s, d8)
+                : launch_pdl(decode_attn_kernel<false>, grid, dim3(kDecThreads), kDecSmem, s, da)))
+    return st;
 
   CombineArgs ca;
   ca.part_o = w.part_o;
@@ -977,8 +977,7 @@ int decode_call(int kind, const beam_attn_params *p, int32_t B, const void *q, c
   ca.split = split;
   ca.n_split_max = n_split_max;
   ca.slots = layout->slots_per_seq;
-  decode_combine_kernel<<<dim3(kHq, B), kCombineThreads, 0, s>>>(ca);
-  return launch_status();
+  return launch_pdl(decode_combine_kernel, dim3(kHq, B), dim3(kCombineThreads), 0, s, ca);
 }
 
 }  // namespace

@@ -76,6 +76,10 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const DecodeAr
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ __align__(16) uint16_t q_prep[kGroup * kD];
   const int s_idx = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  // launched with programmatic serialization: wait for the kernel before (it may have written
+  // any of the inputs), then let the merge kernel after this one be scheduled
+  pdl_wait();
+  pdl_trigger();
   const int64_t t = a.pos[b];
   const int64_t n_vis = decode_visible(a, t);
   if (n_vis == 0) {   // a position outside the cache: nothing is written (a whole cluster
@@ -383,6 +387,7 @@ constexpr int kCombineThreads = 256;
 __global__ void __launch_bounds__(kCombineThreads) decode_combine_kernel(const CombineArgs a) {
   const int h = blockIdx.x, b = blockIdx.y;
   const int g = h / kGroup, hh = h - g * kGroup;
+  pdl_wait();   // the partials of the attention kernel before this one
   const int64_t t = a.pos[b];
   int64_t n_vis;
   if (t < 0) n_vis = 0;

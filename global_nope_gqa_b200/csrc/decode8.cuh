@@ -108,6 +108,9 @@ __global__ void __launch_bounds__(kDecThreads) decode8_attn_kernel(const Decode8
   __shared__ __align__(16) uint8_t q_hi[kGroup * kD];   // E4M3 codes of 16 q
   __shared__ __align__(16) uint8_t q_lo[kGroup * kD];   // E4M3 codes of 16 q - hi
   const int s_idx = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  // launched with programmatic serialization (see decode_attn_kernel)
+  pdl_wait();
+  pdl_trigger();
   const int64_t t = a.pos[b];
   const int64_t n_vis = decode_visible(a, t);
   if (n_vis == 0) {   // a position outside the cache: nothing is written
