@@ -29,6 +29,10 @@
  *     is a DEVICE pointer owned by the caller and must be 16-byte aligned;
  *   - parameter and layout structs are HOST pointers, read during the call only;
  *   - calls are asynchronous on `stream`, never synchronise and never allocate;
+ *   - stream order holds as usual: the decode and chunk calls launch their kernels
+ *     with programmatic stream serialization, so a kernel may be scheduled while
+ *     the one before it on the stream finishes, but it waits for that kernel to
+ *     complete before it reads or writes any caller buffer or workspace;
  *   - errors found on the host (bad kind, sizes, null or misaligned pointers, a
  *     workspace that is too small) return before any launch, writing nothing;
  *   - launch failures return BEAM_ERR_CUDA;
