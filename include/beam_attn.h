@@ -31,8 +31,10 @@
  *   - calls are asynchronous on `stream`, never synchronise and never allocate;
  *   - stream order holds as usual: the decode and chunk calls launch their kernels
  *     with programmatic stream serialization, so a kernel may be scheduled while
- *     the one before it on the stream finishes, but it waits for that kernel to
- *     complete before it reads or writes any caller buffer or workspace;
+ *     the one before it on the stream finishes; the first kernel of a call waits for
+ *     the kernel before it to complete before it touches any caller buffer or
+ *     workspace, and a later kernel of the call waits for the earlier ones before it
+ *     reads what they wrote;
  *   - errors found on the host (bad kind, sizes, null or misaligned pointers, a
  *     workspace that is too small) return before any launch, writing nothing;
  *   - launch failures return BEAM_ERR_CUDA;
