@@ -413,8 +413,7 @@ int beam_attn_prefill(int kind, const beam_attn_params *p, int32_t B, int32_t T,
   pa.window = p->window;
   pa.eps = p->rms_eps;
   fill_inv_freq(pa.inv_freq, p->rope_theta);
-  pa.n_tokens = (int)tok;
-  prologue_kernel<<<(unsigned)((tok + kProTok - 1) / kProTok), 128, 0, s>>>(pa);
+  prologue_kernel<<<(unsigned)tok, 128, 0, s>>>(pa);
   if ((st = launch_status())) return st;
 
   if ((st = encode_fn())) return st;
@@ -703,9 +702,7 @@ int chunk_call(int kind, const beam_attn_params *p, int32_t B, int32_t T, const 
   pa.k_view = k_view;
   pa.v_view = v_view;
   if ((int64_t)B * T + pa.n_prep > INT32_MAX) return BEAM_ERR_UNSUPPORTED;
-  pa.n_tokens = B * T;
-  if ((st = launch_pdl(prologue_kernel,
-                       dim3((unsigned)(((int64_t)B * T + kProTok - 1) / kProTok + pa.n_prep)), dim3(128), 0,
+  if ((st = launch_pdl(prologue_kernel, dim3((unsigned)((int64_t)B * T + pa.n_prep)), dim3(128), 0,
                        s, pa)))
     return st;
 
@@ -849,9 +846,7 @@ int beam_kv_append(int kind, const beam_attn_params *p, int32_t B, int32_t T, co
   pa.window = p->window;
   pa.eps = p->rms_eps;
   fill_inv_freq(pa.inv_freq, p->rope_theta);
-  pa.n_tokens = B * T;
-  prologue_kernel<<<(unsigned)(((size_t)B * T + kProTok - 1) / kProTok), 128, 0,
-                    reinterpret_cast<cudaStream_t>(stream)>>>(pa);
+  prologue_kernel<<<(unsigned)((size_t)B * T), 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(pa);
   return launch_status();
 }
 
@@ -1057,9 +1052,7 @@ int beam_kv_append_fp8(int kind, const beam_attn_params *p, int32_t B, int32_t T
   pa.window = p->window;
   pa.eps = p->rms_eps;
   fill_inv_freq(pa.inv_freq, p->rope_theta);
-  pa.n_tokens = B * T;
-  prologue_kernel<<<(unsigned)(((size_t)B * T + kProTok - 1) / kProTok), 128, 0,
-                    reinterpret_cast<cudaStream_t>(stream)>>>(pa);
+  prologue_kernel<<<(unsigned)((size_t)B * T), 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(pa);
   return launch_status();
 }
 

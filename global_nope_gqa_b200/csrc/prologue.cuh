@@ -83,10 +83,6 @@ __device__ __forceinline__ void chunk_prep_row(const ChunkPrepArgs &a, int cta) 
   }
 }
 
-// Tokens per prologue CTA: each CTA issues the K and V row loads of all its tokens before it
-// works on any, so that their latencies overlap instead of adding up one CTA wave after another.
-constexpr int kProTok = 4;
-
 struct PrologueArgs {
   const uint16_t *k;     // [tokens][8*128]
   const uint16_t *v;     // [tokens][8*128] (read only when a cache is written)
@@ -111,8 +107,7 @@ struct PrologueArgs {
   uint16_t *k_view, *v_view;
   int32_t *status;
   int T;                 // tokens per sequence in this call
-  int n_tokens;          // B * T: the token CTAs are the first ceil(n_tokens / kProTok)
-  // chunked prefill: n_prep extra CTAs after the token CTAs prepare the chunk (the
+  // chunked prefill: n_prep extra CTAs after the B * T token CTAs prepare the chunk (the
   // ring rows it still sees, or the value padding); ring_save: a token that takes the ring
   // slot of one of those rows copies the row out first
   ChunkPrepArgs prep;
@@ -191,84 +186,73 @@ __device__ __forceinline__ void load_weights8(const float *w, int l16, float (&o
   out[4] = x1.x; out[5] = x1.y; out[6] = x1.z; out[7] = x1.w;
 }
 
-__global__ void __launch_bounds__(128, 4) prologue_kernel(const PrologueArgs a) {
+__global__ void __launch_bounds__(128, 8) prologue_kernel(const PrologueArgs a) {
   // the workspace and the caches may still be in use by the kernel before this one (the
   // previous call on the stream); the attention kernel after this one waits for all of it
   pdl_wait();
   pdl_trigger();
-  const int n_tok = a.n_tokens;
-  const int n_tok_ctas = (n_tok + kProTok - 1) / kProTok;
-  if ((int)blockIdx.x >= n_tok_ctas) {   // a chunk-preparation CTA (the whole CTA returns)
-    chunk_prep_row(a.prep, (int)blockIdx.x - n_tok_ctas);
+  const int n_tok = (int)gridDim.x - a.n_prep;
+  if ((int)blockIdx.x >= n_tok) {   // a chunk-preparation CTA (the whole CTA returns)
+    chunk_prep_row(a.prep, (int)blockIdx.x - n_tok);
     return;
   }
+  const int tok = blockIdx.x;
+  const int b = tok / a.T;
+  const int i = tok - b * a.T;
+  if (a.tickets && i == 0 && threadIdx.x < kHkv) a.tickets[(size_t)b * kHkv + threadIdx.x] = 0u;
+  const int64_t t = (a.pos0 ? a.pos0[b] : 0) + i;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int half = lane >> 4, l16 = lane & 15;
   const bool local = a.kind == BEAM_LOCAL;
-  // Rows: half-warp w * 2 + half (0 .. 7) owns key head w * 2 + half and value head
-  // w * 2 + half of each of the CTA's kProTok tokens.
-  const int head = warp * 2 + half;
 
-  // Each token's cache target, then its K and V row loads: all issued before any is used,
-  // so that their latencies overlap one another and the angle computation below.
-  uint4 raw_k[kProTok], raw_v[kProTok];
-  int64_t tpos[kProTok];
-  unsigned wc_mask = 0u;   // bit u: token u writes the cache
-#pragma unroll
-  for (int u = 0; u < kProTok; ++u) {
-    const int64_t tok64 = (int64_t)blockIdx.x * kProTok + u;
-    raw_k[u] = raw_v[u] = make_uint4(0u, 0u, 0u, 0u);
-    tpos[u] = 0;
-    if (tok64 >= n_tok) continue;
-    const int tok = (int)tok64;
-    const int b = tok / a.T;
-    const int i = tok - b * a.T;
-    if (a.tickets && i == 0 && threadIdx.x < kHkv) a.tickets[(size_t)b * kHkv + threadIdx.x] = 0u;
-    const int64_t t = (a.pos0 ? a.pos0[b] : 0) + i;
-    tpos[u] = t;
-    bool write_cache = a.k_cache != nullptr;
-    if (write_cache && a.whole_seq) {
-      const int64_t p0 = a.pos0 ? a.pos0[b] : 0;
-      if (p0 < 0 || (!local && p0 + a.T > a.slots)) {
-        if (threadIdx.x == 0 && i == 0) set_status(a.status, BEAM_ERR_CAPACITY);
-        write_cache = false;
-      }
+  // Cache target of this token.
+  bool write_cache = a.k_cache != nullptr;
+  int64_t slot = 0;
+  if (write_cache && a.whole_seq) {
+    const int64_t p0 = a.pos0 ? a.pos0[b] : 0;
+    if (p0 < 0 || (!local && p0 + a.T > a.slots)) {
+      if (threadIdx.x == 0 && i == 0) set_status(a.status, BEAM_ERR_CAPACITY);
+      write_cache = false;
     }
-    if (write_cache) {
-      if (t < 0) {
-        if (threadIdx.x == 0) set_status(a.status, BEAM_ERR_CAPACITY);
-        write_cache = false;
-      } else if (local) {
-        write_cache = i >= a.T - a.window;  // earlier tokens of the call leave the window
-      } else if (t >= a.slots) {
+  }
+  if (write_cache) {
+    if (t < 0) {
+      set_status(a.status, BEAM_ERR_CAPACITY);
+      write_cache = false;
+    } else if (local) {
+      write_cache = i >= a.T - a.window;  // earlier tokens of the call leave the window
+      slot = t % a.window;
+    } else {
+      slot = t;
+      if (t >= a.slots) {
         if (threadIdx.x == 0) set_status(a.status, BEAM_ERR_CAPACITY);
         write_cache = false;
       }
     }
-    if (write_cache) wc_mask |= 1u << u;
-    const bool k_on = a.k_out != nullptr || write_cache;
-    const bool v_on = write_cache || a.v_out != nullptr;
-    const size_t src_off = (size_t)tok * (kHkv * kD) + head * kD + l16 * 8;
-    if (k_on) raw_k[u] = *reinterpret_cast<const uint4 *>(a.k + src_off);
-    if (v_on) raw_v[u] = *reinterpret_cast<const uint4 *>(a.v + src_off);
   }
 
-  // The tokens' 64 angles each, formed once per (token, angle) by the CTA's threads and
-  // shared through shared memory: every row of a token uses the same angles (and, for the
-  // table at positions 0 .. T-1, every sequence).
-  __shared__ float4 s_cs[kProTok][16], s_sn[kProTok][16];
+  // Rows: half-warp w * 2 + half (0 .. 7) owns key head w * 2 + half and value head
+  // w * 2 + half.  Their loads are issued first, so that their latency overlaps the angle
+  // computation below.
+  const int head = warp * 2 + half;
+  const bool k_on = a.k_out != nullptr || write_cache;
+  const bool v_on = write_cache || a.v_out != nullptr;
+  const size_t src_off = (size_t)tok * (kHkv * kD) + head * kD + l16 * 8;
+  const uint4 raw_k = k_on ? *reinterpret_cast<const uint4 *>(a.k + src_off) : make_uint4(0u, 0u, 0u, 0u);
+  const uint4 raw_v = v_on ? *reinterpret_cast<const uint4 *>(a.v + src_off) : make_uint4(0u, 0u, 0u, 0u);
+
+  // The token's 64 angles, one per thread of warps 0-1, shared through shared memory: every
+  // row of the token uses the same angles (and, for the table at positions 0 .. T-1,
+  // every sequence).
+  __shared__ float4 s_cs[16], s_sn[16];
+  float cs[8], sn[8];
   if (local) {
-    for (int item = threadIdx.x; item < kProTok * 64; item += blockDim.x) {
-      const int u = item >> 6, f = item & 63;
-      const int64_t tok64 = (int64_t)blockIdx.x * kProTok + u;
-      if (tok64 >= n_tok) continue;
-      const int tok = (int)tok64;
-      const int b = tok / a.T, i = tok - b * a.T;
+    if (threadIdx.x < 64) {
+      const int f = threadIdx.x;
       float c, s;
-      const int64_t tu = (a.pos0 ? a.pos0[b] : 0) + i;
-      rope_angle(a.inv_freq[f], tu < 0 ? 0 : tu, c, s);
-      reinterpret_cast<float *>(s_cs[u])[f] = c;
-      reinterpret_cast<float *>(s_sn[u])[f] = s;
+      rope_angle(a.inv_freq[f], t < 0 ? 0 : t, c, s);
+      reinterpret_cast<float *>(s_cs)[f] = c;
+      reinterpret_cast<float *>(s_sn)[f] = s;
       if (a.rope_tab && (a.rope_per_seq || b == 0)) {
         // angle-major: (cos, sin) of angle f at row f * rows + (the token's row)
         const size_t rows = a.rope_per_seq ? (size_t)n_tok : (size_t)a.T;
@@ -277,94 +261,78 @@ __global__ void __launch_bounds__(128, 4) prologue_kernel(const PrologueArgs a) 
       }
     }
     __syncthreads();
+    const int sub = l16 & 7;   // coordinates 8 l16 .. 8 l16 + 7 use angles 8 sub .. 8 sub + 7
+    const float4 c0 = s_cs[2 * sub], c1 = s_cs[2 * sub + 1];
+    const float4 s0 = s_sn[2 * sub], s1 = s_sn[2 * sub + 1];
+    cs[0] = c0.x; cs[1] = c0.y; cs[2] = c0.z; cs[3] = c0.w;
+    cs[4] = c1.x; cs[5] = c1.y; cs[6] = c1.z; cs[7] = c1.w;
+    sn[0] = s0.x; sn[1] = s0.y; sn[2] = s0.z; sn[3] = s0.w;
+    sn[4] = s1.x; sn[5] = s1.y; sn[6] = s1.z; sn[7] = s1.w;
   }
 
   float wk[8];
   load_weights8(a.kw, l16, wk);
-  const unsigned half_mask = 0xFFFFu << (half * 16);  // shuffles stay inside the half-warp
 
+  const unsigned half_mask = 0xFFFFu << (half * 16);  // shuffles stay inside the half-warp
 #pragma unroll
-  for (int u = 0; u < kProTok; ++u) {
-    const int64_t tok64 = (int64_t)blockIdx.x * kProTok + u;
-    if (tok64 >= n_tok) continue;
-    const int tok = (int)tok64;
-    const int b = tok / a.T;
-    const int i = tok - b * a.T;
-    const int64_t t = tpos[u];
-    const bool write_cache = (wc_mask >> u) & 1u;
-    const int64_t slot = local ? t % a.window : t;
-    const bool k_on = a.k_out != nullptr || write_cache;
-    const bool v_on = write_cache || a.v_out != nullptr;
-    float cs[8], sn[8];
-    if (local) {
-      const int sub = l16 & 7;   // coordinates 8 l16 .. 8 l16 + 7 use angles 8 sub .. 8 sub + 7
-      const float4 c0 = s_cs[u][2 * sub], c1 = s_cs[u][2 * sub + 1];
-      const float4 s0 = s_sn[u][2 * sub], s1 = s_sn[u][2 * sub + 1];
-      cs[0] = c0.x; cs[1] = c0.y; cs[2] = c0.z; cs[3] = c0.w;
-      cs[4] = c1.x; cs[5] = c1.y; cs[6] = c1.z; cs[7] = c1.w;
-      sn[0] = s0.x; sn[1] = s0.y; sn[2] = s0.z; sn[3] = s0.w;
-      sn[4] = s1.x; sn[5] = s1.y; sn[6] = s1.z; sn[7] = s1.w;
+  for (int kv = 0; kv < 2; ++kv) {
+    const bool is_k = kv == 0;
+    if (!(is_k ? k_on : v_on)) continue;   // the same for the whole CTA
+    const uint4 raw = is_k ? raw_k : raw_v;
+    float x[8];
+    if (!is_k) {
+      x[0] = bf16_lo(raw.x); x[1] = bf16_hi(raw.x); x[2] = bf16_lo(raw.y); x[3] = bf16_hi(raw.y);
+      x[4] = bf16_lo(raw.z); x[5] = bf16_hi(raw.z); x[6] = bf16_lo(raw.w); x[7] = bf16_hi(raw.w);
+    } else {
+      norm_rope_f32(raw, wk, local, cs, sn, l16, half_mask, a.eps, x);
     }
-#pragma unroll
-    for (int kv = 0; kv < 2; ++kv) {
-      const bool is_k = kv == 0;
-      if (!(is_k ? k_on : v_on)) continue;   // the same for the whole CTA
-      const uint4 raw = is_k ? raw_k[u] : raw_v[u];
-      float x[8];
-      if (!is_k) {
-        x[0] = bf16_lo(raw.x); x[1] = bf16_hi(raw.x); x[2] = bf16_lo(raw.y); x[3] = bf16_hi(raw.y);
-        x[4] = bf16_lo(raw.z); x[5] = bf16_hi(raw.z); x[6] = bf16_lo(raw.w); x[7] = bf16_hi(raw.w);
-      } else {
-        norm_rope_f32(raw, wk, local, cs, sn, l16, half_mask, a.eps, x);
-      }
-      uint4 res = raw;
-      if (is_k) {
-        res.x = pack_bf16(x[0], x[1]); res.y = pack_bf16(x[2], x[3]);
-        res.z = pack_bf16(x[4], x[5]); res.w = pack_bf16(x[6], x[7]);
-      }
-      uint16_t *dst = is_k ? a.k_out : a.v_out;
-      // an FP8 cache stores codes of the fp32 rows, not of their bf16 rounding; the attention
-      // of an FP8 chunk reads the codes' unscaled values (its scales apply in the kernel)
-      uint2 codes = make_uint2(0u, 0u);
-      if (a.cache_fp8 && (write_cache || dst)) codes = f32x8_to_e4m3_div(x, is_k ? a.k_scale : a.v_scale);
-      const uint4 att = a.cache_fp8 ? e4m3x8_to_bf16x8(codes) : res;
-      if (dst) {
-        const size_t orow = (size_t)b * (a.out_rows ? a.out_rows : a.T) + a.out_row0 + i;
-        *reinterpret_cast<uint4 *>(dst + orow * (kHkv * kD) + head * kD + l16 * 8) = att;
-      }
-      if (write_cache) {
-        const size_t off = (size_t)b * a.stride_seq + (size_t)head * a.stride_head +
-                           (size_t)slot * kD + l16 * 8;
-        if (a.cache_fp8) {
-          uint8_t *cache = reinterpret_cast<uint8_t *>(is_k ? a.k_cache : a.v_cache);
-          const int r = a.ring_save ? i % a.window : 0;
-          if (r >= 1) {   // as below, for a ring of codes: its old row's values go to the workspace
-            const int64_t q = (t - i) + r - a.window;
-            const uint4 old = q >= 0 ? e4m3x8_to_bf16x8(*reinterpret_cast<const uint2 *>(cache + off))
-                                     : make_uint4(0u, 0u, 0u, 0u);
-            uint16_t *ext = is_k ? a.k_out : a.v_out;
-            *reinterpret_cast<uint4 *>(ext + ((size_t)b * a.out_rows + r - 1) * (kHkv * kD) +
-                                       head * kD + l16 * 8) = old;
-          }
-          *reinterpret_cast<uint2 *>(cache + off) = codes;
-          uint16_t *view = is_k ? a.k_view : a.v_view;
-          if (view) *reinterpret_cast<uint4 *>(view + off) = att;
-        } else {
-          uint16_t *cache = is_k ? a.k_cache : a.v_cache;
-          const int r = a.ring_save ? i % a.window : 0;
-          if (r >= 1) {
-            // before this call the slot held position q = pos0 + r - window, row r - 1 of the
-            // earlier keys the chunk still sees: save it (zeros before position 0) before
-            // overwriting it
-            const int64_t q = (t - i) + r - a.window;
-            const uint4 old = q >= 0 ? *reinterpret_cast<const uint4 *>(cache + off)
-                                     : make_uint4(0u, 0u, 0u, 0u);
-            uint16_t *ext = is_k ? a.k_out : a.v_out;
-            *reinterpret_cast<uint4 *>(ext + ((size_t)b * a.out_rows + r - 1) * (kHkv * kD) +
-                                       head * kD + l16 * 8) = old;
-          }
-          *reinterpret_cast<uint4 *>(cache + off) = res;
+    uint4 res = raw;
+    if (is_k) {
+      res.x = pack_bf16(x[0], x[1]); res.y = pack_bf16(x[2], x[3]);
+      res.z = pack_bf16(x[4], x[5]); res.w = pack_bf16(x[6], x[7]);
+    }
+    uint16_t *dst = is_k ? a.k_out : a.v_out;
+    // an FP8 cache stores codes of the fp32 rows, not of their bf16 rounding; the attention
+    // of an FP8 chunk reads the codes' unscaled values (its scales apply in the kernel)
+    uint2 codes = make_uint2(0u, 0u);
+    if (a.cache_fp8 && (write_cache || dst)) codes = f32x8_to_e4m3_div(x, is_k ? a.k_scale : a.v_scale);
+    const uint4 att = a.cache_fp8 ? e4m3x8_to_bf16x8(codes) : res;
+    if (dst) {
+      const size_t orow = (size_t)b * (a.out_rows ? a.out_rows : a.T) + a.out_row0 + i;
+      *reinterpret_cast<uint4 *>(dst + orow * (kHkv * kD) + head * kD + l16 * 8) = att;
+    }
+    if (write_cache) {
+      const size_t off = (size_t)b * a.stride_seq + (size_t)head * a.stride_head +
+                         (size_t)slot * kD + l16 * 8;
+      if (a.cache_fp8) {
+        uint8_t *cache = reinterpret_cast<uint8_t *>(is_k ? a.k_cache : a.v_cache);
+        const int r = a.ring_save ? i % a.window : 0;
+        if (r >= 1) {   // as below, for a ring of codes: its old row's values go to the workspace
+          const int64_t q = (t - i) + r - a.window;
+          const uint4 old = q >= 0 ? e4m3x8_to_bf16x8(*reinterpret_cast<const uint2 *>(cache + off))
+                                   : make_uint4(0u, 0u, 0u, 0u);
+          uint16_t *ext = is_k ? a.k_out : a.v_out;
+          *reinterpret_cast<uint4 *>(ext + ((size_t)b * a.out_rows + r - 1) * (kHkv * kD) +
+                                     head * kD + l16 * 8) = old;
         }
+        *reinterpret_cast<uint2 *>(cache + off) = codes;
+        uint16_t *view = is_k ? a.k_view : a.v_view;
+        if (view) *reinterpret_cast<uint4 *>(view + off) = att;
+      } else {
+        uint16_t *cache = is_k ? a.k_cache : a.v_cache;
+        const int r = a.ring_save ? i % a.window : 0;
+        if (r >= 1) {
+          // before this call the slot held position q = pos0 + r - window, row r - 1 of the
+          // earlier keys the chunk still sees: save it (zeros before position 0) before
+          // overwriting it
+          const int64_t q = (t - i) + r - a.window;
+          const uint4 old = q >= 0 ? *reinterpret_cast<const uint4 *>(cache + off)
+                                   : make_uint4(0u, 0u, 0u, 0u);
+          uint16_t *ext = is_k ? a.k_out : a.v_out;
+          *reinterpret_cast<uint4 *>(ext + ((size_t)b * a.out_rows + r - 1) * (kHkv * kD) +
+                                     head * kD + l16 * 8) = old;
+        }
+        *reinterpret_cast<uint4 *>(cache + off) = res;
       }
     }
   }
